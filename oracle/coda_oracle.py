@@ -1,0 +1,325 @@
+"""fp64 CPU oracle for the CODA GEMM + epilogue hot path.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its
+``cpu_baseline`` leg and its ``--impl reference`` arm) may use it.  It shares
+no code, constants or helpers with the CUDA library; it widens bf16 bit
+patterns to fp64 itself and computes everything in fp64 with numpy.  The one
+library primitive it uses as a step is the dense fp64 matrix product
+(``numpy.matmul``); there is no blocking, fusion or reordering beyond what
+each definition states.
+
+Source: KuCoin news flash "CODA: new research optimizes transformer training
+with GEMM epilogue programming" (three translations of one article).  Section
+names below are that article's:
+
+* "CODA: the secret in the epilogue" - the GEMM-RMSNorm-GEMM pattern (matmul,
+  residual add, RMS normalisation, second matmul); the per-row scale r of the
+  RMS normalisation commutes with the following matmul, so it can be applied
+  at the end of the second GEMM; the first GEMM then only emits a partial RMS
+  which a light reduction kernel combines.  The same re-parameterisation
+  covers SwiGLU, RoPE, cross-entropy and the backward pass, and a theorem
+  states that a block-local forward epilogue gives a block-local backward.
+* "Five kinds of building blocks" - elementwise transform (residual add,
+  activation), vector load (RMSNorm weight broadcast), matrix-block
+  load/store (saving activations for the backward), chunk reduction (local
+  RMS, chunk log-sum-exp) and stateful transform (running max and sum-exp of
+  online normalisation).
+
+Two families of functions live here:
+
+1. The unfused definitions (``*_unfused``): what the transformer block
+   computes, written out plainly.  These are what the method must reproduce.
+2. The re-parameterised steps, one per library call (``gemm_res_partialrms``,
+   ``rms_reduce``, ``gemm_rowscale``, ``gemm_swiglu``, ``lmhead_ce``,
+   ``gemm_rowscale_bwd``, ``rms_reduce_bwd``, ``gemm_res_partialrms_bwd``), in
+   fp64.  In exact arithmetic the composition of the steps equals the unfused
+   definition; the pins in ``tests/test_oracle_pins.py`` check that, and pin
+   the unfused definitions to closed forms, brute force and finite differences.
+
+Readings where the article is silent (each listed in the design notes):
+eps sits inside the square root; the mean of h^2 is over all N columns;
+partials are sums of squares (not RMS values) so they add; gamma is applied in
+the first GEMM's epilogue (hg = gamma * h); SwiGLU is silu(gate) * up with the
+gate in the first half of the fused gate/up columns and r applied before silu;
+cross-entropy uses the natural log and the mean over all tokens.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+# ---------------------------------------------------------------------------
+# bf16 bit patterns -> fp64 (own widening: a bf16 is the top half of an fp32)
+# ---------------------------------------------------------------------------
+
+def bf16_to_f64(bits) -> np.ndarray:
+    """Widen bf16 bit patterns (uint16 array) to fp64 exactly."""
+    b = np.ascontiguousarray(np.asarray(bits, dtype=np.uint16))
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def as_f64(a) -> np.ndarray:
+    """Accept either bf16 bit patterns (uint16) or real arrays; return fp64."""
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return bf16_to_f64(a)
+    return a.astype(np.float64)
+
+
+def matmul(A, B) -> np.ndarray:
+    """Dense fp64 product A @ B (library primitive)."""
+    return np.matmul(as_f64(A), as_f64(B))
+
+
+def silu(v: np.ndarray) -> np.ndarray:
+    """silu(v) = v / (1 + exp(-v)), written to stay finite for large |v|."""
+    v = np.asarray(v, dtype=np.float64)
+    out = np.empty_like(v)
+    pos = v >= 0
+    out[pos] = v[pos] / (1.0 + np.exp(-v[pos]))
+    e = np.exp(v[~pos])
+    out[~pos] = v[~pos] * e / (1.0 + e)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# 1. Unfused definitions
+# ---------------------------------------------------------------------------
+
+def rmsnorm_block_unfused(x, res, W1, W2, gamma, eps: float) -> dict:
+    """GEMM-RMSNorm-GEMM as three separate operators ("CODA: the secret in the
+    epilogue"): h = x W1 + res; ms_i = mean_j h_ij^2; r_i = 1/sqrt(ms_i + eps);
+    y = gamma * h * r; out = y W2."""
+    h = matmul(x, W1) + as_f64(res)
+    N = h.shape[1]
+    ms = (h * h).sum(axis=1) / N
+    r = 1.0 / np.sqrt(ms + eps)
+    y = as_f64(gamma)[None, :] * h * r[:, None]
+    out = matmul(y, W2)
+    return {"h": h, "ms": ms, "r": r, "y": y, "out": out}
+
+
+def swiglu_down_unfused(y, W_gu, W_down, res) -> dict:
+    """SwiGLU MLP tail after the norm: gate = y W_g, up = y W_u (W_g the first
+    half of the fused gate/up columns, W_u the second), a = silu(gate) * up,
+    h2 = a W_down + res ("CODA: the secret in the epilogue" lists SwiGLU among
+    the operations that the same re-parameterisation covers)."""
+    gu = matmul(y, W_gu)
+    F = gu.shape[1] // 2
+    gate, up = gu[:, :F], gu[:, F:]
+    a = silu(gate) * up
+    h2 = matmul(a, W_down) + as_f64(res)
+    return {"gate": gate, "up": up, "a": a, "h2": h2}
+
+
+def cross_entropy_unfused(H, W, labels) -> dict:
+    """Softmax cross-entropy over the vocabulary with materialised logits:
+    z = H W; lse_i = log sum_j exp(z_ij); loss_i = lse_i - z_i,label; mean over
+    tokens.  A label outside [0, V) gives a NaN loss for that token."""
+    z = matmul(H, W)
+    V = z.shape[1]
+    m = z.max(axis=1)
+    lse = m + np.log(np.exp(z - m[:, None]).sum(axis=1))
+    lab = np.asarray(labels, dtype=np.int64)
+    ok = (lab >= 0) & (lab < V)
+    zl = np.full(z.shape[0], np.nan)
+    idx = np.nonzero(ok)[0]
+    zl[idx] = z[idx, lab[idx]]
+    loss = lse - zl
+    return {"z": z, "lse": lse, "loss": loss, "mean": loss.sum() / loss.shape[0]}
+
+
+def rmsnorm_block_backward_unfused(x, res, W1, W2, gamma, eps: float, dOut) -> dict:
+    """Backward of out = (gamma * h * r) W2 with h = x W1 + res, by the chain
+    rule on the unfused definition, for the loss L = sum(dOut * out):
+
+    dy = dOut W2^T;  dW2 = y^T dOut;  dgamma_j = sum_i dy_ij h_ij r_i;
+    dh_ij = r_i gamma_j dy_ij - (r_i^3 / N) h_ij sum_k dy_ik gamma_k h_ik;
+    dres = dh;  dx = dh W1^T;  dW1 = x^T dh.
+    """
+    f = rmsnorm_block_unfused(x, res, W1, W2, gamma, eps)
+    h, r, y = f["h"], f["r"], f["y"]
+    g = as_f64(gamma)
+    dO = as_f64(dOut)
+    N = h.shape[1]
+    dy = matmul(dO, as_f64(W2).T)
+    dW2 = matmul(y.T, dO)
+    dgamma = (dy * h * r[:, None]).sum(axis=0)
+    c = (dy * g[None, :] * h).sum(axis=1)
+    dh = r[:, None] * g[None, :] * dy - (r ** 3 / N)[:, None] * h * c[:, None]
+    dx = matmul(dh, as_f64(W1).T)
+    dW1 = matmul(as_f64(x).T, dh)
+    return {"dy": dy, "dW2": dW2, "dgamma": dgamma, "dh": dh, "dres": dh.copy(),
+            "dx": dx, "dW1": dW1, "c": c, **f}
+
+
+# ---------------------------------------------------------------------------
+# 2. Re-parameterised steps (one per library call), fp64
+# ---------------------------------------------------------------------------
+
+def n_col_tiles(N: int, tile_cols: int) -> int:
+    return -(-N // tile_cols)
+
+
+def gemm_res_partialrms(x, W, res, gamma, tile_cols: int) -> dict:
+    """First GEMM with its epilogue ("CODA: the secret in the epilogue": the
+    first GEMM only computes a partial RMS; "Five kinds of building blocks":
+    residual add is an elementwise transform, gamma a broadcast vector load,
+    the local RMS a chunk reduction).
+
+    h = x W + res (res may be None);  hg = gamma * h (gamma None -> no hg);
+    partial[t, i] = sum over columns j of tile t (width tile_cols) of h_ij^2.
+    """
+    h = matmul(x, W)
+    if res is not None:
+        h = h + as_f64(res)
+    M, N = h.shape
+    T = n_col_tiles(N, tile_cols)
+    partial = np.zeros((T, M))
+    for t in range(T):
+        blk = h[:, t * tile_cols:(t + 1) * tile_cols]
+        partial[t] = (blk * blk).sum(axis=1)
+    hg = None if gamma is None else as_f64(gamma)[None, :] * h
+    return {"h": h, "hg": hg, "partial": partial}
+
+
+def rms_reduce(partial, N: int, eps: float) -> np.ndarray:
+    """The light reduction kernel: r_i = 1 / sqrt(sum_t partial[t, i] / N + eps)."""
+    p = np.asarray(partial, dtype=np.float64)
+    return 1.0 / np.sqrt(p.sum(axis=0) / N + eps)
+
+
+def gemm_rowscale(A, W, r) -> np.ndarray:
+    """Second GEMM with r applied in its epilogue: out_ij = r_i (A W)_ij.
+    r commutes with the matmul because it is one scalar per row."""
+    acc = matmul(A, W)
+    if r is None:
+        return acc
+    return np.asarray(r, dtype=np.float64)[:, None] * acc
+
+
+def gemm_swiglu(A, W_gu, r) -> dict:
+    """Gate/up GEMM with SwiGLU in its epilogue: g = r * (A W_g), u = r * (A W_u),
+    act = silu(g) * u.  W_g is the first half of W_gu's columns."""
+    acc = matmul(A, W_gu)
+    if r is not None:
+        acc = np.asarray(r, dtype=np.float64)[:, None] * acc
+    F = acc.shape[1] // 2
+    g, u = acc[:, :F], acc[:, F:]
+    return {"gate": g, "up": u, "act": silu(g) * u}
+
+
+def lmhead_ce(H, W, labels, r=None, chunk_cols: int = 256) -> dict:
+    """LM-head cross-entropy as chunk log-sum-exp with an online running max
+    and sum-exp ("Five kinds of building blocks": chunk reduction and stateful
+    transform).  Logits z = r * (H W) (r optional) are visited in column chunks
+    of width ``chunk_cols``; per token the state (m, s) is updated as
+    m' = max(m, max_chunk z), s' = s exp(m - m') + sum_chunk exp(z - m').
+    lse = m + log s; loss = lse - z_label; mean over tokens.
+    """
+    z = matmul(H, W)
+    if r is not None:
+        z = np.asarray(r, dtype=np.float64)[:, None] * z
+    M, V = z.shape
+    m = np.full(M, -np.inf)
+    s = np.zeros(M)
+    for c0 in range(0, V, chunk_cols):
+        blk = z[:, c0:c0 + chunk_cols]
+        m_new = np.maximum(m, blk.max(axis=1))
+        s = s * np.exp(m - m_new) + np.exp(blk - m_new[:, None]).sum(axis=1)
+        m = m_new
+    lse = m + np.log(s)
+    lab = np.asarray(labels, dtype=np.int64)
+    ok = (lab >= 0) & (lab < V)
+    zl = np.full(M, np.nan)
+    idx = np.nonzero(ok)[0]
+    zl[idx] = z[idx, lab[idx]]
+    loss = lse - zl
+    return {"lse": lse, "loss": loss, "mean": loss.sum() / M}
+
+
+def gemm_rowscale_bwd(dOut, hg, W2, r, tile_cols: int) -> dict:
+    """Backward of out = r * (hg W2), block-local form.
+
+    P = dOut W2^T (the gradient of y = r * hg); its epilogue forms
+    d_hg = r * P, y = r * hg and the chunk reduction
+    pdr[t, i] = sum over columns j of tile t of hg_ij P_ij;
+    the weight gradient is dW2 = y^T dOut.
+    """
+    P = matmul(dOut, as_f64(W2).T)
+    hg = as_f64(hg)
+    rr = np.asarray(r, dtype=np.float64)[:, None]
+    M, N = P.shape
+    T = n_col_tiles(N, tile_cols)
+    pdr = np.zeros((T, M))
+    for t in range(T):
+        sl = slice(t * tile_cols, (t + 1) * tile_cols)
+        pdr[t] = (hg[:, sl] * P[:, sl]).sum(axis=1)
+    y = rr * hg
+    return {"P": P, "d_hg": rr * P, "y": y, "pdr": pdr, "dW2": matmul(y.T, dOut)}
+
+
+def rms_reduce_bwd(pdr, r, d_hg, h, gamma) -> dict:
+    """Row reduction of the RMSNorm backward: dr_i = sum_t pdr[t, i];
+    coef_i = -r_i^3 dr_i / N; dh = gamma * d_hg + coef * h; dgamma_j = sum_i d_hg_ij h_ij."""
+    d_hg = as_f64(d_hg)
+    h = as_f64(h)
+    N = h.shape[1]
+    rr = np.asarray(r, dtype=np.float64)
+    dr = np.asarray(pdr, dtype=np.float64).sum(axis=0)
+    coef = -rr ** 3 * dr / N
+    dh = as_f64(gamma)[None, :] * d_hg + coef[:, None] * h
+    dgamma = (d_hg * h).sum(axis=0)
+    return {"dh": dh, "dgamma": dgamma, "dr": dr}
+
+
+def gemm_res_partialrms_bwd(dh, x, W1) -> dict:
+    """Backward of h = x W1 + res: dx = dh W1^T, dW1 = x^T dh, dres = dh."""
+    dh = as_f64(dh)
+    return {"dx": matmul(dh, as_f64(W1).T), "dW1": matmul(as_f64(x).T, dh), "dres": dh}
+
+
+# ---------------------------------------------------------------------------
+# Compositions of the steps (what the library's call sequence computes)
+# ---------------------------------------------------------------------------
+
+def rmsnorm_block_reparam(x, res, W1, W2, gamma, eps: float, tile_cols: int = 256) -> dict:
+    """The re-parameterised block: partials from GEMM1's epilogue, r from the
+    light reduction, r applied in GEMM2's epilogue on hg = gamma * h."""
+    a = gemm_res_partialrms(x, W1, res, gamma, tile_cols)
+    N = a["h"].shape[1]
+    r = rms_reduce(a["partial"], N, eps)
+    out = gemm_rowscale(a["hg"], W2, r)
+    return {"h": a["h"], "hg": a["hg"], "partial": a["partial"], "r": r, "out": out}
+
+
+def rmsnorm_block_backward_reparam(x, res, W1, W2, gamma, eps: float, dOut,
+                                   tile_cols: int = 256) -> dict:
+    """Backward through the block-local steps (fp64): rowscale backward, row
+    reduction backward, first-GEMM backward."""
+    f = rmsnorm_block_reparam(x, res, W1, W2, gamma, eps, tile_cols)
+    b1 = gemm_rowscale_bwd(dOut, f["hg"], W2, f["r"], tile_cols)
+    b2 = rms_reduce_bwd(b1["pdr"], f["r"], b1["d_hg"], f["h"], gamma)
+    b3 = gemm_res_partialrms_bwd(b2["dh"], x, W1)
+    return {"dW2": b1["dW2"], "dgamma": b2["dgamma"], "dh": b2["dh"], "dres": b3["dres"],
+            "dx": b3["dx"], "dW1": b3["dW1"], "pdr": b1["pdr"], "d_hg": b1["d_hg"],
+            "y": b1["y"], **{k: f[k] for k in ("h", "hg", "r")}}
+
+
+# ---------------------------------------------------------------------------
+# Row-sampled helpers for full-size checks (forward is row-independent)
+# ---------------------------------------------------------------------------
+
+def rmsnorm_block_rows(x_rows, res_rows, W1, W2, gamma, eps: float) -> dict:
+    """Unfused block forward on a subset of token rows (rows are independent)."""
+    return rmsnorm_block_unfused(x_rows, res_rows, W1, W2, gamma, eps)
+
+
+def tolerance_ok(got, ref, rel: float = 2e-2) -> tuple[bool, float, float]:
+    """Acceptance bar: max|got - ref| <= rel * rms(ref).  Returns (ok, maxerr, rms)."""
+    g = np.asarray(got, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    err = float(np.max(np.abs(g - r))) if r.size else 0.0
+    rms = float(np.sqrt(np.mean(r * r))) if r.size else 0.0
+    return (err <= rel * rms) if r.size else True, err, rms
