@@ -1,0 +1,366 @@
+"""Thin Python binding of libcoda.so (the C ABI declared in include/coda.h).
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+PyTorch provides device memory and the current stream.  There is no fallback:
+if the shared library is missing or the device is not a B200, the calls raise.
+
+Names follow the C ABI without the ``coda_`` prefix.  bf16 tensors are passed
+as their bit patterns (the C ABI takes ``uint16_t*``), fp32 as ``float*``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcoda.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "coda.h")
+
+CODA_OK = 0
+STATUS_NAMES = {
+    0: "CODA_OK", 1: "CODA_ERR_NULL", 2: "CODA_ERR_SHAPE", 3: "CODA_ERR_ALIGN",
+    4: "CODA_ERR_WORKSPACE", 5: "CODA_ERR_DEVICE", 6: "CODA_ERR_LAUNCH",
+    7: "CODA_ERR_DEVICE_TIMEOUT", 8: "CODA_ERR_INTERNAL",
+}
+
+
+class CodaError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {msg} (status {status})")
+        self.status = status
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+_ST = ctypes.c_int
+
+_SIGS = {
+    "coda_status_string": (ctypes.c_char_p, [_ST]),
+    "coda_version": (ctypes.c_int, []),
+    "coda_partial_tile_width": (_I64, []),
+    "coda_partial_cols": (_I64, [_I64]),
+    "coda_set_wait_limit_ns": (_ST, [_I64]),
+    "coda_poll_status": (_ST, [_P]),
+    "coda_gemm_res_partialrms": (_ST, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "coda_rms_reduce": (_ST, [_P, _I64, _I64, _I64, _F, _P, _P]),
+    "coda_gemm_rowscale": (_ST, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "coda_gemm_swiglu": (_ST, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "coda_lmhead_ce_workspace_size": (_SZ, [_I64, _I64]),
+    "coda_lmhead_ce": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _P]),
+    "coda_gemm_rowscale_bwd_workspace_size": (_SZ, [_I64, _I64]),
+    "coda_gemm_rowscale_bwd": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _P]),
+    "coda_rms_reduce_bwd_workspace_size": (_SZ, [_I64, _I64]),
+    "coda_rms_reduce_bwd": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _P]),
+    "coda_gemm_res_partialrms_bwd": (_ST, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "coda_unfused_add": (_ST, [_P, _P, _P, _I64, _P]),
+    "coda_unfused_rmsnorm": (_ST, [_P, _P, _F, _P, _P, _I64, _I64, _P]),
+    "coda_selftest_bounded_wait": (_ST, [_I64, _P, _P]),
+}
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libcoda.so from the package directory (raises if it is not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"libcoda.so not found at {LIB_PATH}; build it with "
+            "`python -m gemm_epilogue_transformer_02_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, status: int):
+    if status != CODA_OK:
+        lib = load_library()
+        raise CodaError(fn, status, lib.coda_status_string(status).decode())
+
+
+def _call(name: str, *args):
+    lib = load_library()
+    st = getattr(lib, name)(*args)
+    _check(name, st)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, dtype, name, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+def _empty(shape, dtype, like):
+    return torch.empty(shape, dtype=dtype, device=like.device)
+
+
+BF16 = torch.bfloat16
+F32 = torch.float32
+
+# ------------------------------------------------------------------ basics
+
+
+def version() -> int:
+    return load_library().coda_version()
+
+
+def partial_tile_width() -> int:
+    return int(load_library().coda_partial_tile_width())
+
+
+def partial_cols(N: int) -> int:
+    return int(load_library().coda_partial_cols(N))
+
+
+def set_wait_limit_ns(ns: int):
+    _call("coda_set_wait_limit_ns", int(ns))
+
+
+def poll_status():
+    """Synchronise the current stream and raise if a kernel recorded a timeout."""
+    _call("coda_poll_status", _stream())
+
+
+# ----------------------------------------------------------------- forward
+
+
+def gemm_res_partialrms(x, W, res=None, gamma=None, *, h=True, hg=True, partial=True,
+                        h_out=None, hg_out=None, partial_out=None):
+    """h = x W + res; hg = gamma * h; partial[t, i] = sum_{j in tile t} h_ij^2.
+    Returns (h, hg, partial); entries not requested are None."""
+    M, K = x.shape
+    N = W.shape[1]
+    _need(x, BF16, "x")
+    _need(W, BF16, "W", (K, N))
+    if res is not None:
+        _need(res, BF16, "res", (M, N))
+    if gamma is not None:
+        _need(gamma, BF16, "gamma", (N,))
+    if h and h_out is None:
+        h_out = _empty((M, N), BF16, x)
+    if hg and hg_out is None:
+        hg_out = _empty((M, N), BF16, x)
+    if partial and partial_out is None:
+        partial_out = _empty((partial_cols(N), M), F32, x)
+    _call("coda_gemm_res_partialrms", _ptr(x), _ptr(W), _ptr(res), _ptr(gamma),
+          _ptr(h_out if h else None), _ptr(hg_out if hg else None),
+          _ptr(partial_out if partial else None), M, N, K, _stream())
+    return (h_out if h else None, hg_out if hg else None, partial_out if partial else None)
+
+
+def rms_reduce(partial, N: int, eps: float, r_out=None):
+    """r_i = 1 / sqrt(sum_t partial[t, i] / N + eps)."""
+    T, M = partial.shape
+    _need(partial, F32, "partial")
+    if r_out is None:
+        r_out = _empty((M,), F32, partial)
+    _call("coda_rms_reduce", _ptr(partial), M, T, N, float(eps), _ptr(r_out), _stream())
+    return r_out
+
+
+def gemm_rowscale(A, W, r=None, out=None):
+    """out = bf16(r * (A W)); r None gives a plain bf16 GEMM."""
+    M, K = A.shape
+    N = W.shape[1]
+    _need(A, BF16, "A")
+    _need(W, BF16, "W", (K, N))
+    if r is not None:
+        _need(r, F32, "r", (M,))
+    if out is None:
+        out = _empty((M, N), BF16, A)
+    _call("coda_gemm_rowscale", _ptr(A), _ptr(W), _ptr(r), _ptr(out), M, N, K, _stream())
+    return out
+
+
+def gemm_swiglu(A, W_gu, r=None, save=False, act_out=None):
+    """act = silu(r * A W_g) * (r * A W_u); returns (act, gateup or None)."""
+    M, K = A.shape
+    F = W_gu.shape[1] // 2
+    _need(A, BF16, "A")
+    _need(W_gu, BF16, "W_gu", (K, 2 * F))
+    if r is not None:
+        _need(r, F32, "r", (M,))
+    if act_out is None:
+        act_out = _empty((M, F), BF16, A)
+    gu = _empty((M, 2 * F), BF16, A) if save else None
+    _call("coda_gemm_swiglu", _ptr(A), _ptr(W_gu), _ptr(r), _ptr(act_out), _ptr(gu), M, F, K, _stream())
+    return act_out, gu
+
+
+def lmhead_ce_workspace_size(M: int, V: int) -> int:
+    return int(load_library().coda_lmhead_ce_workspace_size(M, V))
+
+
+def lmhead_ce(H, W, labels, r=None, ws=None):
+    """Fused LM-head cross-entropy; returns (loss[M], lse[M], mean[1]) fp32."""
+    M, K = H.shape
+    V = W.shape[1]
+    _need(H, BF16, "H")
+    _need(W, BF16, "W", (K, V))
+    _need(labels, torch.int64, "labels", (M,))
+    if r is not None:
+        _need(r, F32, "r", (M,))
+    loss = _empty((M,), F32, H)
+    lse = _empty((M,), F32, H)
+    mean = _empty((1,), F32, H)
+    nb = lmhead_ce_workspace_size(M, V)
+    if ws is None:
+        ws = _empty((max(nb, 16),), torch.uint8, H)
+    _call("coda_lmhead_ce", _ptr(H), _ptr(W), _ptr(labels), _ptr(r), _ptr(loss), _ptr(lse), _ptr(mean),
+          _ptr(ws), ws.numel(), M, V, K, _stream())
+    return loss, lse, mean
+
+
+# ---------------------------------------------------------------- backward
+
+
+def gemm_rowscale_bwd(dOut, hg, W2, r, ws=None):
+    """Backward of out = r * (hg W2); returns (d_hg, dW2, pdr)."""
+    M, N2 = dOut.shape
+    N = hg.shape[1]
+    _need(dOut, BF16, "dOut")
+    _need(hg, BF16, "hg", (M, N))
+    _need(W2, BF16, "W2", (N, N2))
+    _need(r, F32, "r", (M,))
+    d_hg = _empty((M, N), F32, dOut)
+    dW2 = _empty((N, N2), F32, dOut)
+    pdr = _empty((partial_cols(N), M), F32, dOut)
+    nb = int(load_library().coda_gemm_rowscale_bwd_workspace_size(M, N))
+    if ws is None:
+        ws = _empty((max(nb, 16),), torch.uint8, dOut)
+    _call("coda_gemm_rowscale_bwd", _ptr(dOut), _ptr(hg), _ptr(W2), _ptr(r), _ptr(d_hg), _ptr(dW2), _ptr(pdr),
+          _ptr(ws), ws.numel(), M, N, N2, _stream())
+    return d_hg, dW2, pdr
+
+
+def rms_reduce_bwd(pdr, r, d_hg, h, gamma, ws=None):
+    """RMSNorm backward row reduction; returns (dh, dgamma)."""
+    T, M = pdr.shape
+    N = h.shape[1]
+    _need(pdr, F32, "pdr")
+    _need(r, F32, "r", (M,))
+    _need(d_hg, F32, "d_hg", (M, N))
+    _need(h, BF16, "h", (M, N))
+    _need(gamma, BF16, "gamma", (N,))
+    dh = _empty((M, N), BF16, h)
+    dgamma = _empty((N,), F32, h)
+    nb = int(load_library().coda_rms_reduce_bwd_workspace_size(M, N))
+    if ws is None:
+        ws = _empty((max(nb, 16),), torch.uint8, h)
+    _call("coda_rms_reduce_bwd", _ptr(pdr), _ptr(r), _ptr(d_hg), _ptr(h), _ptr(gamma), _ptr(dh), _ptr(dgamma),
+          _ptr(ws), ws.numel(), M, T, N, _stream())
+    return dh, dgamma
+
+
+def gemm_res_partialrms_bwd(dh, x, W1, dx=True, dW1=True):
+    """Backward of h = x W1 + res; returns (dx, dW1) (dres is dh)."""
+    M, N = dh.shape
+    K = x.shape[1]
+    _need(dh, BF16, "dh")
+    _need(x, BF16, "x", (M, K))
+    _need(W1, BF16, "W1", (K, N))
+    dx_out = _empty((M, K), BF16, dh) if dx else None
+    dW1_out = _empty((K, N), F32, dh) if dW1 else None
+    _call("coda_gemm_res_partialrms_bwd", _ptr(dh), _ptr(x), _ptr(W1), _ptr(dx_out), _ptr(dW1_out), M, N, K,
+          _stream())
+    return dx_out, dW1_out
+
+
+# ------------------------------------------------------ unfused comparison chain
+
+
+def unfused_add(a, b, out=None):
+    _need(a, BF16, "a")
+    _need(b, BF16, "b", tuple(a.shape))
+    if out is None:
+        out = torch.empty_like(a)
+    _call("coda_unfused_add", _ptr(a), _ptr(b), _ptr(out), a.numel(), _stream())
+    return out
+
+
+def unfused_rmsnorm(h, gamma, eps: float, y_out=None, r_out=None):
+    M, N = h.shape
+    _need(h, BF16, "h")
+    _need(gamma, BF16, "gamma", (N,))
+    if y_out is None:
+        y_out = torch.empty_like(h)
+    _call("coda_unfused_rmsnorm", _ptr(h), _ptr(gamma), float(eps), _ptr(y_out), _ptr(r_out), M, N, _stream())
+    return y_out
+
+
+def selftest_bounded_wait(limit_ns: int) -> int:
+    """Runs the bounded-wait self test; returns 1 if the wait gave up."""
+    flag = torch.zeros(4, dtype=torch.int32, device="cuda")
+    _call("coda_selftest_bounded_wait", int(limit_ns), _ptr(flag), _stream())
+    torch.cuda.synchronize()
+    return int(flag[0].item())
+
+
+# -------------------------------------------------- call sequences of the path
+
+
+def gemm_rmsnorm_gemm(x, res, W1, W2, gamma, eps: float, out=None, bufs=None):
+    """The fused block: first GEMM + residual + partial RMS, light reduction,
+    row-scaled second GEMM.  Returns dict(out, h, hg, partial, r)."""
+    M = x.shape[0]
+    N = W1.shape[1]
+    b = bufs or {}
+    h, hg, partial = gemm_res_partialrms(x, W1, res, gamma, h_out=b.get("h"), hg_out=b.get("hg"),
+                                         partial_out=b.get("partial"))
+    r = rms_reduce(partial, N, eps, r_out=b.get("r"))
+    out = gemm_rowscale(hg, W2, r, out=out)
+    return {"out": out, "h": h, "hg": hg, "partial": partial, "r": r}
+
+
+def unfused_block(x, res, W1, W2, gamma, eps: float, out=None, bufs=None):
+    """The unfused comparison chain: GEMM -> add -> RMSNorm -> GEMM, each
+    intermediate written to and read back from HBM."""
+    b = bufs or {}
+    t = gemm_rowscale(x, W1, None, out=b.get("t"))
+    h = unfused_add(t, res, out=b.get("h"))
+    y = unfused_rmsnorm(h, gamma, eps, y_out=b.get("y"))
+    out = gemm_rowscale(y, W2, None, out=out)
+    return {"out": out, "h": h, "y": y}
+
+
+def swiglu_down(hg, r, h, W_gu, W_down, save=False):
+    """SwiGLU + down projection + residual + partials for the next norm."""
+    act, gu = gemm_swiglu(hg, W_gu, r, save=save)
+    h2, _, partial2 = gemm_res_partialrms(act, W_down, h, None, hg=False)
+    return {"act": act, "gateup": gu, "h2": h2, "partial2": partial2}
+
+
+def block_backward(dOut, x, W1, W2, gamma, fwd):
+    """Backward of the fused block from its saved state (h, hg, r)."""
+    d_hg, dW2, pdr = gemm_rowscale_bwd(dOut, fwd["hg"], W2, fwd["r"])
+    dh, dgamma = rms_reduce_bwd(pdr, fwd["r"], d_hg, fwd["h"], gamma)
+    dx, dW1 = gemm_res_partialrms_bwd(dh, x, W1)
+    return {"dW2": dW2, "dgamma": dgamma, "dh": dh, "dres": dh, "dx": dx, "dW1": dW1, "d_hg": d_hg, "pdr": pdr}

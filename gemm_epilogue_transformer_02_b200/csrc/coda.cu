@@ -1,0 +1,545 @@
+// C ABI of the CODA GEMM + epilogue hot path (declarations and contracts in
+// include/coda.h).  Host side: argument validation (before any CUDA call),
+// tensor-map encoding, and launches on the caller's stream.  The library keeps
+// no device allocations of its own.
+#include <mutex>
+
+#include "coda.h"
+#include "coda_device.cuh"
+#include "coda_gemm.cuh"
+#include "coda_rowops.cuh"
+
+namespace {
+
+using namespace coda;
+
+constexpr int64_t kPartialTile = 256;  // BN of the tiles that emit partial sums
+constexpr int kVersion = 1;
+
+int64_t g_wait_ns = 1000000000LL;
+
+// --------------------------------------------------------------- validation
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool dim_ok(int64_t v) { return v > 0 && (v % 8) == 0 && v <= (int64_t(1) << 31) - 1; }
+
+#define CODA_CHECK(cond, code) \
+  do {                         \
+    if (!(cond)) return code;  \
+  } while (0)
+
+// ------------------------------------------------------------------ devices
+
+struct DevInfo {
+  bool init = false;
+  bool ok = false;
+  int sms = 0;
+  uint32_t attr_set = 0;  // bit per kernel kind: dynamic smem attribute applied
+};
+
+std::mutex g_mu;
+DevInfo g_dev[64];
+
+coda_status_t current_device(int* dev_out, DevInfo** info) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return CODA_ERR_DEVICE;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return CODA_ERR_DEVICE;
+    }
+    d.init = true;
+    d.ok = (major == 10 && minor == 0);
+    d.sms = sms;
+  }
+  if (!d.ok) return CODA_ERR_DEVICE;
+  *dev_out = dev;
+  *info = &d;
+  return CODA_OK;
+}
+
+// -------------------------------------------------------------- tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows, cols] with row stride `stride` elements; box
+// box_cols x box_rows; 128-byte swizzle; out-of-range elements read as zero.
+bool tmap2d(CUtensorMap* m, const void* base, bool f32, uint64_t cols, uint64_t rows, uint64_t stride,
+            uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const uint64_t es = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {stride * es};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Operand maps of the mainloop.  A: [M, K] K-major (box 64 x 128) or stored
+// transposed as [K, M] (MN-major, box 64 x 64).  B: [K, N] MN-major (box 64 x 64)
+// or stored transposed as [N, K] (K-major, box 64 x BN).
+bool map_a(CUtensorMap* m, const void* p, bool mn, uint64_t M, uint64_t K) {
+  return mn ? tmap2d(m, p, false, M, K, M, 64, kBK) : tmap2d(m, p, false, K, M, K, kBK, kBM);
+}
+bool map_b(CUtensorMap* m, const void* p, bool mn, uint64_t N, uint64_t K, uint64_t stride, uint32_t bn) {
+  return mn ? tmap2d(m, p, false, N, K, stride, 64, kBK) : tmap2d(m, p, false, K, N, stride, kBK, bn);
+}
+// Epilogue tile maps: 32 rows per warp, 128-byte rows.
+bool map_out_bf16(CUtensorMap* m, const void* p, uint64_t rows, uint64_t cols, uint64_t stride) {
+  return tmap2d(m, p, false, cols, rows, stride, 64, 32);
+}
+bool map_out_f32(CUtensorMap* m, const void* p, uint64_t rows, uint64_t cols) {
+  return tmap2d(m, p, true, cols, rows, cols, 32, 32);
+}
+
+// ------------------------------------------------------------------ launch
+
+enum KernelKind : uint32_t {
+  kKindResPartial = 0,
+  kKindRowScale,
+  kKindRowScaleKK,
+  kKindSwiGLU,
+  kKindCE,
+  kKindBwdP,
+  kKindF32MN,
+};
+
+template <int BN, int STAGES, bool A_MN, bool B_MN, class Epi>
+coda_status_t run_gemm(DevInfo* info, GemmParams<Epi>& p, int M, int N, int K, int n_nt, int group_m,
+                       KernelKind kind, cudaStream_t stream) {
+  auto kern = coda_gemm_kernel<BN, STAGES, A_MN, B_MN, Epi>;
+  constexpr int smem = GemmSmem<BN, STAGES, Epi>::kBytes;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!(info->attr_set & (1u << kind))) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return CODA_ERR_LAUNCH;
+      info->attr_set |= (1u << kind);
+    }
+  }
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.sched.n_mt = (M + kBM - 1) / kBM;
+  p.sched.n_nt = n_nt;
+  p.sched.group_m = group_m < 1 ? 1 : group_m;
+  p.sched.ntiles = p.sched.n_mt * n_nt;
+  p.wait_ns = static_cast<uint64_t>(g_wait_ns);
+  const int grid = p.sched.ntiles < info->sms ? p.sched.ntiles : info->sms;
+  kern<<<grid, kThreads, smem, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+size_t ce_ws_bytes(int64_t M, int64_t V) {
+  const int64_t n_nt = (V + 255) / 256;
+  return 2 * align256(static_cast<size_t>(n_nt) * M * 4) + align256(static_cast<size_t>(M) * 4);
+}
+
+}  // namespace
+
+// =========================================================================
+// extern "C"
+// =========================================================================
+
+extern "C" {
+
+const char* coda_status_string(coda_status_t s) {
+  switch (s) {
+    case CODA_OK: return "CODA_OK";
+    case CODA_ERR_NULL: return "CODA_ERR_NULL: a required pointer is NULL";
+    case CODA_ERR_SHAPE: return "CODA_ERR_SHAPE: invalid size (sizes must be > 0 and multiples of 8; M >= 0)";
+    case CODA_ERR_ALIGN: return "CODA_ERR_ALIGN: a pointer is not 16-byte aligned";
+    case CODA_ERR_WORKSPACE: return "CODA_ERR_WORKSPACE: workspace missing or too small";
+    case CODA_ERR_DEVICE: return "CODA_ERR_DEVICE: no CUDA device or not compute capability 10.0";
+    case CODA_ERR_LAUNCH: return "CODA_ERR_LAUNCH: a CUDA runtime call failed";
+    case CODA_ERR_DEVICE_TIMEOUT: return "CODA_ERR_DEVICE_TIMEOUT: a kernel gave up on a bounded wait";
+    case CODA_ERR_INTERNAL: return "CODA_ERR_INTERNAL: internal failure (tensor map encoding)";
+  }
+  return "CODA_ERR_UNKNOWN";
+}
+
+int coda_version(void) { return kVersion; }
+
+int64_t coda_partial_tile_width(void) { return kPartialTile; }
+
+int64_t coda_partial_cols(int64_t N) { return N <= 0 ? -1 : (N + kPartialTile - 1) / kPartialTile; }
+
+coda_status_t coda_set_wait_limit_ns(int64_t ns) {
+  if (ns <= 0) return CODA_ERR_SHAPE;
+  g_wait_ns = ns;
+  return CODA_OK;
+}
+
+coda_status_t coda_poll_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return CODA_ERR_LAUNCH;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_coda_status, sizeof(int)) != cudaSuccess) return CODA_ERR_LAUNCH;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_coda_status, &zero, sizeof(int)) != cudaSuccess) return CODA_ERR_LAUNCH;
+    return CODA_ERR_DEVICE_TIMEOUT;
+  }
+  return CODA_OK;
+}
+
+// ------------------------------------------------------------------ forward
+
+coda_status_t coda_gemm_res_partialrms(const uint16_t* x, const uint16_t* W, const uint16_t* res,
+                                       const uint16_t* gamma, uint16_t* h_out, uint16_t* hg_out, float* partial,
+                                       int64_t M, int64_t N, int64_t K, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(N) && dim_ok(K), CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(x && W, CODA_ERR_NULL);
+  CODA_CHECK(h_out || hg_out || partial, CODA_ERR_NULL);
+  CODA_CHECK(!hg_out || gamma, CODA_ERR_NULL);
+  CODA_CHECK(al16(x) && al16(W) && al16(res) && al16(gamma) && al16(h_out) && al16(hg_out) && al16(partial),
+             CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  using Epi = EpiLoadStore2<0>;
+  GemmParams<Epi> p{};
+  bool ok = map_a(&p.tmA, x, false, M, K) && map_b(&p.tmB, W, true, N, K, N, 256);
+  if (res) ok = ok && map_out_bf16(&p.ep.tmIn, res, M, N, N);
+  if (h_out) ok = ok && map_out_bf16(&p.ep.tmOut1, h_out, M, N, N);
+  if (hg_out) ok = ok && map_out_bf16(&p.ep.tmOut2, hg_out, M, N, N);
+  if (!ok) return CODA_ERR_INTERNAL;
+  p.ep.gamma = reinterpret_cast<const __nv_bfloat16*>(gamma);
+  p.ep.r = nullptr;
+  p.ep.partial = partial;
+  p.ep.has_in = res != nullptr;
+  p.ep.has_out1 = h_out != nullptr;
+  p.ep.has_out2 = hg_out != nullptr;
+  const int n_nt = static_cast<int>((N + 255) / 256);
+  return run_gemm<256, 3, false, true, Epi>(info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), n_nt,
+                                            16, kKindResPartial, static_cast<cudaStream_t>(stream));
+}
+
+coda_status_t coda_rms_reduce(const float* partial, int64_t M, int64_t T, int64_t N, float eps, float* r_out,
+                              void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && T > 0 && N > 0 && T <= 1 << 20 && eps >= 0.f, CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(partial && r_out, CODA_ERR_NULL);
+  CODA_CHECK(al16(partial) && al16(r_out), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  coda_status_t st = current_device(&dev, &info);
+  if (st != CODA_OK) return st;
+  const int threads = 256;
+  const int blocks = static_cast<int>((M + threads - 1) / threads);
+  rms_reduce_kernel<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      partial, static_cast<int>(M), static_cast<int>(T), 1.0f / static_cast<float>(N), eps, r_out);
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}
+
+coda_status_t coda_gemm_rowscale(const uint16_t* A, const uint16_t* W, const float* r, uint16_t* out, int64_t M,
+                                 int64_t N, int64_t K, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(N) && dim_ok(K), CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(A && W && out, CODA_ERR_NULL);
+  CODA_CHECK(al16(A) && al16(W) && al16(r) && al16(out), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  using Epi = EpiRowScale;
+  GemmParams<Epi> p{};
+  if (!(map_a(&p.tmA, A, false, M, K) && map_b(&p.tmB, W, true, N, K, N, 256) &&
+        map_out_bf16(&p.ep.tmOut, out, M, N, N)))
+    return CODA_ERR_INTERNAL;
+  p.ep.r = r;
+  const int n_nt = static_cast<int>((N + 255) / 256);
+  return run_gemm<256, 4, false, true, Epi>(info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), n_nt,
+                                            16, kKindRowScale, static_cast<cudaStream_t>(stream));
+}
+
+coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const float* r, uint16_t* act_out,
+                               uint16_t* gateup_save, int64_t M, int64_t F, int64_t K, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(F) && dim_ok(K), CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(A && W_gu && act_out, CODA_ERR_NULL);
+  CODA_CHECK(al16(A) && al16(W_gu) && al16(r) && al16(act_out) && al16(gateup_save), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  using Epi = EpiSwiGLU;
+  GemmParams<Epi> p{};
+  bool ok = map_a(&p.tmA, A, false, M, K) && map_b(&p.tmB, W_gu, true, F, K, 2 * F, 256) &&
+            map_b(&p.tmB2, W_gu + F, true, F, K, 2 * F, 256) && map_out_bf16(&p.ep.tmAct, act_out, M, F, F);
+  if (gateup_save)
+    ok = ok && map_out_bf16(&p.ep.tmSaveG, gateup_save, M, F, 2 * F) &&
+         map_out_bf16(&p.ep.tmSaveU, gateup_save + F, M, F, 2 * F);
+  if (!ok) return CODA_ERR_INTERNAL;
+  p.ep.r = r;
+  p.ep.has_save = gateup_save != nullptr;
+  const int n_nt = static_cast<int>((F + 127) / 128);
+  return run_gemm<256, 3, false, true, Epi>(info, p, static_cast<int>(M), static_cast<int>(F), static_cast<int>(K), n_nt,
+                                            16, kKindSwiGLU, static_cast<cudaStream_t>(stream));
+}
+
+size_t coda_lmhead_ce_workspace_size(int64_t M, int64_t V) {
+  if (M < 0 || V <= 0) return 0;
+  return ce_ws_bytes(M, V);
+}
+
+coda_status_t coda_lmhead_ce(const uint16_t* H, const uint16_t* W, const int64_t* labels, const float* r,
+                             float* loss_out, float* lse_out, float* mean_out, void* ws, size_t ws_bytes,
+                             int64_t M, int64_t V, int64_t K, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(V) && dim_ok(K), CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(H && W && labels && loss_out && lse_out, CODA_ERR_NULL);
+  CODA_CHECK(al16(H) && al16(W) && al16(labels) && al16(r) && al16(loss_out) && al16(lse_out) && al16(ws),
+             CODA_ERR_ALIGN);
+  CODA_CHECK(ws != nullptr && ws_bytes >= ce_ws_bytes(M, V), CODA_ERR_WORKSPACE);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  using Epi = EpiCE;
+  GemmParams<Epi> p{};
+  if (!(map_a(&p.tmA, H, false, M, K) && map_b(&p.tmB, W, true, V, K, V, 256))) return CODA_ERR_INTERNAL;
+  const int n_nt = static_cast<int>((V + 255) / 256);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  p.ep.ws_m = reinterpret_cast<float*>(w);
+  p.ep.ws_s = reinterpret_cast<float*>(w + align256(static_cast<size_t>(n_nt) * M * 4));
+  p.ep.zlab = reinterpret_cast<float*>(w + 2 * align256(static_cast<size_t>(n_nt) * M * 4));
+  p.ep.labels = labels;
+  p.ep.r = r;
+  const int n_mt = static_cast<int>((M + kBM - 1) / kBM);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  coda_status_t st = run_gemm<256, 4, false, true, Epi>(info, p, static_cast<int>(M), static_cast<int>(V),
+                                                        static_cast<int>(K), n_nt, n_mt, kKindCE, s);
+  if (st != CODA_OK) return st;
+  ce_combine_kernel<<<static_cast<int>((M + 31) / 32), 32 * kCombWarps, 0, s>>>(
+      p.ep.ws_m, p.ep.ws_s, p.ep.zlab, labels, static_cast<int>(M), n_nt, V, lse_out, loss_out);
+  if (cudaGetLastError() != cudaSuccess) return CODA_ERR_LAUNCH;
+  if (mean_out) {
+    mean_kernel<<<1, 1024, 0, s>>>(loss_out, static_cast<int>(M), mean_out);
+    if (cudaGetLastError() != cudaSuccess) return CODA_ERR_LAUNCH;
+  }
+  return CODA_OK;
+}
+
+// ----------------------------------------------------------------- backward
+
+size_t coda_gemm_rowscale_bwd_workspace_size(int64_t M, int64_t N) {
+  if (M < 0 || N <= 0) return 0;
+  return align256(static_cast<size_t>(M) * N * 2);
+}
+
+coda_status_t coda_gemm_rowscale_bwd(const uint16_t* dOut, const uint16_t* hg, const uint16_t* W2, const float* r,
+                                     float* d_hg_out, float* dW2_out, float* pdr_out, void* ws, size_t ws_bytes,
+                                     int64_t M, int64_t N, int64_t N2, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(N) && dim_ok(N2), CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(dOut && hg && W2 && r && d_hg_out && dW2_out && pdr_out, CODA_ERR_NULL);
+  CODA_CHECK(al16(dOut) && al16(hg) && al16(W2) && al16(r) && al16(d_hg_out) && al16(dW2_out) && al16(pdr_out) &&
+                 al16(ws),
+             CODA_ERR_ALIGN);
+  CODA_CHECK(ws != nullptr && ws_bytes >= coda_gemm_rowscale_bwd_workspace_size(M, N), CODA_ERR_WORKSPACE);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  uint16_t* y = static_cast<uint16_t*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  {
+    // P = dOut W2^T with the block-local epilogue (d_hg, y, pdr).
+    using Epi = EpiLoadStore2<1>;
+    GemmParams<Epi> p{};
+    if (!(map_a(&p.tmA, dOut, false, M, N2) && map_b(&p.tmB, W2, false, N, N2, N2, 256) &&
+          map_out_bf16(&p.ep.tmIn, hg, M, N, N) && map_out_bf16(&p.ep.tmOut1, y, M, N, N) &&
+          map_out_f32(&p.ep.tmOut2, d_hg_out, M, N)))
+      return CODA_ERR_INTERNAL;
+    p.ep.gamma = nullptr;
+    p.ep.r = r;
+    p.ep.partial = pdr_out;
+    p.ep.has_in = 1;
+    p.ep.has_out1 = 1;
+    p.ep.has_out2 = 1;
+    coda_status_t st = run_gemm<256, 3, false, false, Epi>(info, p, static_cast<int>(M), static_cast<int>(N),
+                                                           static_cast<int>(N2), static_cast<int>((N + 255) / 256),
+                                                           16, kKindBwdP, s);
+    if (st != CODA_OK) return st;
+  }
+  {
+    // dW2 = y^T dOut: A = y read transposed (MN-major), B = dOut (MN-major), K = tokens.
+    using Epi = EpiStoreF32;
+    GemmParams<Epi> p{};
+    if (!(map_a(&p.tmA, y, true, N, M) && map_b(&p.tmB, dOut, true, N2, M, N2, 256) &&
+          map_out_f32(&p.ep.tmOut, dW2_out, N, N2)))
+      return CODA_ERR_INTERNAL;
+    return run_gemm<256, 4, true, true, Epi>(info, p, static_cast<int>(N), static_cast<int>(N2), static_cast<int>(M),
+                                             static_cast<int>((N2 + 255) / 256), 16, kKindF32MN, s);
+  }
+}
+
+size_t coda_rms_reduce_bwd_workspace_size(int64_t M, int64_t N) {
+  if (M < 0 || N <= 0) return 0;
+  return align256(static_cast<size_t>((M + kBwdRows - 1) / kBwdRows) * N * 4);
+}
+
+coda_status_t coda_rms_reduce_bwd(const float* pdr, const float* r, const float* d_hg, const uint16_t* h,
+                                  const uint16_t* gamma, uint16_t* dh_out, float* dgamma_out, void* ws,
+                                  size_t ws_bytes, int64_t M, int64_t T, int64_t N, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && T > 0 && T <= 1 << 20 && dim_ok(N), CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(pdr && r && d_hg && h && gamma && dh_out && dgamma_out, CODA_ERR_NULL);
+  CODA_CHECK(al16(pdr) && al16(r) && al16(d_hg) && al16(h) && al16(gamma) && al16(dh_out) && al16(dgamma_out) &&
+                 al16(ws),
+             CODA_ERR_ALIGN);
+  CODA_CHECK(ws != nullptr && ws_bytes >= coda_rms_reduce_bwd_workspace_size(M, N), CODA_ERR_WORKSPACE);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  coda_status_t st = current_device(&dev, &info);
+  if (st != CODA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int nblk = static_cast<int>((M + kBwdRows - 1) / kBwdRows);
+  float* part = static_cast<float*>(ws);
+  rms_reduce_bwd_kernel<<<nblk, kBwdThreads, 0, s>>>(
+      pdr, r, d_hg, reinterpret_cast<const __nv_bfloat16*>(h),
+      reinterpret_cast<const __nv_bfloat16*>(gamma), reinterpret_cast<__nv_bfloat16*>(dh_out), part,
+      static_cast<int>(M), static_cast<int>(T), static_cast<int>(N));
+  if (cudaGetLastError() != cudaSuccess) return CODA_ERR_LAUNCH;
+  dgamma_final_kernel<<<static_cast<int>((N + 255) / 256), 256, 0, s>>>(part, nblk, static_cast<int>(N), dgamma_out);
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}
+
+coda_status_t coda_gemm_res_partialrms_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* W1,
+                                           uint16_t* dx_out, float* dW1_out, int64_t M, int64_t N, int64_t K,
+                                           void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(N) && dim_ok(K), CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(dh && x && W1, CODA_ERR_NULL);
+  CODA_CHECK(dx_out || dW1_out, CODA_ERR_NULL);
+  CODA_CHECK(al16(dh) && al16(x) && al16(W1) && al16(dx_out) && al16(dW1_out), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dx_out) {
+    // dx = dh W1^T: B = W1 read as [K rows of length N] (K-major), GEMM K = N.
+    using Epi = EpiRowScale;
+    GemmParams<Epi> p{};
+    if (!(map_a(&p.tmA, dh, false, M, N) && map_b(&p.tmB, W1, false, K, N, N, 256) &&
+          map_out_bf16(&p.ep.tmOut, dx_out, M, K, K)))
+      return CODA_ERR_INTERNAL;
+    p.ep.r = nullptr;
+    coda_status_t st = run_gemm<256, 4, false, false, Epi>(info, p, static_cast<int>(M), static_cast<int>(K),
+                                                           static_cast<int>(N), static_cast<int>((K + 255) / 256),
+                                                           16, kKindRowScaleKK, s);
+    if (st != CODA_OK) return st;
+  }
+  if (dW1_out) {
+    // dW1 = x^T dh: A = x read transposed (MN-major), B = dh (MN-major), K = tokens.
+    using Epi = EpiStoreF32;
+    GemmParams<Epi> p{};
+    if (!(map_a(&p.tmA, x, true, K, M) && map_b(&p.tmB, dh, true, N, M, N, 256) &&
+          map_out_f32(&p.ep.tmOut, dW1_out, K, N)))
+      return CODA_ERR_INTERNAL;
+    return run_gemm<256, 4, true, true, Epi>(info, p, static_cast<int>(K), static_cast<int>(N), static_cast<int>(M),
+                                             static_cast<int>((N + 255) / 256), 16, kKindF32MN, s);
+  }
+  return CODA_OK;
+}
+
+// --------------------------------------------------- unfused comparison chain
+
+coda_status_t coda_unfused_add(const uint16_t* a, const uint16_t* b, uint16_t* out, int64_t n, void* stream) {
+  CODA_CHECK(a && b && out, CODA_ERR_NULL);
+  CODA_CHECK(n >= 0 && n % 8 == 0, CODA_ERR_SHAPE);
+  CODA_CHECK(al16(a) && al16(b) && al16(out), CODA_ERR_ALIGN);
+  if (n == 0) return CODA_OK;
+  int dev = 0;
+  DevInfo* info = nullptr;
+  coda_status_t st = current_device(&dev, &info);
+  if (st != CODA_OK) return st;
+  const size_t n8 = static_cast<size_t>(n / 8);
+  const int threads = 256;
+  size_t blocks = (n8 + threads - 1) / threads;
+  const size_t cap = static_cast<size_t>(info->sms) * 8;
+  if (blocks > cap) blocks = cap;
+  add_bf16_kernel<<<static_cast<int>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const __nv_bfloat16*>(a), reinterpret_cast<const __nv_bfloat16*>(b),
+      reinterpret_cast<__nv_bfloat16*>(out), n8);
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}
+
+coda_status_t coda_unfused_rmsnorm(const uint16_t* h, const uint16_t* gamma, float eps, uint16_t* y_out,
+                                   float* r_out, int64_t M, int64_t N, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(N) && eps >= 0.f, CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(h && gamma && y_out, CODA_ERR_NULL);
+  CODA_CHECK(al16(h) && al16(gamma) && al16(y_out) && al16(r_out), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  coda_status_t st = current_device(&dev, &info);
+  if (st != CODA_OK) return st;
+  rmsnorm_kernel<<<static_cast<int>(M), kNormThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const __nv_bfloat16*>(h), reinterpret_cast<const __nv_bfloat16*>(gamma), eps,
+      reinterpret_cast<__nv_bfloat16*>(y_out), r_out, static_cast<int>(N));
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}
+
+// ------------------------------------------------------------------- testing
+
+coda_status_t coda_selftest_bounded_wait(int64_t limit_ns, int* gave_up_dev, void* stream) {
+  CODA_CHECK(gave_up_dev, CODA_ERR_NULL);
+  CODA_CHECK(limit_ns > 0 && limit_ns <= 10000000000LL, CODA_ERR_SHAPE);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  coda_status_t st = current_device(&dev, &info);
+  if (st != CODA_OK) return st;
+  bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_ns),
+                                                                                gave_up_dev);
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}
+
+}  // extern "C"

@@ -1,0 +1,753 @@
+// Persistent, warp-specialised tcgen05 GEMM with programmable epilogues.
+//
+// This is the "fixed mainloop + programmable epilogue" structure of the KuCoin
+// news flash "CODA: new research optimizes transformer training with GEMM
+// epilogue programming" (section "CODA: the secret in the epilogue": a GEMM is
+// a mainloop of tiled multiply-accumulate and an epilogue that post-processes
+// the tile while it is still on chip; section "Five kinds of building blocks":
+// the mainloop stays fixed and the epilogue is composed of elementwise
+// transforms, vector loads, matrix-block loads/stores, chunk reductions and
+// stateful transforms).
+//
+// Mainloop (one CTA per SM, 192 threads):
+//   warp 0  - one thread issues TMA loads of A and B k-blocks into a ring of
+//             shared-memory stages (128-byte swizzle).
+//   warp 1  - one thread issues tcgen05.mma (bf16 x bf16 -> fp32) into one of
+//             two tensor-memory accumulators (128 lanes x BN columns each).
+//   warps 2-5 - the epilogue: each warp owns 32 accumulator rows (the TMEM
+//             lane quarter warp % 4), reads its rows with tcgen05.ld while the
+//             MMA warp already fills the other accumulator, and runs the
+//             epilogue functor.  One thread owns one output row, so per-row
+//             reductions (partial sums of squares, online max / sum-exp) are
+//             thread-local.
+// Tiles are handed out round-robin over a grouped raster (group_m M-tiles per
+// column sweep) so that concurrently running CTAs share operand tiles in L2.
+// Operands: A is [M, K] K-major (row-major activations) or MN-major (a
+// transposed view for weight gradients); B is [K, N] MN-major (row-major
+// weights) or K-major (a transposed weight).  Rows beyond M, columns beyond N
+// and k beyond K are zero-filled by TMA and clipped on store.
+#pragma once
+
+#include "coda_device.cuh"
+
+namespace coda {
+
+constexpr int kBM = 128;        // accumulator rows per tile (TMEM lanes)
+constexpr int kBK = 64;         // k-block: 64 bf16 = one 128-byte swizzle row
+constexpr int kThreads = 192;   // 6 warps
+constexpr int kEpiWarps = 4;
+
+struct TileSched {
+  int n_mt;     // M tiles
+  int n_nt;     // N tiles
+  int group_m;  // M tiles per raster group
+  int ntiles;
+
+  __device__ __forceinline__ void map(int t, int& mb, int& nb) const {
+    const int per_group = group_m * n_nt;
+    const int g = t / per_group;
+    const int first = g * group_m;
+    const int gs = min(n_mt - first, group_m);
+    const int r = t - g * per_group;
+    mb = first + r % gs;
+    nb = r / gs;
+  }
+};
+
+template <class Epi>
+struct GemmParams {
+  CUtensorMap tmA;
+  CUtensorMap tmB;
+  CUtensorMap tmB2;  // second half of a paired B operand (SwiGLU up columns)
+  typename Epi::Params ep;
+  int M, N, K;       // GEMM sizes; N counts accumulator columns of the output space
+  TileSched sched;
+  uint64_t wait_ns;
+};
+
+// Per-warp context handed to the epilogue for one tile.
+struct TileCtx {
+  int M, N;          // output rows / columns
+  int mb, nb;        // tile coordinates
+  int row0;          // first global row of this warp's 32 rows
+  uint32_t taddr;    // TMEM address of (this warp's lane 0, accumulator column 0)
+  int lane;
+  uint8_t* wsmem;    // this warp's epilogue shared memory
+  uint64_t* wbars;   // this warp's epilogue mbarriers
+};
+
+template <int BN, int STAGES, class Epi>
+struct GemmSmem {
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kEpiBytes = kEpiWarps * Epi::kSmemPerWarp;
+  static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1 + kEpiWarps * Epi::kBarsPerWarp;
+  static constexpr int kBytes = 1024 /*align slack*/ + STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 16;
+};
+
+// Bounded wait that ignores the abort flag (used to drain copies in flight
+// before the CTA exits).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  int dummy_abort = 0;
+  WaitCtx w{&dummy_abort, limit_ns};
+  (void)mbar_wait(bar, parity, w);
+}
+
+template <int BN, int STAGES, bool A_MN, bool B_MN, class Epi>
+__global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_constant__ GemmParams<Epi> p) {
+  using S = GemmSmem<BN, STAGES, Epi>;
+  static_assert(BN % 64 == 0 && BN <= 256, "BN must be a multiple of 64, at most 256");
+  static_assert(2 * BN == 512 || 2 * BN == 256 || 2 * BN == 128, "TMEM columns must be a power of two");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * S::kABytes;
+  uint8_t* sEpi = smem + STAGES * S::kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + S::kEpiBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint64_t* ebars = drain + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ebars + kEpiWarps * Epi::kBarsPerWarp);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    for (int i = 0; i < kEpiWarps * Epi::kBarsPerWarp; ++i) mbar_init(&ebars[i], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmA);
+    tma_prefetch_desc(&p.tmB);
+    if (Epi::kPairedB) tma_prefetch_desc(&p.tmB2);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 2 * BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const WaitCtx w{abort_flag, p.wait_ns};
+  const int nkb = (p.K + kBK - 1) / kBK;
+  const int ntiles = p.sched.ntiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+        int mb, nb;
+        p.sched.map(t, mb, nb);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, w)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+          uint8_t* a = sA + stage * S::kABytes;
+          uint8_t* b = sB + stage * S::kBBytes;
+          if (!A_MN) {
+            tma_load_2d(a, &p.tmA, &full[stage], kb * kBK, mb * kBM);
+          } else {
+#pragma unroll
+            for (int j = 0; j < kBM / 64; ++j)
+              tma_load_2d(a + j * (64 * kBK * 2), &p.tmA, &full[stage], mb * kBM + j * 64, kb * kBK);
+          }
+          if (!B_MN) {
+            tma_load_2d(b, &p.tmB, &full[stage], kb * kBK, nb * BN);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) {
+              if (Epi::kPairedB) {
+                const CUtensorMap* m = (j < BN / 128) ? &p.tmB : &p.tmB2;
+                const int col = nb * (BN / 2) + (j % (BN / 128)) * 64;
+                tma_load_2d(b + j * (64 * kBK * 2), m, &full[stage], col, kb * kBK);
+              } else {
+                tma_load_2d(b + j * (64 * kBK * 2), &p.tmB, &full[stage], nb * BN + j * 64, kb * kBK);
+              }
+            }
+          }
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Drain: every load issued must have landed before shared memory goes away.
+      const long n = issued < STAGES ? issued : STAGES;
+      for (long i = 0; i < n; ++i) {
+        if (stage == 0) {
+          stage = STAGES - 1;
+          phase ^= 1u;
+        } else {
+          --stage;
+        }
+        drain_wait(&full[stage], phase, p.wait_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, A_MN, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, w)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * BN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, w)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * S::kABytes);
+          const uint32_t b0 = smem_u32(sB + stage * S::kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = A_MN ? sdesc_sw128(a0 + kk * 16 * 128, 64 * kBK * 2, 1024)
+                                     : sdesc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sdesc_sw128(b0 + kk * 16 * 128, 64 * kBK * 2, 1024)
+                                     : sdesc_sw128(b0 + kk * 32, 16, 1024);
+            tc_mma_bf16(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);
+      }
+      // All MMAs issued by this thread have completed once this arrives.
+      tc_commit(drain);
+      drain_wait(drain, 0, p.wait_ns);
+    }
+  } else {
+    // --------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int ew = warp - 2;
+    uint8_t* wsmem = sEpi + ew * Epi::kSmemPerWarp;
+    uint64_t* wbars = ebars + ew * Epi::kBarsPerWarp;
+    typename Epi::State st;
+    Epi::init_state(st);
+    int it = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+      int mb, nb;
+      p.sched.map(t, mb, nb);
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      // Warp-uniform outcome: tcgen05.ld below is a warp-collective instruction.
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aph, w))) break;
+      tc_fence_after();
+      TileCtx c;
+      c.M = p.M;
+      c.N = p.N;
+      c.mb = mb;
+      c.nb = nb;
+      c.row0 = mb * kBM + q * 32;
+      c.taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+      c.lane = lane;
+      c.wsmem = wsmem;
+      c.wbars = wbars;
+      const bool ok = Epi::template tile<BN>(p.ep, c, st, w);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (!ok) break;
+    }
+    Epi::finish(p.ep, st, wbars, lane, p.wait_ns);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * BN);
+  }
+}
+
+// =========================================================================
+// Epilogues
+// =========================================================================
+
+// Loads 64 accumulator columns [col, col + 64) of this thread's row.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&v0)[32], uint32_t (&v1)[32]) {
+  tmem_ld32(taddr, v0);
+  tmem_ld32(taddr + 32, v1);
+  tmem_ld_wait(v0);
+  reg_pin(v1);
+}
+
+__device__ __forceinline__ float acc_at(const uint32_t (&v0)[32], const uint32_t (&v1)[32], int i) {
+  return __uint_as_float(i < 32 ? v0[i] : v1[i - 32]);
+}
+
+// ---------------------------------------------------------------------------
+// Load one bf16 tile, store two tiles and a per-row partial sum.
+//   MODE 0 (first GEMM of the block, "GEMM-Residual-PartialRMS"):
+//     h = acc + res;  out1 = bf16(h);  out2 = hg = bf16(gamma * h);  partial += h^2
+//     (double-buffered: the residual of the next chunk loads while this one computes)
+//   MODE 1 (backward of the row-scaled second GEMM, acc = P = dOut W2^T):
+//     in = hg;  out1 = y = bf16(r * hg);  out2 = d_hg = r * P (fp32);  partial += hg * P
+//     (single-buffered: its mainloop is long enough to hide the epilogue)
+// partial is laid out [column tile][row] (fp32).
+// ---------------------------------------------------------------------------
+template <int MODE>
+struct EpiLoadStore2 {
+  static constexpr int kNBuf = MODE == 0 ? 2 : 1;
+  static constexpr int kOut2Bytes = MODE == 0 ? 4096 : 8192;  // 32 x 64 bf16, or 32 x 64 fp32 as two 32 x 32 boxes
+  static constexpr int kBufBytes = 4096 + kOut2Bytes;
+  static constexpr int kSmemPerWarp = kNBuf * kBufBytes;
+  static constexpr int kBarsPerWarp = kNBuf;
+  static constexpr bool kPairedB = false;
+
+  struct Params {
+    CUtensorMap tmIn;    // [M, N] bf16, box 64 x 32
+    CUtensorMap tmOut1;  // [M, N] bf16, box 64 x 32
+    CUtensorMap tmOut2;  // [M, N] bf16 box 64 x 32 (MODE 0) or fp32 box 32 x 32 (MODE 1)
+    const __nv_bfloat16* gamma;  // MODE 0 (may be null when out2 is not stored)
+    const float* r;              // MODE 1
+    float* partial;              // [T, M] or null
+    int has_in, has_out1, has_out2;
+  };
+
+  struct State {
+    uint32_t cnt;        // chunks processed by this warp (selects the buffer)
+    uint32_t phase[2];   // parity of the next completion of each input barrier
+    uint32_t pending;    // bit b set: a load into buffer b is in flight
+  };
+
+  __device__ static void init_state(State& s) {
+    s.cnt = 0;
+    s.phase[0] = s.phase[1] = 0;
+    s.pending = 0;
+  }
+
+  template <int BN>
+  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx& w) {
+    const int col0 = c.nb * BN;
+    const int row = c.row0 + c.lane;
+    int nch = (c.N - col0 + 63) / 64;
+    if (nch > BN / 64) nch = BN / 64;
+    const bool rows_live = c.row0 < c.M;
+    float rs = 1.f;
+    if (MODE == 1) rs = (row < c.M) ? __ldg(ep.r + row) : 0.f;
+    const bool has_in = ep.has_in != 0;
+
+    auto buf_of = [&](uint32_t cnt) -> int { return kNBuf == 2 ? static_cast<int>(cnt & 1) : 0; };
+    auto issue = [&](int ch, int b) {
+      if (c.lane == 0) {
+        mbar_arrive_expect_tx(&c.wbars[b], 32 * 128);
+        tma_load_2d(c.wsmem + b * kBufBytes, &ep.tmIn, &c.wbars[b], col0 + ch * 64, c.row0);
+      }
+      st.pending |= (1u << b);
+    };
+
+    if (kNBuf == 2 && has_in && nch > 0) {
+      if (c.lane == 0) bulk_wait_read<1>();  // buffer cnt&1 was last stored two chunks ago
+      __syncwarp();
+      issue(0, buf_of(st.cnt));
+    }
+    float ss = 0.f;
+    for (int ch = 0; ch < nch; ++ch) {
+      const int b = buf_of(st.cnt);
+      uint8_t* R = c.wsmem + b * kBufBytes;
+      uint8_t* G = R + 4096;
+      if (kNBuf == 1) {
+        if (c.lane == 0) bulk_wait_read<0>();  // the previous chunk's stores have read the buffer
+        __syncwarp();
+        if (has_in) issue(ch, 0);
+      } else if (has_in) {
+        if (ch + 1 < nch) {
+          if (c.lane == 0) bulk_wait_read<0>();  // the other buffer's store must have read it
+          __syncwarp();
+          issue(ch + 1, b ^ 1);
+        }
+      } else {
+        if (c.lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+      }
+      uint32_t v0[32], v1[32];
+      tmem_ld64(c.taddr + ch * 64, v0, v1);
+      if (has_in) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&c.wbars[b], st.phase[b], w))) return false;
+        st.phase[b] ^= 1u;
+        st.pending &= ~(1u << b);
+      }
+      const int cc = col0 + ch * 64;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t off = sw128_off(c.lane, j);
+        uint4 in4 = make_uint4(0, 0, 0, 0);
+        if (has_in) in4 = ld_shared_v4(R + off);
+        const uint32_t inw[4] = {in4.x, in4.y, in4.z, in4.w};
+        uint32_t o1[4];
+        if (MODE == 0) {
+          uint32_t o2[4];
+          uint4 g4 = make_uint4(0, 0, 0, 0);  // gamma absent: hg is neither formed nor stored
+          if (ep.gamma != nullptr && cc + j * 8 < c.N)
+            g4 = __ldg(reinterpret_cast<const uint4*>(ep.gamma + cc + j * 8));
+          const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float h0 = acc_at(v0, v1, j * 8 + 2 * e) + bf16lo(inw[e]);
+            const float h1 = acc_at(v0, v1, j * 8 + 2 * e + 1) + bf16hi(inw[e]);
+            ss = fmaf(h0, h0, ss);
+            ss = fmaf(h1, h1, ss);
+            o1[e] = pack_bf16x2(h0, h1);
+            o2[e] = pack_bf16x2(h0 * bf16lo(gw[e]), h1 * bf16hi(gw[e]));
+          }
+          st_shared_v4(G + off, make_uint4(o2[0], o2[1], o2[2], o2[3]));
+        } else {
+          float dg[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p0 = acc_at(v0, v1, j * 8 + 2 * e);
+            const float p1 = acc_at(v0, v1, j * 8 + 2 * e + 1);
+            const float g0 = bf16lo(inw[e]);
+            const float g1 = bf16hi(inw[e]);
+            ss = fmaf(g0, p0, ss);
+            ss = fmaf(g1, p1, ss);
+            o1[e] = pack_bf16x2(rs * g0, rs * g1);
+            dg[2 * e] = rs * p0;
+            dg[2 * e + 1] = rs * p1;
+          }
+          // fp32 columns j*8 .. j*8+7 live in box j/4, 16-byte chunks 2*(j%4) and 2*(j%4)+1
+          uint8_t* Gb = G + (j >> 2) * 4096;
+          st_shared_v4(Gb + sw128_off(c.lane, 2 * (j & 3)),
+                       make_uint4(__float_as_uint(dg[0]), __float_as_uint(dg[1]), __float_as_uint(dg[2]),
+                                  __float_as_uint(dg[3])));
+          st_shared_v4(Gb + sw128_off(c.lane, 2 * (j & 3) + 1),
+                       make_uint4(__float_as_uint(dg[4]), __float_as_uint(dg[5]), __float_as_uint(dg[6]),
+                                  __float_as_uint(dg[7])));
+        }
+        st_shared_v4(R + off, make_uint4(o1[0], o1[1], o1[2], o1[3]));
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (c.lane == 0 && rows_live) {
+        if (ep.has_out1) tma_store_2d(&ep.tmOut1, R, cc, c.row0);
+        if (ep.has_out2) {
+          tma_store_2d(&ep.tmOut2, G, cc, c.row0);
+          if (MODE == 1 && cc + 32 < c.N) tma_store_2d(&ep.tmOut2, G + 4096, cc + 32, c.row0);
+        }
+      }
+      if (c.lane == 0) bulk_commit();
+      ++st.cnt;
+    }
+    if (ep.partial != nullptr && row < c.M) ep.partial[static_cast<size_t>(c.nb) * c.M + row] = ss;
+    return true;
+  }
+
+  __device__ static void finish(const Params& ep, State& st, uint64_t* wbars, int lane, uint64_t limit_ns) {
+    for (int b = 0; b < kNBuf; ++b)
+      if (st.pending & (1u << b)) drain_wait(&wbars[b], st.phase[b], limit_ns);
+    if (lane == 0) bulk_wait_all<0>();
+    __syncwarp();
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Row-scaled bf16 output: out = r * acc (r null: out = acc).  The second GEMM
+// of the block applies the RMSNorm row scale here.
+// ---------------------------------------------------------------------------
+struct EpiRowScale {
+  static constexpr int kSmemPerWarp = 2 * 4096;
+  static constexpr int kBarsPerWarp = 0;
+  static constexpr bool kPairedB = false;
+
+  struct Params {
+    CUtensorMap tmOut;  // [M, N] bf16, box 64 x 32
+    const float* r;     // [M] or null
+  };
+  struct State {
+    uint32_t cnt;
+  };
+  __device__ static void init_state(State& s) { s.cnt = 0; }
+
+  template <int BN>
+  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
+    const int col0 = c.nb * BN;
+    const int row = c.row0 + c.lane;
+    int nch = (c.N - col0 + 63) / 64;
+    if (nch > BN / 64) nch = BN / 64;
+    float rs = 1.f;
+    if (ep.r != nullptr) rs = (row < c.M) ? __ldg(ep.r + row) : 0.f;
+    for (int ch = 0; ch < nch; ++ch) {
+      uint8_t* O = c.wsmem + (st.cnt & 1) * 4096;
+      if (c.lane == 0) bulk_wait_read<1>();
+      __syncwarp();
+      uint32_t v0[32], v1[32];
+      tmem_ld64(c.taddr + ch * 64, v0, v1);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          o[e] = pack_bf16x2(rs * acc_at(v0, v1, j * 8 + 2 * e), rs * acc_at(v0, v1, j * 8 + 2 * e + 1));
+        st_shared_v4(O + sw128_off(c.lane, j), make_uint4(o[0], o[1], o[2], o[3]));
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (c.lane == 0) {
+        if (c.row0 < c.M) tma_store_2d(&ep.tmOut, O, col0 + ch * 64, c.row0);
+        bulk_commit();
+      }
+      ++st.cnt;
+    }
+    return true;
+  }
+
+  __device__ static void finish(const Params&, State&, uint64_t*, int lane, uint64_t) {
+    if (lane == 0) bulk_wait_all<0>();
+    __syncwarp();
+  }
+};
+
+// ---------------------------------------------------------------------------
+// fp32 output (weight gradients): out = acc.
+// ---------------------------------------------------------------------------
+struct EpiStoreF32 {
+  static constexpr int kSmemPerWarp = 2 * 4096;
+  static constexpr int kBarsPerWarp = 0;
+  static constexpr bool kPairedB = false;
+
+  struct Params {
+    CUtensorMap tmOut;  // [M, N] fp32, box 32 x 32
+  };
+  struct State {
+    uint32_t cnt;
+  };
+  __device__ static void init_state(State& s) { s.cnt = 0; }
+
+  template <int BN>
+  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
+    const int col0 = c.nb * BN;
+    int nch = (c.N - col0 + 31) / 32;
+    if (nch > BN / 32) nch = BN / 32;
+    for (int ch = 0; ch < nch; ++ch) {
+      uint8_t* O = c.wsmem + (st.cnt & 1) * 4096;
+      if (c.lane == 0) bulk_wait_read<1>();
+      __syncwarp();
+      uint32_t v[32];
+      tmem_ld32(c.taddr + ch * 32, v);
+      tmem_ld_wait(v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        st_shared_v4(O + sw128_off(c.lane, j), make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+      fence_async_smem();
+      __syncwarp();
+      if (c.lane == 0) {
+        if (c.row0 < c.M) tma_store_2d(&ep.tmOut, O, col0 + ch * 32, c.row0);
+        bulk_commit();
+      }
+      ++st.cnt;
+    }
+    return true;
+  }
+
+  __device__ static void finish(const Params&, State&, uint64_t*, int lane, uint64_t) {
+    if (lane == 0) bulk_wait_all<0>();
+    __syncwarp();
+  }
+};
+
+// ---------------------------------------------------------------------------
+// SwiGLU: the accumulator of one tile holds [gate 128 | up 128] columns for
+// output columns nb*128 .. nb*128+127 (the B operand is loaded as two halves,
+// gate columns from W_gu[:, :F] and up columns from W_gu[:, F:]).
+//   g = r * acc_gate, u = r * acc_up, act = silu(g) * u;
+//   optionally g and u (bf16) are saved for the backward.
+// ---------------------------------------------------------------------------
+struct EpiSwiGLU {
+  static constexpr int kSmemPerWarp = 2 * 4096 + 8192;  // act double buffer + gate/up save buffer
+  static constexpr int kBarsPerWarp = 0;
+  static constexpr bool kPairedB = true;
+
+  struct Params {
+    CUtensorMap tmAct;    // [M, F] bf16, box 64 x 32
+    CUtensorMap tmSaveG;  // gate view of the [M, 2F] save tensor, box 64 x 32
+    CUtensorMap tmSaveU;  // up view of the [M, 2F] save tensor, box 64 x 32
+    const float* r;       // [M] or null
+    int has_save;
+  };
+  struct State {
+    uint32_t cnt;
+  };
+  __device__ static void init_state(State& s) { s.cnt = 0; }
+
+  __device__ static __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
+
+  template <int BN>
+  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
+    constexpr int kHalf = BN / 2;  // output columns per tile
+    const int ocol0 = c.nb * kHalf;
+    const int row = c.row0 + c.lane;
+    int nch = (c.N - ocol0 + 63) / 64;  // c.N = F here
+    if (nch > kHalf / 64) nch = kHalf / 64;
+    float rs = 1.f;
+    if (ep.r != nullptr) rs = (row < c.M) ? __ldg(ep.r + row) : 0.f;
+    const bool save = ep.has_save != 0;
+    uint8_t* SG = c.wsmem + 2 * 4096;
+    uint8_t* SU = SG + 4096;
+    for (int ch = 0; ch < nch; ++ch) {
+      uint8_t* O = c.wsmem + (st.cnt & 1) * 4096;
+      if (c.lane == 0) {
+        if (save)
+          bulk_wait_read<0>();
+        else
+          bulk_wait_read<1>();
+      }
+      __syncwarp();
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t vg[32], vu[32];
+        tmem_ld32(c.taddr + ch * 64 + hh * 32, vg);
+        tmem_ld32(c.taddr + kHalf + ch * 64 + hh * 32, vu);
+        tmem_ld_wait(vg);
+        reg_pin(vu);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          uint32_t o[4], og[4], ou[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = jj * 8 + 2 * e;
+            const float g0 = rs * __uint_as_float(vg[i]), g1 = rs * __uint_as_float(vg[i + 1]);
+            const float u0 = rs * __uint_as_float(vu[i]), u1 = rs * __uint_as_float(vu[i + 1]);
+            o[e] = pack_bf16x2(silu(g0) * u0, silu(g1) * u1);
+            og[e] = pack_bf16x2(g0, g1);
+            ou[e] = pack_bf16x2(u0, u1);
+          }
+          const uint32_t off = sw128_off(c.lane, hh * 4 + jj);
+          st_shared_v4(O + off, make_uint4(o[0], o[1], o[2], o[3]));
+          if (save) {
+            st_shared_v4(SG + off, make_uint4(og[0], og[1], og[2], og[3]));
+            st_shared_v4(SU + off, make_uint4(ou[0], ou[1], ou[2], ou[3]));
+          }
+        }
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (c.lane == 0) {
+        if (c.row0 < c.M) {
+          tma_store_2d(&ep.tmAct, O, ocol0 + ch * 64, c.row0);
+          if (save) {
+            tma_store_2d(&ep.tmSaveG, SG, ocol0 + ch * 64, c.row0);
+            tma_store_2d(&ep.tmSaveU, SU, ocol0 + ch * 64, c.row0);
+          }
+        }
+        bulk_commit();
+      }
+      ++st.cnt;
+    }
+    return true;
+  }
+
+  __device__ static void finish(const Params&, State&, uint64_t*, int lane, uint64_t) {
+    if (lane == 0) bulk_wait_all<0>();
+    __syncwarp();
+  }
+};
+
+// ---------------------------------------------------------------------------
+// LM-head cross-entropy: block log-sum-exp of the tile with an online
+// (running max, running sum-exp) state over 32-column chunks.  Logits stay in
+// fp32 registers and never reach memory.  Per (column tile, row) the tile's
+// (max, sum-exp) goes to the workspace; the tile that holds a row's label
+// also writes that logit.  A combine kernel merges the tiles.
+// ---------------------------------------------------------------------------
+struct EpiCE {
+  static constexpr int kSmemPerWarp = 0;
+  static constexpr int kBarsPerWarp = 0;
+  static constexpr bool kPairedB = false;
+
+  struct Params {
+    float* ws_m;            // [n_tiles_v, M] tile max
+    float* ws_s;            // [n_tiles_v, M] tile sum of exp(z - max)
+    float* zlab;            // [M] label logit
+    const int64_t* labels;  // [M]
+    const float* r;         // [M] or null (row scale of a preceding RMSNorm)
+  };
+  struct State {
+    int unused;
+  };
+  __device__ static void init_state(State&) {}
+
+  template <int BN>
+  __device__ static bool tile(const Params& ep, const TileCtx& c, State&, const WaitCtx&) {
+    constexpr float kL2E = 1.4426950408889634f;
+    const int col0 = c.nb * BN;
+    const int row = c.row0 + c.lane;
+    const bool valid = row < c.M;
+    const int V = c.N;
+    long long lab = valid ? ep.labels[row] : -1;
+    const float rs = (ep.r != nullptr && valid) ? __ldg(ep.r + row) : 1.f;
+    float m = -INFINITY, s = 0.f, zl = 0.f;
+    bool got = false;
+    int nch = (V - col0 + 31) / 32;
+    if (nch > BN / 32) nch = BN / 32;
+    for (int ch = 0; ch < nch; ++ch) {
+      const int cc = col0 + ch * 32;
+      uint32_t v[32];
+      tmem_ld32(c.taddr + ch * 32, v);
+      tmem_ld_wait(v);
+      float z[32];
+      float cm = -INFINITY;
+      const long long d = lab - cc;  // label position inside this chunk, if any
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        z[e] = (cc + e < V) ? rs * __uint_as_float(v[e]) : -INFINITY;
+        cm = fmaxf(cm, z[e]);
+        if (d == e) {
+          zl = z[e];
+          got = true;
+        }
+      }
+      const float mn = fmaxf(m, cm);
+      const float base = mn * kL2E;
+      float sum = 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) sum += exp2f(fmaf(z[e], kL2E, -base));
+      s = s * exp2f((m - mn) * kL2E) + sum;
+      m = mn;
+    }
+    if (valid) {
+      const size_t o = static_cast<size_t>(c.nb) * c.M + row;
+      ep.ws_m[o] = m;
+      ep.ws_s[o] = s;
+      if (got) ep.zlab[row] = zl;
+    }
+    return true;
+  }
+
+  __device__ static void finish(const Params&, State&, uint64_t*, int, uint64_t) {}
+};
+
+}  // namespace coda

@@ -1,0 +1,201 @@
+/*
+ * coda.h - C ABI of the CODA GEMM + epilogue hot path for NVIDIA B200 (sm_100a).
+ *
+ * Source of the operations: KuCoin news flash "CODA: new research optimizes
+ * transformer training with GEMM epilogue programming".
+ *   - Section "CODA: the secret in the epilogue": the GEMM-RMSNorm-GEMM
+ *     pattern (matmul, residual add, RMS normalisation, second matmul).  The
+ *     RMSNorm row scale r is one scalar per row, so it commutes with the
+ *     second matmul and is applied in that GEMM's epilogue; the first GEMM's
+ *     epilogue only emits a partial RMS, which a light reduction kernel
+ *     combines; SwiGLU, cross-entropy and the backward pass get the same
+ *     treatment, and a block-local forward epilogue gives a block-local
+ *     backward.
+ *   - Section "Five kinds of building blocks": elementwise transforms
+ *     (residual add, activation), vector loads (RMSNorm weight broadcast),
+ *     matrix-block loads/stores (saving activations for the backward), chunk
+ *     reductions (local RMS, chunk log-sum-exp) and stateful transforms
+ *     (running max and sum-exp of online normalisation).
+ *
+ * Conventions (all calls):
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller; the library
+ *     never allocates, frees or keeps a pointer after the call returns.
+ *     Scratch space is passed in by the caller, sized by the *_workspace_size
+ *     queries.
+ *   - Tensors are dense row-major.  Weights are stored [in, out]; activations
+ *     [tokens, features].  bf16 tensors are passed as uint16_t bit patterns
+ *     (IEEE bfloat16); float tensors are fp32; labels are int64.
+ *   - Every tensor base pointer must be 16-byte aligned.  M (tokens) may be any
+ *     value >= 0 (M == 0 is a no-op); feature sizes N, K, F, V must be > 0 and
+ *     multiples of 8 (the tensor-memory-access copies need 16-byte rows).
+ *   - Outputs must not alias inputs unless a call says otherwise.
+ *   - Each call enqueues its kernels on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and returns without synchronising.  Calls are
+ *     reentrant and keep no state between calls, except the device status
+ *     word read by coda_poll_status().
+ *   - Arithmetic: bf16 inputs, fp32 accumulation in tensor memory, fp32
+ *     epilogue math, bf16 outputs rounded to nearest-even.
+ *   - Return value: CODA_OK, or an error.  Argument errors (NULL, SHAPE,
+ *     ALIGN, WORKSPACE) are detected on the host before any CUDA call and
+ *     nothing is launched.  CODA_ERR_DEVICE: the current device is not
+ *     compute capability 10.0 (B200).  CODA_ERR_LAUNCH: a CUDA runtime call
+ *     failed (the CUDA error is left for the caller to query).  Kernels never
+ *     trap: a wait that exceeds its time limit records CODA_ERR_DEVICE_TIMEOUT
+ *     in the device status word, which coda_poll_status() reports.
+ */
+#ifndef CODA_H_
+#define CODA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum coda_status_t {
+  CODA_OK = 0,
+  CODA_ERR_NULL = 1,           /* a required pointer is NULL */
+  CODA_ERR_SHAPE = 2,          /* a size is negative, zero where it must not be, or not a multiple of 8 */
+  CODA_ERR_ALIGN = 3,          /* a pointer is not 16-byte aligned */
+  CODA_ERR_WORKSPACE = 4,      /* workspace missing or smaller than *_workspace_size */
+  CODA_ERR_DEVICE = 5,         /* no device, or not sm_100 */
+  CODA_ERR_LAUNCH = 6,         /* a CUDA runtime call failed */
+  CODA_ERR_DEVICE_TIMEOUT = 7, /* a kernel gave up on a bounded wait (from coda_poll_status) */
+  CODA_ERR_INTERNAL = 8        /* unexpected internal failure (e.g. tensor-map encoding) */
+} coda_status_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* coda_status_string(coda_status_t s);
+
+/* Library ABI version (increments on any signature change). */
+int coda_version(void);
+
+/* Column-tile width used by the partial-sum layouts (partial, pdr): 256. */
+int64_t coda_partial_tile_width(void);
+
+/* Number of column tiles T = ceil(N / coda_partial_tile_width()) for a hidden
+ * size N; partial and pdr arrays are [T, M] fp32 (tile-major: entry (t, i) at
+ * index t * M + i).  Returns -1 if N <= 0. */
+int64_t coda_partial_cols(int64_t N);
+
+/* Sets the time limit of every bounded device wait (nanoseconds, > 0;
+ * default 1e9).  Affects later launches only.  Returns CODA_ERR_SHAPE if <= 0. */
+coda_status_t coda_set_wait_limit_ns(int64_t ns);
+
+/* Synchronises `stream`, then reads and clears the device status word.
+ * Returns CODA_ERR_DEVICE_TIMEOUT if any kernel recorded a timeout since the
+ * last poll, CODA_ERR_LAUNCH if the stream reported a CUDA error, else CODA_OK. */
+coda_status_t coda_poll_status(void* stream);
+
+/* ---------------------------------------------------------------- forward */
+
+/* First GEMM of the block with the residual + partial-RMS epilogue
+ * (section "CODA: the secret in the epilogue": the first GEMM only computes a
+ * partial RMS while its output is on chip).
+ *   acc = x W (fp32);  h = acc + res (res may be NULL: h = acc);
+ *   h_out  = bf16(h)                     [M, N]  (NULL: not stored)
+ *   hg_out = bf16(gamma * h)             [M, N]  (NULL: not stored; needs gamma)
+ *   partial[t, i] = sum_{j in tile t} h_ij^2 (fp32, from the unrounded h) [T, M] (NULL: not stored)
+ * x [M, K] bf16, W [K, N] bf16, res [M, N] bf16, gamma [N] bf16.
+ * At least one output must be non-NULL.  Also used as the down projection of
+ * the SwiGLU chain (x = act, res = h, partials for the next layer's norm). */
+coda_status_t coda_gemm_res_partialrms(const uint16_t* x, const uint16_t* W, const uint16_t* res,
+                                       const uint16_t* gamma, uint16_t* h_out, uint16_t* hg_out, float* partial,
+                                       int64_t M, int64_t N, int64_t K, void* stream);
+
+/* The light reduction: r_i = 1 / sqrt(sum_t partial[t, i] / N + eps).
+ * partial [T, M] fp32 with T = coda_partial_cols(N); r_out [M] fp32; eps >= 0. */
+coda_status_t coda_rms_reduce(const float* partial, int64_t M, int64_t T, int64_t N, float eps, float* r_out,
+                              void* stream);
+
+/* Second GEMM with the RMSNorm row scale in its epilogue (r commutes with the
+ * matmul): out = bf16(r_i * (A W)_ij); r == NULL gives a plain bf16 GEMM.
+ * A [M, K] bf16 (hg of the first GEMM), W [K, N] bf16, r [M] fp32, out [M, N] bf16. */
+coda_status_t coda_gemm_rowscale(const uint16_t* A, const uint16_t* W, const float* r, uint16_t* out, int64_t M,
+                                 int64_t N, int64_t K, void* stream);
+
+/* Gate/up GEMM with SwiGLU in its epilogue (section "CODA: the secret in the
+ * epilogue" lists SwiGLU among the re-parameterised operations):
+ *   g = r_i (A W_gu[:, :F])_ij,  u = r_i (A W_gu[:, F:])_ij,  act = bf16(silu(g) * u)
+ * with silu(g) = g / (1 + exp(-g)).  The [M, 2F] gate/up product never reaches
+ * memory unless gateup_save is given (then bf16 g in columns [0, F) and u in
+ * [F, 2F) of gateup_save [M, 2F], for the backward).
+ * A [M, K] bf16, W_gu [K, 2F] bf16, r [M] fp32 or NULL (scale 1), act_out [M, F] bf16. */
+coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const float* r, uint16_t* act_out,
+                               uint16_t* gateup_save, int64_t M, int64_t F, int64_t K, void* stream);
+
+/* Bytes of workspace coda_lmhead_ce needs for M tokens and vocabulary V. */
+size_t coda_lmhead_ce_workspace_size(int64_t M, int64_t V);
+
+/* LM-head cross-entropy with a block log-sum-exp epilogue (section "Five kinds
+ * of building blocks": chunk log-sum-exp and the running max / sum-exp of
+ * online normalisation).  Logits z = r_i (H W)_ij (fp32, never stored; r NULL
+ * means scale 1).  Per token lse_i = log sum_j exp(z_ij), loss_i = lse_i -
+ * z_{i,label_i} (natural log); mean = sum_i loss_i / M.  A label outside
+ * [0, V) gives a NaN loss for that token (no device trap).
+ * H [M, K] bf16, W [K, V] bf16, labels [M] int64, loss_out/lse_out [M] fp32,
+ * mean_out [1] fp32 (may be NULL), ws >= coda_lmhead_ce_workspace_size(M, V). */
+coda_status_t coda_lmhead_ce(const uint16_t* H, const uint16_t* W, const int64_t* labels, const float* r,
+                             float* loss_out, float* lse_out, float* mean_out, void* ws, size_t ws_bytes,
+                             int64_t M, int64_t V, int64_t K, void* stream);
+
+/* ---------------------------------------------------------------- backward */
+
+/* Bytes of workspace coda_gemm_rowscale_bwd needs (holds y = r * hg, bf16 [M, N]). */
+size_t coda_gemm_rowscale_bwd_workspace_size(int64_t M, int64_t N);
+
+/* Backward of out = r * (hg W2) in block-local form.
+ *   P = dOut W2^T (fp32, on chip);  d_hg_out = r * P (fp32)           [M, N]
+ *   y = bf16(r * hg) (workspace);  pdr[t, i] = sum_{j in tile t} hg_ij P_ij   [T, M] fp32
+ *   dW2_out = y^T dOut (fp32)                                          [N, N2]
+ * dOut [M, N2] bf16, hg [M, N] bf16, W2 [N, N2] bf16, r [M] fp32.
+ * d_hg and pdr feed coda_rms_reduce_bwd. */
+coda_status_t coda_gemm_rowscale_bwd(const uint16_t* dOut, const uint16_t* hg, const uint16_t* W2, const float* r,
+                                     float* d_hg_out, float* dW2_out, float* pdr_out, void* ws, size_t ws_bytes,
+                                     int64_t M, int64_t N, int64_t N2, void* stream);
+
+/* Bytes of workspace coda_rms_reduce_bwd needs (per-row-block dgamma partials). */
+size_t coda_rms_reduce_bwd_workspace_size(int64_t M, int64_t N);
+
+/* RMSNorm backward row reduction:
+ *   dr_i = sum_t pdr[t, i];  coef_i = -r_i^3 dr_i / N;
+ *   dh_out = bf16(gamma * d_hg + coef_i * h)   [M, N]  (this is also dres)
+ *   dgamma_out_j = sum_i d_hg_ij h_ij           [N] fp32 (fixed summation order)
+ * pdr [T, M], r [M] fp32; d_hg [M, N] fp32; h [M, N] bf16; gamma [N] bf16.
+ * d_hg is kept in fp32 so that dh is rounded to bf16 only once. */
+coda_status_t coda_rms_reduce_bwd(const float* pdr, const float* r, const float* d_hg, const uint16_t* h,
+                                  const uint16_t* gamma, uint16_t* dh_out, float* dgamma_out, void* ws,
+                                  size_t ws_bytes, int64_t M, int64_t T, int64_t N, void* stream);
+
+/* Backward of h = x W1 + res: dx_out = bf16(dh W1^T) [M, K], dW1_out = x^T dh
+ * (fp32) [K, N]; dres equals dh.  dh [M, N] bf16, x [M, K] bf16, W1 [K, N] bf16.
+ * Either output may be NULL (not computed). */
+coda_status_t coda_gemm_res_partialrms_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* W1,
+                                           uint16_t* dx_out, float* dW1_out, int64_t M, int64_t N, int64_t K,
+                                           void* stream);
+
+/* ------------------------------------------------- unfused comparison chain */
+
+/* out = bf16(a + b), n elements (n a multiple of 8); the separate residual add
+ * of the unfused GEMM -> add -> RMSNorm -> GEMM chain. */
+coda_status_t coda_unfused_add(const uint16_t* a, const uint16_t* b, uint16_t* out, int64_t n, void* stream);
+
+/* Standalone RMSNorm of the unfused chain: y = bf16(gamma * h / sqrt(mean_j h_ij^2 + eps)),
+ * r_out [M] fp32 (may be NULL).  h, y [M, N] bf16; gamma [N] bf16. */
+coda_status_t coda_unfused_rmsnorm(const uint16_t* h, const uint16_t* gamma, float eps, uint16_t* y_out,
+                                   float* r_out, int64_t M, int64_t N, void* stream);
+
+/* ---------------------------------------------------------------- testing */
+
+/* Launches one block that waits on a barrier nothing ever signals, with time
+ * limit limit_ns.  The wait must give up: *gave_up_dev (device int) becomes 1
+ * and the device status word records a timeout (read it with
+ * coda_poll_status).  Used to test the bounded-wait path without a fault. */
+coda_status_t coda_selftest_bounded_wait(int64_t limit_ns, int* gave_up_dev, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CODA_H_ */

@@ -64,7 +64,7 @@ def as_f64(a) -> np.ndarray:
     a = np.asarray(a)
     if a.dtype == np.uint16:
         return bf16_to_f64(a)
-    return a.astype(np.float64)
+    return np.asarray(a, dtype=np.float64)
 
 
 def matmul(A, B) -> np.ndarray:
@@ -152,6 +152,28 @@ def rmsnorm_block_backward_unfused(x, res, W1, W2, gamma, eps: float, dOut) -> d
     dW1 = matmul(as_f64(x).T, dh)
     return {"dy": dy, "dW2": dW2, "dgamma": dgamma, "dh": dh, "dres": dh.copy(),
             "dx": dx, "dW1": dW1, "c": c, **f}
+
+
+def rmsnorm_block_backward_cols(x, res, W1, W2, gamma, eps: float, dOut, dW2_cols) -> dict:
+    """The same chain-rule backward as ``rmsnorm_block_backward_unfused``, with
+    dW2 evaluated only on the columns ``dW2_cols`` and without the forward
+    output (for full-size checks, where the whole dW2 = y^T dOut is too large
+    a product for a sampled test).  Every other gradient is complete."""
+    h = matmul(x, W1) + as_f64(res)
+    N = h.shape[1]
+    ms = (h * h).sum(axis=1) / N
+    r = 1.0 / np.sqrt(ms + eps)
+    g = as_f64(gamma)
+    y = g[None, :] * h * r[:, None]
+    dO = as_f64(dOut)
+    dy = matmul(dO, as_f64(W2).T)
+    cols = np.asarray(dW2_cols, dtype=np.int64)
+    dW2_cols_val = matmul(y.T, dO[:, cols])
+    dgamma = (dy * h * r[:, None]).sum(axis=0)
+    c = (dy * g[None, :] * h).sum(axis=1)
+    dh = r[:, None] * g[None, :] * dy - (r ** 3 / N)[:, None] * h * c[:, None]
+    return {"dW2_cols": dW2_cols_val, "dgamma": dgamma, "dh": dh, "dres": dh,
+            "dx": matmul(dh, as_f64(W1).T), "dW1": matmul(as_f64(x).T, dh), "h": h, "r": r}
 
 
 # ---------------------------------------------------------------------------

@@ -17,3 +17,26 @@ def pytest_configure(config):
 def oracle():
     from oracle import coda_oracle
     return coda_oracle
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """Write the measured error ratios of the parity checks (if any ran)."""
+    try:
+        from tests import _util
+    except Exception:
+        return
+    if not _util.RESULTS:
+        return
+    import json
+    out = os.path.join(ROOT, "gpurun_out")
+    if os.path.isdir(out):
+        path = os.path.join(out, "parity_errors.json")
+        prev = {}
+        if os.path.exists(path):
+            try:
+                prev = json.load(open(path))
+            except ValueError:
+                prev = {}
+        prev.update(_util.RESULTS)
+        with open(path, "w") as f:
+            json.dump(prev, f, indent=1, sort_keys=True)

@@ -1,0 +1,118 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel launched).
+
+The library must load, export every function include/coda.h declares, and
+reject bad arguments with the documented status codes before touching CUDA
+(the pointers below are fake and are never dereferenced).
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from gemm_epilogue_transformer_02_b200 import binding
+from gemm_epilogue_transformer_02_b200.build import build
+
+OK, NULL, SHAPE, ALIGN, WS, DEVICE = 0, 1, 2, 3, 4, 5
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.load_library()
+
+
+def declared_functions():
+    text = open(binding.HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(coda_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 20
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (coda_\w+)", out))
+    for n in names:
+        assert n in exported, n
+        assert hasattr(lib, n), n
+    # the binding declares a signature for every exported call
+    assert set(names) == set(binding._SIGS), set(names) ^ set(binding._SIGS)
+
+
+def test_status_strings_and_constants(lib):
+    for code in range(9):
+        s = lib.coda_status_string(code).decode()
+        assert s.startswith(binding.STATUS_NAMES[code])
+    assert lib.coda_status_string(99).decode() == "CODA_ERR_UNKNOWN"
+    assert lib.coda_version() >= 1
+    assert lib.coda_partial_tile_width() == 256
+    assert lib.coda_partial_cols(2048) == 8
+    assert lib.coda_partial_cols(512) == 2
+    assert lib.coda_partial_cols(520) == 3
+    assert lib.coda_partial_cols(0) == -1
+    assert lib.coda_lmhead_ce_workspace_size(8192, 128256) >= 2 * 501 * 8192 * 4 + 8192 * 4
+    assert lib.coda_gemm_rowscale_bwd_workspace_size(8192, 2048) >= 8192 * 2048 * 2
+    assert lib.coda_rms_reduce_bwd_workspace_size(8192, 2048) >= 256 * 2048 * 4
+    assert lib.coda_set_wait_limit_ns(0) == SHAPE
+    assert lib.coda_set_wait_limit_ns(1_000_000_000) == OK
+
+
+A = ctypes.c_void_p(0x10000)
+B = ctypes.c_void_p(0x20000)
+C = ctypes.c_void_p(0x30000)
+D = ctypes.c_void_p(0x40000)
+MIS = ctypes.c_void_p(0x30008)  # 8-byte aligned only
+
+
+def test_argument_errors_are_reported_before_any_launch(lib):
+    f = lib.coda_gemm_rowscale
+    assert f(None, B, None, C, 256, 512, 512, None) == NULL
+    assert f(A, B, None, None, 256, 512, 512, None) == NULL
+    assert f(A, B, None, C, -1, 512, 512, None) == SHAPE
+    assert f(A, B, None, C, 256, 500, 512, None) == SHAPE   # N not a multiple of 8
+    assert f(A, B, None, C, 256, 512, 0, None) == SHAPE
+    assert f(A, B, None, MIS, 256, 512, 512, None) == ALIGN
+    assert f(A, B, MIS, C, 256, 512, 512, None) == ALIGN
+    assert f(A, B, None, C, 0, 512, 512, None) == OK           # M == 0 is a no-op
+
+    g = lib.coda_gemm_res_partialrms
+    assert g(A, B, None, None, None, None, None, 16, 64, 64, None) == NULL   # no output
+    assert g(A, B, None, None, None, C, None, 16, 64, 64, None) == NULL      # hg needs gamma
+    assert g(A, B, C, D, C, MIS, None, 16, 64, 64, None) == ALIGN
+
+    assert lib.coda_rms_reduce(A, 16, 0, 64, 1e-6, B, None) == SHAPE
+    assert lib.coda_rms_reduce(A, 16, 1, 64, -1.0, B, None) == SHAPE
+
+    h = lib.coda_lmhead_ce
+    assert h(A, B, C, None, D, D, None, None, 0, 16, 64, 64, None) == WS
+    assert h(A, B, C, None, D, D, None, A, 16, 16, 64, 64, None) == WS
+    assert h(A, B, None, None, D, D, None, A, 1 << 20, 16, 64, 64, None) == NULL
+
+    k = lib.coda_gemm_rowscale_bwd
+    assert k(A, B, C, D, A, B, C, None, 0, 16, 64, 64, None) == WS
+    assert lib.coda_rms_reduce_bwd(A, B, C, D, A, B, C, None, 0, 16, 1, 64, None) == WS
+    assert lib.coda_gemm_res_partialrms_bwd(A, B, C, None, None, 16, 64, 64, None) == NULL
+    assert lib.coda_gemm_swiglu(A, B, None, C, MIS, 16, 64, 64, None) == ALIGN
+    assert lib.coda_unfused_add(A, B, C, 12, None) == SHAPE
+    assert lib.coda_unfused_rmsnorm(A, B, 1e-6, None, None, 16, 64, None) == NULL
+    assert lib.coda_selftest_bounded_wait(0, A, None) == SHAPE
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_arguments_without_a_gpu_report_device_error(lib):
+    assert lib.coda_gemm_rowscale(A, B, None, C, 256, 512, 512, None) == DEVICE
+    assert lib.coda_rms_reduce(A, 16, 1, 64, 1e-6, B, None) == DEVICE
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    x = torch.zeros(8, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.gemm_rowscale(x, x)
+
+
+def test_build_flags_target_sm100a():
+    src = open(os.path.join(os.path.dirname(binding.LIB_PATH), "build.py")).read()
+    assert "arch=compute_100a,code=sm_100a" in src

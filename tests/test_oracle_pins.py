@@ -340,3 +340,16 @@ def test_tolerance_helper():
     assert ok and math.isclose(rms, math.sqrt((1 + (1 - 0.019) ** 2) / 2))
     ok, _, _ = O.tolerance_ok(np.array([1.0, -1.0]), np.array([1.0, -1.0 + 0.03]))
     assert not ok
+
+
+def test_column_sampled_backward_equals_full_definition():
+    r = rng(17)
+    M, K, N, N2 = 9, 12, 16, 20
+    args = (r.normal(size=(M, K)), r.normal(size=(M, N)), r.normal(size=(K, N)), r.normal(size=(N, N2)),
+            1 + 0.1 * r.normal(size=N), 1e-6, r.normal(size=(M, N2)))
+    full = O.rmsnorm_block_backward_unfused(*args)
+    cols = np.array([0, 3, 19, 7])
+    part = O.rmsnorm_block_backward_cols(*args, cols)
+    np.testing.assert_array_equal(part["dW2_cols"], full["dW2"][:, cols])
+    for k in ("dgamma", "dh", "dres", "dx", "dW1"):
+        np.testing.assert_array_equal(part[k], full[k])
