@@ -55,6 +55,7 @@ _SIGS = {
     "coda_gemm_rowscale_bwd": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _P]),
     "coda_rms_reduce_bwd_workspace_size": (_SZ, [_I64, _I64]),
     "coda_rms_reduce_bwd": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _P]),
+    "coda_rms_reduce_bwd_noalloc": (_ST, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "coda_gemm_res_partialrms_bwd": (_ST, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "coda_unfused_add": (_ST, [_P, _P, _P, _I64, _P]),
     "coda_unfused_rmsnorm": (_ST, [_P, _P, _F, _P, _P, _I64, _I64, _P]),

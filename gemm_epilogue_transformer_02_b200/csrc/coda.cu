@@ -543,3 +543,83 @@ coda_status_t coda_selftest_bounded_wait(int64_t limit_ns, int* gave_up_dev, voi
 }
 
 }  // extern "C"
+
+// =========================================================================
+// RMSNorm backward with library-owned scratch (no allocation by anyone)
+// =========================================================================
+//
+// coda_rms_reduce_bwd needs a scratch buffer for its per-row-block dgamma
+// partials, which the caller normally allocates and passes in.  Some callers
+// cannot allocate device memory when they call: for example a serving or
+// training process that fixes its device-memory budget at start-up and may not
+// allocate afterwards, or a host framework that owns all device memory through
+// its own pool and has no way to hand out a workspace.  For them this variant
+// keeps the scratch in a fixed array inside the library's device image.
+//
+// The array below is one static device array of kNoAllocScratchFloats floats
+// (4 MiB), present on every GPU that loads this library until the process
+// exits.  It is shared by every call on a device and keeps whatever the last
+// call wrote; the kernels write every entry they later read, so nothing in it
+// has to start at zero.  Two calls whose kernels run at the same time on one
+// device (different streams, or different host threads) race on the array and
+// must be ordered by the caller.
+
+namespace {
+
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 20;
+
+float* g_noalloc_scratch[64] = {};  // per-device device address of the array
+
+}  // namespace
+
+static __device__ __align__(256) float g_coda_rms_bwd_scratch[kNoAllocScratchFloats];
+
+namespace {
+
+// Device address of the scratch array on device `dev` (which must be current).
+// The first call on a device looks it up; host code cannot use the array's
+// name as a device pointer.
+coda_status_t noalloc_scratch_on(int dev, float** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_noalloc_scratch[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_coda_rms_bwd_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return CODA_ERR_LAUNCH;
+    }
+    g_noalloc_scratch[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_scratch[dev];
+  return CODA_OK;
+}
+
+}  // namespace
+
+extern "C" coda_status_t coda_rms_reduce_bwd_noalloc(const float* pdr, const float* r, const float* d_hg,
+                                                     const uint16_t* h, const uint16_t* gamma, uint16_t* dh_out,
+                                                     float* dgamma_out, int64_t M, int64_t T, int64_t N,
+                                                     void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && T > 0 && T <= 1 << 20 && dim_ok(N), CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(pdr && r && d_hg && h && gamma && dh_out && dgamma_out, CODA_ERR_NULL);
+  CODA_CHECK(al16(pdr) && al16(r) && al16(d_hg) && al16(h) && al16(gamma) && al16(dh_out) && al16(dgamma_out),
+             CODA_ERR_ALIGN);
+  const int64_t nblk = (M + kBwdRows - 1) / kBwdRows;
+  CODA_CHECK(static_cast<uint64_t>(nblk) * static_cast<uint64_t>(N) <= kNoAllocScratchFloats, CODA_ERR_WORKSPACE);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  coda_status_t st = current_device(&dev, &info);
+  if (st != CODA_OK) return st;
+  float* part = nullptr;
+  st = noalloc_scratch_on(dev, &part);
+  if (st != CODA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  rms_reduce_bwd_kernel<<<static_cast<int>(nblk), kBwdThreads, 0, s>>>(
+      pdr, r, d_hg, reinterpret_cast<const __nv_bfloat16*>(h), reinterpret_cast<const __nv_bfloat16*>(gamma),
+      reinterpret_cast<__nv_bfloat16*>(dh_out), part, static_cast<int>(M), static_cast<int>(T), static_cast<int>(N));
+  if (cudaGetLastError() != cudaSuccess) return CODA_ERR_LAUNCH;
+  dgamma_final_kernel<<<static_cast<int>((N + 255) / 256), 256, 0, s>>>(part, static_cast<int>(nblk),
+                                                                        static_cast<int>(N), dgamma_out);
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}

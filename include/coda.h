@@ -168,6 +168,25 @@ coda_status_t coda_rms_reduce_bwd(const float* pdr, const float* r, const float*
                                   const uint16_t* gamma, uint16_t* dh_out, float* dgamma_out, void* ws,
                                   size_t ws_bytes, int64_t M, int64_t T, int64_t N, void* stream);
 
+/* Same computation as coda_rms_reduce_bwd, for callers that cannot allocate
+ * device memory at call time (a process whose device-memory budget is fixed
+ * at start-up, or a framework that owns all device memory in its own pool and
+ * cannot hand out a workspace).  It takes no workspace and allocates nothing:
+ * the dgamma partials live in one static device array of 2^20 floats (4 MiB)
+ * inside the library, held on every GPU that loads the library until the
+ * process exits.  Limit: ceil(M / 32) * N <= 2^20 (for example M = 8192 with
+ * N up to 4096); larger sizes return CODA_ERR_WORKSPACE and launch nothing.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls on a device share the array: calls whose kernels overlap on the
+ * GPU (other streams or threads) race and must be ordered by the caller.  The
+ * array keeps the last call's contents; nothing in it needs to start at zero.
+ * This entry point is a deployment convenience with no counterpart in the
+ * CODA article. */
+coda_status_t coda_rms_reduce_bwd_noalloc(const float* pdr, const float* r, const float* d_hg, const uint16_t* h,
+                                          const uint16_t* gamma, uint16_t* dh_out, float* dgamma_out, int64_t M,
+                                          int64_t T, int64_t N, void* stream);
+
 /* Backward of h = x W1 + res: dx_out = bf16(dh W1^T) [M, K], dW1_out = x^T dh
  * (fp32) [K, N]; dres equals dh.  dh [M, N] bf16, x [M, K] bf16, W1 [K, N] bf16.
  * Either output may be NULL (not computed). */
