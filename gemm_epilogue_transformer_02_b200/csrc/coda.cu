@@ -134,29 +134,82 @@ enum KernelKind : uint32_t {
   kKindF32MN,
 };
 
-template <int BN, int STAGES, bool A_MN, bool B_MN, class Epi>
-coda_status_t run_gemm(DevInfo* info, GemmParams<Epi>& p, int M, int N, int K, int n_nt, int group_m,
+// Pipeline depth of the pair kernels: as many 32 KB stages (this CTA's halves
+// of A and B) as fit next to the epilogue's shared memory, at most 8.
+template <class Epi>
+constexpr int pair_stages() {
+  constexpr int budget = 232448 - 1024 - 256 - kEpiWarps * Epi::kSmemPerWarp;
+  constexpr int st = budget / (2 * kBM * kBK * 2);
+  return st > 8 ? 8 : st;
+}
+
+struct KernelCache {
+  bool attr = false;
+  int max_clusters = 0;  // resident clusters of two CTAs (pair kernels)
+};
+KernelCache g_kcache[64][16];
+
+template <int BN, int STAGES, bool A_MN, bool B_MN, bool PAIR, class Epi>
+coda_status_t run_gemm(int dev, DevInfo* info, GemmParams<Epi>& p, int M, int N, int K, int n_nt, int group_m,
                        KernelKind kind, cudaStream_t stream) {
-  auto kern = coda_gemm_kernel<BN, STAGES, A_MN, B_MN, Epi>;
-  constexpr int smem = GemmSmem<BN, STAGES, Epi>::kBytes;
+  auto kern = coda_gemm_kernel<BN, STAGES, A_MN, B_MN, PAIR, Epi>;
+  constexpr int smem = GemmSmem<BN, STAGES, PAIR, Epi>::kBytes;
+  constexpr int kTileM = PAIR ? 2 * kBM : kBM;
+  KernelCache& kc = g_kcache[dev][kind];
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!(info->attr_set & (1u << kind))) {
+    if (!kc.attr) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return CODA_ERR_LAUNCH;
-      info->attr_set |= (1u << kind);
+      if (PAIR) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * (info->sms / 2), 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+          cudaGetLastError();
+          n = info->sms / 2;
+        }
+        kc.max_clusters = n;
+      }
+      kc.attr = true;
     }
   }
   p.M = M;
   p.N = N;
   p.K = K;
-  p.sched.n_mt = (M + kBM - 1) / kBM;
+  p.sched.n_mt = (M + kTileM - 1) / kTileM;
   p.sched.n_nt = n_nt;
   p.sched.group_m = group_m < 1 ? 1 : group_m;
   p.sched.ntiles = p.sched.n_mt * n_nt;
   p.wait_ns = static_cast<uint64_t>(g_wait_ns);
-  const int grid = p.sched.ntiles < info->sms ? p.sched.ntiles : info->sms;
-  kern<<<grid, kThreads, smem, stream>>>(p);
+  if (!PAIR) {
+    const int grid = p.sched.ntiles < info->sms ? p.sched.ntiles : info->sms;
+    kern<<<grid, kThreads, smem, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+  }
+  const int clusters = p.sched.ntiles < kc.max_clusters ? p.sched.ntiles : kc.max_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return CODA_ERR_LAUNCH;
   return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
 }
 
@@ -234,7 +287,7 @@ coda_status_t coda_gemm_res_partialrms(const uint16_t* x, const uint16_t* W, con
   }
   using Epi = EpiLoadStore2<0>;
   GemmParams<Epi> p{};
-  bool ok = map_a(&p.tmA, x, false, M, K) && map_b(&p.tmB, W, true, N, K, N, 256);
+  bool ok = map_a(&p.tmA, x, false, M, K) && map_b(&p.tmB, W, true, N, K, N, 128);
   if (res) ok = ok && map_out_bf16(&p.ep.tmIn, res, M, N, N);
   if (h_out) ok = ok && map_out_bf16(&p.ep.tmOut1, h_out, M, N, N);
   if (hg_out) ok = ok && map_out_bf16(&p.ep.tmOut2, hg_out, M, N, N);
@@ -246,7 +299,7 @@ coda_status_t coda_gemm_res_partialrms(const uint16_t* x, const uint16_t* W, con
   p.ep.has_out1 = h_out != nullptr;
   p.ep.has_out2 = hg_out != nullptr;
   const int n_nt = static_cast<int>((N + 255) / 256);
-  return run_gemm<256, 3, false, true, Epi>(info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), n_nt,
+  return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), n_nt,
                                             16, kKindResPartial, static_cast<cudaStream_t>(stream));
 }
 
@@ -281,12 +334,12 @@ coda_status_t coda_gemm_rowscale(const uint16_t* A, const uint16_t* W, const flo
   }
   using Epi = EpiRowScale;
   GemmParams<Epi> p{};
-  if (!(map_a(&p.tmA, A, false, M, K) && map_b(&p.tmB, W, true, N, K, N, 256) &&
+  if (!(map_a(&p.tmA, A, false, M, K) && map_b(&p.tmB, W, true, N, K, N, 128) &&
         map_out_bf16(&p.ep.tmOut, out, M, N, N)))
     return CODA_ERR_INTERNAL;
   p.ep.r = r;
   const int n_nt = static_cast<int>((N + 255) / 256);
-  return run_gemm<256, 4, false, true, Epi>(info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), n_nt,
+  return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), n_nt,
                                             16, kKindRowScale, static_cast<cudaStream_t>(stream));
 }
 
@@ -304,8 +357,8 @@ coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const fl
   }
   using Epi = EpiSwiGLU;
   GemmParams<Epi> p{};
-  bool ok = map_a(&p.tmA, A, false, M, K) && map_b(&p.tmB, W_gu, true, F, K, 2 * F, 256) &&
-            map_b(&p.tmB2, W_gu + F, true, F, K, 2 * F, 256) && map_out_bf16(&p.ep.tmAct, act_out, M, F, F);
+  bool ok = map_a(&p.tmA, A, false, M, K) && map_b(&p.tmB, W_gu, true, F, K, 2 * F, 128) &&
+            map_b(&p.tmB2, W_gu + F, true, F, K, 2 * F, 128) && map_out_bf16(&p.ep.tmAct, act_out, M, F, F);
   if (gateup_save)
     ok = ok && map_out_bf16(&p.ep.tmSaveG, gateup_save, M, F, 2 * F) &&
          map_out_bf16(&p.ep.tmSaveU, gateup_save + F, M, F, 2 * F);
@@ -313,7 +366,7 @@ coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const fl
   p.ep.r = r;
   p.ep.has_save = gateup_save != nullptr;
   const int n_nt = static_cast<int>((F + 127) / 128);
-  return run_gemm<256, 3, false, true, Epi>(info, p, static_cast<int>(M), static_cast<int>(F), static_cast<int>(K), n_nt,
+  return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(F), static_cast<int>(K), n_nt,
                                             16, kKindSwiGLU, static_cast<cudaStream_t>(stream));
 }
 
@@ -339,7 +392,7 @@ coda_status_t coda_lmhead_ce(const uint16_t* H, const uint16_t* W, const int64_t
   }
   using Epi = EpiCE;
   GemmParams<Epi> p{};
-  if (!(map_a(&p.tmA, H, false, M, K) && map_b(&p.tmB, W, true, V, K, V, 256))) return CODA_ERR_INTERNAL;
+  if (!(map_a(&p.tmA, H, false, M, K) && map_b(&p.tmB, W, true, V, K, V, 128))) return CODA_ERR_INTERNAL;
   const int n_nt = static_cast<int>((V + 255) / 256);
   uint8_t* w = static_cast<uint8_t*>(ws);
   p.ep.ws_m = reinterpret_cast<float*>(w);
@@ -349,7 +402,7 @@ coda_status_t coda_lmhead_ce(const uint16_t* H, const uint16_t* W, const int64_t
   p.ep.r = r;
   const int n_mt = static_cast<int>((M + kBM - 1) / kBM);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  coda_status_t st = run_gemm<256, 4, false, true, Epi>(info, p, static_cast<int>(M), static_cast<int>(V),
+  coda_status_t st = run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(V),
                                                         static_cast<int>(K), n_nt, n_mt, kKindCE, s);
   if (st != CODA_OK) return st;
   ce_combine_kernel<<<static_cast<int>((M + 31) / 32), 32 * kCombWarps, 0, s>>>(
@@ -391,7 +444,7 @@ coda_status_t coda_gemm_rowscale_bwd(const uint16_t* dOut, const uint16_t* hg, c
     // P = dOut W2^T with the block-local epilogue (d_hg, y, pdr).
     using Epi = EpiLoadStore2<1>;
     GemmParams<Epi> p{};
-    if (!(map_a(&p.tmA, dOut, false, M, N2) && map_b(&p.tmB, W2, false, N, N2, N2, 256) &&
+    if (!(map_a(&p.tmA, dOut, false, M, N2) && map_b(&p.tmB, W2, false, N, N2, N2, 128) &&
           map_out_bf16(&p.ep.tmIn, hg, M, N, N) && map_out_bf16(&p.ep.tmOut1, y, M, N, N) &&
           map_out_f32(&p.ep.tmOut2, d_hg_out, M, N)))
       return CODA_ERR_INTERNAL;
@@ -401,7 +454,7 @@ coda_status_t coda_gemm_rowscale_bwd(const uint16_t* dOut, const uint16_t* hg, c
     p.ep.has_in = 1;
     p.ep.has_out1 = 1;
     p.ep.has_out2 = 1;
-    coda_status_t st = run_gemm<256, 3, false, false, Epi>(info, p, static_cast<int>(M), static_cast<int>(N),
+    coda_status_t st = run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(N),
                                                            static_cast<int>(N2), static_cast<int>((N + 255) / 256),
                                                            16, kKindBwdP, s);
     if (st != CODA_OK) return st;
@@ -410,10 +463,10 @@ coda_status_t coda_gemm_rowscale_bwd(const uint16_t* dOut, const uint16_t* hg, c
     // dW2 = y^T dOut: A = y read transposed (MN-major), B = dOut (MN-major), K = tokens.
     using Epi = EpiStoreF32;
     GemmParams<Epi> p{};
-    if (!(map_a(&p.tmA, y, true, N, M) && map_b(&p.tmB, dOut, true, N2, M, N2, 256) &&
+    if (!(map_a(&p.tmA, y, true, N, M) && map_b(&p.tmB, dOut, true, N2, M, N2, 128) &&
           map_out_f32(&p.ep.tmOut, dW2_out, N, N2)))
       return CODA_ERR_INTERNAL;
-    return run_gemm<256, 4, true, true, Epi>(info, p, static_cast<int>(N), static_cast<int>(N2), static_cast<int>(M),
+    return run_gemm<256, pair_stages<Epi>(), true, true, true, Epi>(dev, info, p, static_cast<int>(N), static_cast<int>(N2), static_cast<int>(M),
                                              static_cast<int>((N2 + 255) / 256), 16, kKindF32MN, s);
   }
 }
@@ -468,11 +521,11 @@ coda_status_t coda_gemm_res_partialrms_bwd(const uint16_t* dh, const uint16_t* x
     // dx = dh W1^T: B = W1 read as [K rows of length N] (K-major), GEMM K = N.
     using Epi = EpiRowScale;
     GemmParams<Epi> p{};
-    if (!(map_a(&p.tmA, dh, false, M, N) && map_b(&p.tmB, W1, false, K, N, N, 256) &&
+    if (!(map_a(&p.tmA, dh, false, M, N) && map_b(&p.tmB, W1, false, K, N, N, 128) &&
           map_out_bf16(&p.ep.tmOut, dx_out, M, K, K)))
       return CODA_ERR_INTERNAL;
     p.ep.r = nullptr;
-    coda_status_t st = run_gemm<256, 4, false, false, Epi>(info, p, static_cast<int>(M), static_cast<int>(K),
+    coda_status_t st = run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(K),
                                                            static_cast<int>(N), static_cast<int>((K + 255) / 256),
                                                            16, kKindRowScaleKK, s);
     if (st != CODA_OK) return st;
@@ -481,10 +534,10 @@ coda_status_t coda_gemm_res_partialrms_bwd(const uint16_t* dh, const uint16_t* x
     // dW1 = x^T dh: A = x read transposed (MN-major), B = dh (MN-major), K = tokens.
     using Epi = EpiStoreF32;
     GemmParams<Epi> p{};
-    if (!(map_a(&p.tmA, x, true, K, M) && map_b(&p.tmB, dh, true, N, M, N, 256) &&
+    if (!(map_a(&p.tmA, x, true, K, M) && map_b(&p.tmB, dh, true, N, M, N, 128) &&
           map_out_f32(&p.ep.tmOut, dW1_out, K, N)))
       return CODA_ERR_INTERNAL;
-    return run_gemm<256, 4, true, true, Epi>(info, p, static_cast<int>(K), static_cast<int>(N), static_cast<int>(M),
+    return run_gemm<256, pair_stages<Epi>(), true, true, true, Epi>(dev, info, p, static_cast<int>(K), static_cast<int>(N), static_cast<int>(M),
                                              static_cast<int>((N + 255) / 256), 16, kKindF32MN, s);
   }
   return CODA_OK;

@@ -76,10 +76,10 @@ struct TileCtx {
   uint64_t* wbars;   // this warp's epilogue mbarriers
 };
 
-template <int BN, int STAGES, class Epi>
+template <int BN, int STAGES, bool PAIR, class Epi>
 struct GemmSmem {
-  static constexpr int kABytes = kBM * kBK * 2;
-  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kABytes = kBM * kBK * 2;                     // this CTA's 128 rows of A
+  static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * kBK * 2;    // this CTA's columns of B
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kEpiBytes = kEpiWarps * Epi::kSmemPerWarp;
   static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1 + kEpiWarps * Epi::kBarsPerWarp;
@@ -94,11 +94,20 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
   (void)mbar_wait(bar, parity, w);
 }
 
-template <int BN, int STAGES, bool A_MN, bool B_MN, class Epi>
+// PAIR = false: one CTA per 128 x BN tile (tcgen05 cta_group::1).
+// PAIR = true: a cluster of two CTAs per 256 x BN tile (cta_group::2); CTA
+// rank r owns accumulator rows [128 r, 128 r + 128) of the tile and loads its
+// own 128 rows of A and its own BN/2 columns of B.  Rank 0 issues the MMAs,
+// waits for both CTAs' copies on its full barriers (the copies of rank 1
+// complete there), and its commits arrive on the barriers of both CTAs.
+template <int BN, int STAGES, bool A_MN, bool B_MN, bool PAIR, class Epi>
 __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_constant__ GemmParams<Epi> p) {
-  using S = GemmSmem<BN, STAGES, Epi>;
+  using S = GemmSmem<BN, STAGES, PAIR, Epi>;
   static_assert(BN % 64 == 0 && BN <= 256, "BN must be a multiple of 64, at most 256");
   static_assert(2 * BN == 512 || 2 * BN == 256 || 2 * BN == 128, "TMEM columns must be a power of two");
+  static_assert(!PAIR || BN == 256, "pair tiles are 256 x 256");
+  constexpr int kTileM = PAIR ? 2 * kBM : kBM;   // rows per tile
+  constexpr int kBCols = PAIR ? BN / 2 : BN;     // B columns loaded by this CTA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -116,6 +125,9 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int tile_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int tile_first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -124,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], kEpiWarps);
+      mbar_init(&tempty[a], PAIR ? 2 * kEpiWarps : kEpiWarps);
     }
     mbar_init(drain, 1);
     for (int i = 0; i < kEpiWarps * Epi::kBarsPerWarp; ++i) mbar_init(&ebars[i], 1);
@@ -137,11 +149,17 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
     if (Epi::kPairedB) tma_prefetch_desc(&p.tmB2);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, 2 * BN);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_holder, 2 * BN);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, 2 * BN);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync_all();  // the peer's barriers exist before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const WaitCtx w{abort_flag, p.wait_ns};
@@ -155,35 +173,63 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
       uint32_t phase = 0;
       long issued = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+      const uint32_t full0 = PAIR ? mapa_shared(smem_u32(full), 0) : 0u;  // rank 0's full[0]
+      for (int t = tile_first; ok && t < ntiles; t += tile_step) {
         int mb, nb;
         p.sched.map(t, mb, nb);
+        const int arow = mb * kTileM + static_cast<int>(rank) * kBM;  // first A row of this CTA
+        const int bcol = nb * BN + static_cast<int>(rank) * kBCols;   // first B column of this CTA
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, w)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
           uint8_t* a = sA + stage * S::kABytes;
           uint8_t* b = sB + stage * S::kBBytes;
-          if (!A_MN) {
-            tma_load_2d(a, &p.tmA, &full[stage], kb * kBK, mb * kBM);
-          } else {
+          if (PAIR) {
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * S::kStageBytes);
+            const uint32_t fb = full0 + stage * 8;
+            if (!A_MN) {
+              tma_load_2d_pair(a, &p.tmA, fb, kb * kBK, arow);
+            } else {
 #pragma unroll
-            for (int j = 0; j < kBM / 64; ++j)
-              tma_load_2d(a + j * (64 * kBK * 2), &p.tmA, &full[stage], mb * kBM + j * 64, kb * kBK);
-          }
-          if (!B_MN) {
-            tma_load_2d(b, &p.tmB, &full[stage], kb * kBK, nb * BN);
-          } else {
+              for (int j = 0; j < kBM / 64; ++j)
+                tma_load_2d_pair(a + j * (64 * kBK * 2), &p.tmA, fb, arow + j * 64, kb * kBK);
+            }
+            if (!B_MN) {
+              tma_load_2d_pair(b, &p.tmB, fb, kb * kBK, bcol);
+            } else if (Epi::kPairedB) {
+              // rank 0 holds the gate half, rank 1 the up half of the accumulator columns
+              const CUtensorMap* m = rank == 0 ? &p.tmB : &p.tmB2;
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j) {
-              if (Epi::kPairedB) {
-                const CUtensorMap* m = (j < BN / 128) ? &p.tmB : &p.tmB2;
-                const int col = nb * (BN / 2) + (j % (BN / 128)) * 64;
-                tma_load_2d(b + j * (64 * kBK * 2), m, &full[stage], col, kb * kBK);
-              } else {
-                tma_load_2d(b + j * (64 * kBK * 2), &p.tmB, &full[stage], nb * BN + j * 64, kb * kBK);
+              for (int j = 0; j < kBCols / 64; ++j)
+                tma_load_2d_pair(b + j * (64 * kBK * 2), m, fb, nb * (BN / 2) + j * 64, kb * kBK);
+            } else {
+#pragma unroll
+              for (int j = 0; j < kBCols / 64; ++j)
+                tma_load_2d_pair(b + j * (64 * kBK * 2), &p.tmB, fb, bcol + j * 64, kb * kBK);
+            }
+          } else {
+            mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+            if (!A_MN) {
+              tma_load_2d(a, &p.tmA, &full[stage], kb * kBK, arow);
+            } else {
+#pragma unroll
+              for (int j = 0; j < kBM / 64; ++j)
+                tma_load_2d(a + j * (64 * kBK * 2), &p.tmA, &full[stage], arow + j * 64, kb * kBK);
+            }
+            if (!B_MN) {
+              tma_load_2d(b, &p.tmB, &full[stage], kb * kBK, bcol);
+            } else {
+#pragma unroll
+              for (int j = 0; j < BN / 64; ++j) {
+                if (Epi::kPairedB) {
+                  const CUtensorMap* m = (j < BN / 128) ? &p.tmB : &p.tmB2;
+                  const int col = nb * (BN / 2) + (j % (BN / 128)) * 64;
+                  tma_load_2d(b + j * (64 * kBK * 2), m, &full[stage], col, kb * kBK);
+                } else {
+                  tma_load_2d(b + j * (64 * kBK * 2), &p.tmB, &full[stage], bcol + j * 64, kb * kBK);
+                }
               }
             }
           }
@@ -194,7 +240,10 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
           }
         }
       }
-      // Drain: every load issued must have landed before shared memory goes away.
+      // Drain: every load issued must have landed before shared memory goes
+      // away.  A single CTA sees its loads complete on its full barriers; in a
+      // pair they complete on rank 0's, so both CTAs wait for the MMA's release
+      // of each stage instead (it follows the completion of both halves).
       const long n = issued < STAGES ? issued : STAGES;
       for (long i = 0; i < n; ++i) {
         if (stage == 0) {
@@ -203,18 +252,18 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
         } else {
           --stage;
         }
-        drain_wait(&full[stage], phase, p.wait_ns);
+        drain_wait(PAIR ? &empty[stage] : &full[stage], phase, p.wait_ns);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, A_MN, B_MN);
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++it) {
+      for (int t = tile_first; ok && t < ntiles; t += tile_step, ++it) {
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         if (!mbar_wait(&tempty[acc], aph ^ 1u, w)) break;
@@ -234,19 +283,31 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
                                      : sdesc_sw128(a0 + kk * 32, 16, 1024);
             const uint64_t bd = B_MN ? sdesc_sw128(b0 + kk * 16 * 128, 64 * kBK * 2, 1024)
                                      : sdesc_sw128(b0 + kk * 32, 16, 1024);
-            tc_mma_bf16(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            if (PAIR)
+              tc_mma_bf16_pair(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            else
+              tc_mma_bf16(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
           }
-          tc_commit(&empty[stage]);
+          if (PAIR)
+            tc_commit_pair_mc(&empty[stage], 0x3);
+          else
+            tc_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(&tfull[acc]);
+        if (PAIR)
+          tc_commit_pair_mc(&tfull[acc], 0x3);
+        else
+          tc_commit(&tfull[acc]);
       }
       // All MMAs issued by this thread have completed once this arrives.
-      tc_commit(drain);
+      if (PAIR)
+        tc_commit_pair(drain);
+      else
+        tc_commit(drain);
       drain_wait(drain, 0, p.wait_ns);
     }
   } else {
@@ -255,10 +316,12 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
     const int ew = warp - 2;
     uint8_t* wsmem = sEpi + ew * Epi::kSmemPerWarp;
     uint64_t* wbars = ebars + ew * Epi::kBarsPerWarp;
+    // accumulator release goes to rank 0's barriers (where the MMA waits)
+    const uint32_t tempty0 = PAIR ? mapa_shared(smem_u32(tempty), 0) : 0u;
     typename Epi::State st;
     Epi::init_state(st);
     int it = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+    for (int t = tile_first; t < ntiles; t += tile_step, ++it) {
       int mb, nb;
       p.sched.map(t, mb, nb);
       const int acc = it & 1;
@@ -271,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
       c.N = p.N;
       c.mb = mb;
       c.nb = nb;
-      c.row0 = mb * kBM + q * 32;
+      c.row0 = mb * kTileM + static_cast<int>(rank) * kBM + q * 32;
       c.taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
       c.lane = lane;
       c.wsmem = wsmem;
@@ -279,7 +342,12 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
       const bool ok = Epi::template tile<BN>(p.ep, c, st, w);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if (PAIR)
+          mbar_arrive_cluster(tempty0 + acc * 8);
+        else
+          mbar_arrive(&tempty[acc]);
+      }
       if (!ok) break;
     }
     Epi::finish(p.ep, st, wbars, lane, p.wait_ns);
@@ -287,9 +355,13 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
 
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync_all();  // no CTA leaves while its peer may still signal it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * BN);
+    if (PAIR)
+      tmem_dealloc_pair(tmem_base, 2 * BN);
+    else
+      tmem_dealloc(tmem_base, 2 * BN);
   }
 }
 
