@@ -48,6 +48,7 @@ _SIGS = {
     "coda_gemm_res_partialrms": (_ST, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "coda_rms_reduce": (_ST, [_P, _I64, _I64, _I64, _F, _P, _P]),
     "coda_gemm_rowscale": (_ST, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "coda_gemm_rowscale_partial": (_ST, [_P, _P, _P, _I64, _I64, _F, _P, _P, _I64, _I64, _I64, _P]),
     "coda_gemm_swiglu": (_ST, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "coda_lmhead_ce_workspace_size": (_SZ, [_I64, _I64]),
     "coda_lmhead_ce": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _P]),
@@ -201,6 +202,24 @@ def gemm_rowscale(A, W, r=None, out=None):
     return out
 
 
+def gemm_rowscale_partial(A, W, partial, N_norm: int, eps: float, out=None, r_out=None):
+    """out = bf16(r * (A W)) with r = 1/sqrt(sum_t partial[t] / N_norm + eps)
+    formed in the epilogue; returns (out, r)."""
+    M, K = A.shape
+    N = W.shape[1]
+    T = partial.shape[0]
+    _need(A, BF16, "A")
+    _need(W, BF16, "W", (K, N))
+    _need(partial, F32, "partial", (T, M))
+    if out is None:
+        out = _empty((M, N), BF16, A)
+    if r_out is None:
+        r_out = _empty((M,), F32, A)
+    _call("coda_gemm_rowscale_partial", _ptr(A), _ptr(W), _ptr(partial), T, int(N_norm), float(eps), _ptr(r_out),
+          _ptr(out), M, N, K, _stream())
+    return out, r_out
+
+
 def gemm_swiglu(A, W_gu, r=None, save=False, act_out=None):
     """act = silu(r * A W_g) * (r * A W_u); returns (act, gateup or None)."""
     M, K = A.shape
@@ -328,16 +347,20 @@ def selftest_bounded_wait(limit_ns: int) -> int:
 # -------------------------------------------------- call sequences of the path
 
 
-def gemm_rmsnorm_gemm(x, res, W1, W2, gamma, eps: float, out=None, bufs=None):
-    """The fused block: first GEMM + residual + partial RMS, light reduction,
-    row-scaled second GEMM.  Returns dict(out, h, hg, partial, r)."""
-    M = x.shape[0]
+def gemm_rmsnorm_gemm(x, res, W1, W2, gamma, eps: float, out=None, bufs=None, fold_reduce=True):
+    """The fused block: first GEMM + residual + partial RMS, the light
+    reduction, and the row-scaled second GEMM.  With fold_reduce (default) the
+    reduction runs inside the second GEMM's epilogue (two launches); without
+    it, as its own kernel (three launches).  Returns dict(out, h, hg, partial, r)."""
     N = W1.shape[1]
     b = bufs or {}
     h, hg, partial = gemm_res_partialrms(x, W1, res, gamma, h_out=b.get("h"), hg_out=b.get("hg"),
                                          partial_out=b.get("partial"))
-    r = rms_reduce(partial, N, eps, r_out=b.get("r"))
-    out = gemm_rowscale(hg, W2, r, out=out)
+    if fold_reduce:
+        out, r = gemm_rowscale_partial(hg, W2, partial, N, eps, out=out, r_out=b.get("r"))
+    else:
+        r = rms_reduce(partial, N, eps, r_out=b.get("r"))
+        out = gemm_rowscale(hg, W2, r, out=out)
     return {"out": out, "h": h, "hg": hg, "partial": partial, "r": r}
 
 

@@ -143,6 +143,11 @@ constexpr int pair_stages() {
   return st > 8 ? 8 : st;
 }
 
+// Raster group of kAllRows: every M tile of a column block runs before the next
+// column block, so each weight column block is read from DRAM once while the
+// (smaller) activation operand stays resident in L2.
+constexpr int kAllRows = 1 << 30;
+
 struct KernelCache {
   bool attr = false;
   int max_clusters = 0;  // resident clusters of two CTAs (pair kernels)
@@ -188,7 +193,7 @@ coda_status_t run_gemm(int dev, DevInfo* info, GemmParams<Epi>& p, int M, int N,
   p.K = K;
   p.sched.n_mt = (M + kTileM - 1) / kTileM;
   p.sched.n_nt = n_nt;
-  p.sched.group_m = group_m < 1 ? 1 : group_m;
+  p.sched.group_m = group_m < 1 ? 1 : (group_m > p.sched.n_mt ? p.sched.n_mt : group_m);
   p.sched.ntiles = p.sched.n_mt * n_nt;
   p.wait_ns = static_cast<uint64_t>(g_wait_ns);
   if (!PAIR) {
@@ -288,14 +293,13 @@ coda_status_t coda_gemm_res_partialrms(const uint16_t* x, const uint16_t* W, con
   using Epi = EpiLoadStore2<0>;
   GemmParams<Epi> p{};
   bool ok = map_a(&p.tmA, x, false, M, K) && map_b(&p.tmB, W, true, N, K, N, 128);
-  if (res) ok = ok && map_out_bf16(&p.ep.tmIn, res, M, N, N);
   if (h_out) ok = ok && map_out_bf16(&p.ep.tmOut1, h_out, M, N, N);
   if (hg_out) ok = ok && map_out_bf16(&p.ep.tmOut2, hg_out, M, N, N);
   if (!ok) return CODA_ERR_INTERNAL;
+  p.ep.in = reinterpret_cast<const __nv_bfloat16*>(res);
   p.ep.gamma = reinterpret_cast<const __nv_bfloat16*>(gamma);
   p.ep.r = nullptr;
   p.ep.partial = partial;
-  p.ep.has_in = res != nullptr;
   p.ep.has_out1 = h_out != nullptr;
   p.ep.has_out2 = hg_out != nullptr;
   const int n_nt = static_cast<int>((N + 255) / 256);
@@ -340,7 +344,38 @@ coda_status_t coda_gemm_rowscale(const uint16_t* A, const uint16_t* W, const flo
   p.ep.r = r;
   const int n_nt = static_cast<int>((N + 255) / 256);
   return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), n_nt,
-                                            16, kKindRowScale, static_cast<cudaStream_t>(stream));
+                                            kAllRows, kKindRowScale, static_cast<cudaStream_t>(stream));
+}
+
+coda_status_t coda_gemm_rowscale_partial(const uint16_t* A, const uint16_t* W, const float* partial, int64_t T,
+                                         int64_t N_norm, float eps, float* r_out, uint16_t* out, int64_t M,
+                                         int64_t N, int64_t K, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(N) && dim_ok(K) && T > 0 && T <= 1 << 20 && N_norm > 0 &&
+                 eps >= 0.f,
+             CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(A && W && partial && out, CODA_ERR_NULL);
+  CODA_CHECK(al16(A) && al16(W) && al16(partial) && al16(r_out) && al16(out), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  using Epi = EpiRowScale;
+  GemmParams<Epi> p{};
+  if (!(map_a(&p.tmA, A, false, M, K) && map_b(&p.tmB, W, true, N, K, N, 128) &&
+        map_out_bf16(&p.ep.tmOut, out, M, N, N)))
+    return CODA_ERR_INTERNAL;
+  p.ep.r = nullptr;
+  p.ep.partial = partial;
+  p.ep.T = static_cast<int>(T);
+  p.ep.inv_n = 1.0f / static_cast<float>(N_norm);
+  p.ep.eps = eps;
+  p.ep.r_out = r_out;
+  const int n_nt = static_cast<int>((N + 255) / 256);
+  return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), n_nt,
+                                            kAllRows, kKindRowScale, static_cast<cudaStream_t>(stream));
 }
 
 coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const float* r, uint16_t* act_out,
@@ -367,7 +402,7 @@ coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const fl
   p.ep.has_save = gateup_save != nullptr;
   const int n_nt = static_cast<int>((F + 127) / 128);
   return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(F), static_cast<int>(K), n_nt,
-                                            16, kKindSwiGLU, static_cast<cudaStream_t>(stream));
+                                            kAllRows, kKindSwiGLU, static_cast<cudaStream_t>(stream));
 }
 
 size_t coda_lmhead_ce_workspace_size(int64_t M, int64_t V) {
@@ -445,13 +480,13 @@ coda_status_t coda_gemm_rowscale_bwd(const uint16_t* dOut, const uint16_t* hg, c
     using Epi = EpiLoadStore2<1>;
     GemmParams<Epi> p{};
     if (!(map_a(&p.tmA, dOut, false, M, N2) && map_b(&p.tmB, W2, false, N, N2, N2, 128) &&
-          map_out_bf16(&p.ep.tmIn, hg, M, N, N) && map_out_bf16(&p.ep.tmOut1, y, M, N, N) &&
+          map_out_bf16(&p.ep.tmOut1, y, M, N, N) &&
           map_out_f32(&p.ep.tmOut2, d_hg_out, M, N)))
       return CODA_ERR_INTERNAL;
+    p.ep.in = reinterpret_cast<const __nv_bfloat16*>(hg);
     p.ep.gamma = nullptr;
     p.ep.r = r;
     p.ep.partial = pdr_out;
-    p.ep.has_in = 1;
     p.ep.has_out1 = 1;
     p.ep.has_out2 = 1;
     coda_status_t st = run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(N),

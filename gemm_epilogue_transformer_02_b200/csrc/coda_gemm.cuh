@@ -74,6 +74,8 @@ struct TileCtx {
   int lane;
   uint8_t* wsmem;    // this warp's epilogue shared memory
   uint64_t* wbars;   // this warp's epilogue mbarriers
+  bool has_next;     // this CTA has another tile after this one
+  int nrow0, ncol0;  // first row of this warp / first column of that next tile
 };
 
 template <int BN, int STAGES, bool PAIR, class Epi>
@@ -339,6 +341,15 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
       c.lane = lane;
       c.wsmem = wsmem;
       c.wbars = wbars;
+      c.has_next = t + tile_step < ntiles;
+      c.nrow0 = 0;
+      c.ncol0 = 0;
+      if (c.has_next) {
+        int nmb, nnb;
+        p.sched.map(t + tile_step, nmb, nnb);
+        c.nrow0 = nmb * kTileM + static_cast<int>(rank) * kBM + q * 32;
+        c.ncol0 = nnb * BN;
+      }
       const bool ok = Epi::template tile<BN>(p.ep, c, st, w);
       tc_fence_before();
       __syncwarp();
@@ -382,13 +393,17 @@ __device__ __forceinline__ float acc_at(const uint32_t (&v0)[32], const uint32_t
 }
 
 // ---------------------------------------------------------------------------
-// Load one bf16 tile, store two tiles and a per-row partial sum.
+// Read one bf16 tile, store two tiles and a per-row partial sum.
 //   MODE 0 (first GEMM of the block, "GEMM-Residual-PartialRMS"):
 //     h = acc + res;  out1 = bf16(h);  out2 = hg = bf16(gamma * h);  partial += h^2
-//     (double-buffered: the residual of the next chunk loads while this one computes)
 //   MODE 1 (backward of the row-scaled second GEMM, acc = P = dOut W2^T):
 //     in = hg;  out1 = y = bf16(r * hg);  out2 = d_hg = r * P (fp32);  partial += hg * P
-//     (single-buffered: its mainloop is long enough to hide the epilogue)
+// The input tile is read straight into registers (each thread its own row,
+// 128 bytes per 64-column chunk) one chunk ahead, and the first chunk of the
+// next tile is requested before this tile's last chunk is processed, so its
+// latency hides behind the epilogue math.  Outputs are staged in shared
+// memory (128-byte swizzle) and written by TMA stores; MODE 0 double-buffers
+// the staging, MODE 1 (whose mainloop is long) uses one buffer.
 // partial is laid out [column tile][row] (fp32).
 // ---------------------------------------------------------------------------
 template <int MODE>
@@ -397,33 +412,43 @@ struct EpiLoadStore2 {
   static constexpr int kOut2Bytes = MODE == 0 ? 4096 : 8192;  // 32 x 64 bf16, or 32 x 64 fp32 as two 32 x 32 boxes
   static constexpr int kBufBytes = 4096 + kOut2Bytes;
   static constexpr int kSmemPerWarp = kNBuf * kBufBytes;
-  static constexpr int kBarsPerWarp = kNBuf;
+  static constexpr int kBarsPerWarp = 0;
   static constexpr bool kPairedB = false;
 
   struct Params {
-    CUtensorMap tmIn;    // [M, N] bf16, box 64 x 32
-    CUtensorMap tmOut1;  // [M, N] bf16, box 64 x 32
-    CUtensorMap tmOut2;  // [M, N] bf16 box 64 x 32 (MODE 0) or fp32 box 32 x 32 (MODE 1)
+    CUtensorMap tmOut1;          // [M, N] bf16, box 64 x 32
+    CUtensorMap tmOut2;          // [M, N] bf16 box 64 x 32 (MODE 0) or fp32 box 32 x 32 (MODE 1)
+    const __nv_bfloat16* in;     // [M, N]: res (MODE 0, may be null) or hg (MODE 1)
     const __nv_bfloat16* gamma;  // MODE 0 (may be null when out2 is not stored)
     const float* r;              // MODE 1
     float* partial;              // [T, M] or null
-    int has_in, has_out1, has_out2;
+    int has_out1, has_out2;
   };
 
   struct State {
-    uint32_t cnt;        // chunks processed by this warp (selects the buffer)
-    uint32_t phase[2];   // parity of the next completion of each input barrier
-    uint32_t pending;    // bit b set: a load into buffer b is in flight
+    uint32_t cnt;   // chunks processed by this warp (selects the staging buffer)
+    uint4 pre[8];   // prefetched input chunk (64 bf16 of this thread's row)
+    int pre_row, pre_col;  // which chunk `pre` holds (pre_col < 0: none)
   };
 
   __device__ static void init_state(State& s) {
     s.cnt = 0;
-    s.phase[0] = s.phase[1] = 0;
-    s.pending = 0;
+    s.pre_row = 0;
+    s.pre_col = -1;
+  }
+
+  __device__ static __forceinline__ void load_chunk(const Params& ep, int M, int N, int row, int col,
+                                                    uint4 (&v)[8]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      v[j] = make_uint4(0, 0, 0, 0);
+      if (ep.in != nullptr && row < M && col + j * 8 < N)
+        v[j] = __ldg(reinterpret_cast<const uint4*>(ep.in + static_cast<size_t>(row) * N + col + j * 8));
+    }
   }
 
   template <int BN>
-  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx& w) {
+  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
     const int col0 = c.nb * BN;
     const int row = c.row0 + c.lane;
     int nch = (c.N - col0 + 63) / 64;
@@ -431,55 +456,43 @@ struct EpiLoadStore2 {
     const bool rows_live = c.row0 < c.M;
     float rs = 1.f;
     if (MODE == 1) rs = (row < c.M) ? __ldg(ep.r + row) : 0.f;
-    const bool has_in = ep.has_in != 0;
 
-    auto buf_of = [&](uint32_t cnt) -> int { return kNBuf == 2 ? static_cast<int>(cnt & 1) : 0; };
-    auto issue = [&](int ch, int b) {
-      if (c.lane == 0) {
-        mbar_arrive_expect_tx(&c.wbars[b], 32 * 128);
-        tma_load_2d(c.wsmem + b * kBufBytes, &ep.tmIn, &c.wbars[b], col0 + ch * 64, c.row0);
-      }
-      st.pending |= (1u << b);
-    };
-
-    if (kNBuf == 2 && has_in && nch > 0) {
-      if (c.lane == 0) bulk_wait_read<1>();  // buffer cnt&1 was last stored two chunks ago
-      __syncwarp();
-      issue(0, buf_of(st.cnt));
-    }
+    if (st.pre_col != col0 || st.pre_row != row) load_chunk(ep, c.M, c.N, row, col0, st.pre);
     float ss = 0.f;
     for (int ch = 0; ch < nch; ++ch) {
-      const int b = buf_of(st.cnt);
+      const int cc = col0 + ch * 64;
+      uint4 cur[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) cur[j] = st.pre[j];
+      // request the next chunk (of this tile, or the first of the next tile)
+      if (ch + 1 < nch) {
+        load_chunk(ep, c.M, c.N, row, cc + 64, st.pre);
+        st.pre_row = row;
+        st.pre_col = cc + 64;
+      } else if (c.has_next) {
+        const int nrow = c.nrow0 + c.lane;
+        load_chunk(ep, c.M, c.N, nrow, c.ncol0, st.pre);
+        st.pre_row = nrow;
+        st.pre_col = c.ncol0;
+      } else {
+        st.pre_col = -1;
+      }
+      const int b = kNBuf == 2 ? static_cast<int>(st.cnt & 1) : 0;
       uint8_t* R = c.wsmem + b * kBufBytes;
       uint8_t* G = R + 4096;
-      if (kNBuf == 1) {
-        if (c.lane == 0) bulk_wait_read<0>();  // the previous chunk's stores have read the buffer
-        __syncwarp();
-        if (has_in) issue(ch, 0);
-      } else if (has_in) {
-        if (ch + 1 < nch) {
-          if (c.lane == 0) bulk_wait_read<0>();  // the other buffer's store must have read it
-          __syncwarp();
-          issue(ch + 1, b ^ 1);
-        }
-      } else {
-        if (c.lane == 0) bulk_wait_read<1>();
-        __syncwarp();
+      if (c.lane == 0) {
+        if (kNBuf == 2)
+          bulk_wait_read<1>();  // buffer b was last stored two chunks ago
+        else
+          bulk_wait_read<0>();
       }
+      __syncwarp();
       uint32_t v0[32], v1[32];
       tmem_ld64(c.taddr + ch * 64, v0, v1);
-      if (has_in) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&c.wbars[b], st.phase[b], w))) return false;
-        st.phase[b] ^= 1u;
-        st.pending &= ~(1u << b);
-      }
-      const int cc = col0 + ch * 64;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const uint32_t off = sw128_off(c.lane, j);
-        uint4 in4 = make_uint4(0, 0, 0, 0);
-        if (has_in) in4 = ld_shared_v4(R + off);
-        const uint32_t inw[4] = {in4.x, in4.y, in4.z, in4.w};
+        const uint32_t inw[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
         uint32_t o1[4];
         if (MODE == 0) {
           uint32_t o2[4];
@@ -538,9 +551,7 @@ struct EpiLoadStore2 {
     return true;
   }
 
-  __device__ static void finish(const Params& ep, State& st, uint64_t* wbars, int lane, uint64_t limit_ns) {
-    for (int b = 0; b < kNBuf; ++b)
-      if (st.pending & (1u << b)) drain_wait(&wbars[b], st.phase[b], limit_ns);
+  __device__ static void finish(const Params&, State&, uint64_t*, int lane, uint64_t) {
     if (lane == 0) bulk_wait_all<0>();
     __syncwarp();
   }
@@ -548,7 +559,11 @@ struct EpiLoadStore2 {
 
 // ---------------------------------------------------------------------------
 // Row-scaled bf16 output: out = r * acc (r null: out = acc).  The second GEMM
-// of the block applies the RMSNorm row scale here.
+// of the block applies the RMSNorm row scale here.  With `partial` given, the
+// epilogue also does the light reduction itself: each thread sums its row's
+// T partial sums of squares (in the same order as the standalone reduction
+// kernel) and forms r = 1 / sqrt(sum / N + eps); the tiles of column block 0
+// write r out for the backward.
 // ---------------------------------------------------------------------------
 struct EpiRowScale {
   static constexpr int kSmemPerWarp = 2 * 4096;
@@ -556,8 +571,12 @@ struct EpiRowScale {
   static constexpr bool kPairedB = false;
 
   struct Params {
-    CUtensorMap tmOut;  // [M, N] bf16, box 64 x 32
-    const float* r;     // [M] or null
+    CUtensorMap tmOut;     // [M, N] bf16, box 64 x 32
+    const float* r;        // [M] or null
+    const float* partial;  // [T, M] partial sums of squares, or null
+    int T;
+    float inv_n, eps;
+    float* r_out;          // [M] or null (written when partial is given)
   };
   struct State {
     uint32_t cnt;
@@ -571,7 +590,17 @@ struct EpiRowScale {
     int nch = (c.N - col0 + 63) / 64;
     if (nch > BN / 64) nch = BN / 64;
     float rs = 1.f;
-    if (ep.r != nullptr) rs = (row < c.M) ? __ldg(ep.r + row) : 0.f;
+    if (ep.partial != nullptr) {
+      rs = 0.f;
+      if (row < c.M) {
+        float sum = 0.f;
+        for (int t = 0; t < ep.T; ++t) sum += __ldg(ep.partial + static_cast<size_t>(t) * c.M + row);
+        rs = rsqrtf(sum * ep.inv_n + ep.eps);
+        if (ep.r_out != nullptr && c.nb == 0) ep.r_out[row] = rs;
+      }
+    } else if (ep.r != nullptr) {
+      rs = (row < c.M) ? __ldg(ep.r + row) : 0.f;
+    }
     for (int ch = 0; ch < nch; ++ch) {
       uint8_t* O = c.wsmem + (st.cnt & 1) * 4096;
       if (c.lane == 0) bulk_wait_read<1>();

@@ -19,7 +19,6 @@ __global__ void rms_reduce_kernel(const float* __restrict__ partial, int M, int 
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= M) return;
   float s = 0.f;
-#pragma unroll 8
   for (int t = 0; t < T; ++t) s += __ldg(partial + static_cast<size_t>(t) * M + i);
   r[i] = rsqrtf(s * inv_n + eps);
 }

@@ -115,6 +115,17 @@ coda_status_t coda_rms_reduce(const float* partial, int64_t M, int64_t T, int64_
 coda_status_t coda_gemm_rowscale(const uint16_t* A, const uint16_t* W, const float* r, uint16_t* out, int64_t M,
                                  int64_t N, int64_t K, void* stream);
 
+/* Second GEMM with the light reduction folded into its epilogue: each output
+ * row's scale r_i = 1 / sqrt(sum_t partial[t, i] / N_norm + eps) is formed by
+ * the epilogue from the first GEMM's partials (same summation order as
+ * coda_rms_reduce, so the same r), then out = bf16(r_i * (A W)_ij).  r_out
+ * [M] fp32 (may be NULL) receives r for the backward.  One launch instead of
+ * two for the block's second half.  partial [T, M] fp32, A [M, K], W [K, N],
+ * out [M, N] bf16; N_norm is the hidden size the partials were taken over. */
+coda_status_t coda_gemm_rowscale_partial(const uint16_t* A, const uint16_t* W, const float* partial, int64_t T,
+                                         int64_t N_norm, float eps, float* r_out, uint16_t* out, int64_t M,
+                                         int64_t N, int64_t K, void* stream);
+
 /* Gate/up GEMM with SwiGLU in its epilogue (section "CODA: the secret in the
  * epilogue" lists SwiGLU among the re-parameterised operations):
  *   g = r_i (A W_gu[:, :F])_ij,  u = r_i (A W_gu[:, F:])_ij,  act = bf16(silu(g) * u)

@@ -82,6 +82,21 @@ def test_gemm_res_partialrms(M, K, N):
     C.poll_status()
 
 
+def test_gemm_rowscale_partial_folds_the_reduction():
+    g = gen(4)
+    M, K, N, Nn = 300, 200, 520, 776
+    T = C.partial_cols(Nn)
+    A = synth.normal_bf16(g, (M, K))
+    W = synth.normal_bf16(g, (K, N), std=1 / math.sqrt(K))
+    part = torch.rand(T, M, generator=g) * 300
+    out, r = C.gemm_rowscale_partial(dev(A), dev(W), dev(part), Nn, 1e-6)
+    r_ref = O.rms_reduce(part.double().numpy(), Nn, 1e-6)
+    check("out", out, O.gemm_rowscale(b(A), b(W), r_ref))
+    check_rel("r", r, r_ref, 1e-5)
+    # the same reduction as the standalone kernel: identical r
+    assert torch.equal(r, C.rms_reduce(dev(part), Nn, 1e-6))
+
+
 def test_rms_reduce():
     g = gen(3)
     M, N = 1000, 2048
@@ -93,10 +108,13 @@ def test_rms_reduce():
 
 # ----------------------------------------------------------- fused block
 
-def test_tiny_block_matches_unfused_definition():
-    """The tiny GEMM-RMSNorm-GEMM workload (256 tokens, 512 -> 1536)."""
+@pytest.mark.parametrize("fold", [True, False])
+def test_tiny_block_matches_unfused_definition(fold):
+    """The tiny GEMM-RMSNorm-GEMM workload (256 tokens, 512 -> 1536), with the
+    light reduction folded into the second GEMM or run as its own kernel."""
     inp = synth.tiny_block()
-    f = C.gemm_rmsnorm_gemm(dev(inp.x), dev(inp.res), dev(inp.W1), dev(inp.W2), dev(inp.gamma), inp.eps)
+    f = C.gemm_rmsnorm_gemm(dev(inp.x), dev(inp.res), dev(inp.W1), dev(inp.W2), dev(inp.gamma), inp.eps,
+                            fold_reduce=fold)
     ref = O.rmsnorm_block_unfused(b(inp.x), b(inp.res), b(inp.W1), b(inp.W2), b(inp.gamma), inp.eps)
     check("out", f["out"], ref["out"])
     check("h", f["h"], ref["h"])
