@@ -440,7 +440,7 @@ def run_ours(args):
                 "speedup_vs_unfused": None if ms_unfused is None else round(ms_unfused / ms_fused_il, 4),
                 "hbm_bytes_fused_alg": BYTES_FUSED, "hbm_bytes_unfused_alg": BYTES_UNFUSED,
                 "hbm_bytes_removed_alg": BYTES_UNFUSED - BYTES_FUSED,
-                "launches_fused": 3, "launches_unfused": 4,
+                "launches_fused": 2, "launches_unfused": 4,
             },
             "e2e": None if e2e_val is None else {
                 "value": round(e2e_val, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
