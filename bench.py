@@ -250,21 +250,18 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    ws, rank, local = dist_env()
-    if ws > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    else:
+    from gemm_epilogue_transformer_02_b200 import binding as C
+    from gemm_epilogue_transformer_02_b200 import dist as DD
+    from gemm_epilogue_transformer_02_b200 import synth
+
+    ws, rank, local = DD.init("nccl")
+    if ws == 1:
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
-
-    from gemm_epilogue_transformer_02_b200 import binding as C
-    from gemm_epilogue_transformer_02_b200 import synth
     C.load_library()
 
     # ---- inputs (seeded, synthetic; one batch per rank)
-    inp = synth.block_inputs(M_TOK, D, D, N2, seed=1 + 1000 * rank, w_std=0.02, with_down=True)
+    inp = synth.block_inputs(M_TOK, D, D, N2, seed=DD.rank_seed(1, rank), w_std=0.02, with_down=True)
     x, res, W1, W2, gamma = (t.to(dev) for t in (inp.x, inp.res, inp.W1, inp.W2, inp.gamma))
     W_down = inp.W_down.to(dev)
     h = torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev)
@@ -322,24 +319,19 @@ def run_ours(args):
     for _ in range(args.warmup):
         block()
     C.poll_status()
-    if ws > 1:
-        dist.barrier()
+    DD.barrier()
     torch.cuda.synchronize()
     if clock:
         clock.start()
     tot, parts = timed(block, args.steps, 0, inner_events=1)
     clocks = clock.stop() if clock else None
-    if ws > 1:
-        dist.barrier()
+    DD.barrier()
     torch.cuda.synchronize()
     C.poll_status()
     ms_block = sum(tot) / len(tot)
     k_ms = [sum(p[i] for p in parts) / len(parts) for i in range(2)]
-    t_max = torch.tensor([sum(tot)], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    total_s = t_max.item() / 1e3
-    value = ws * FLOPS_BLOCK * args.steps / total_s / 1e12
+    total_s = DD.max_over_ranks(sum(tot), dev) / 1e3
+    value = DD.weak_scaling_value(FLOPS_BLOCK, args.steps, total_s, ws) / 1e12
 
     # ---- unfused chain, same protocol
     # ---- fused vs unfused chain (and the three-launch block), interleaved
@@ -386,10 +378,7 @@ def run_ours(args):
             e2e_step()
         tot_e, _ = timed(e2e_step, e_steps, 0)
         ms_e2e = sum(tot_e) / len(tot_e)
-        e_max = torch.tensor([sum(tot_e)], dtype=torch.float64, device=dev)
-        if ws > 1:
-            dist.all_reduce(e_max, op=dist.ReduceOp.MAX)
-        e2e_val = ws * FLOPS_BLOCK * e_steps / (e_max.item() / 1e3) / 1e12
+        e2e_val = DD.weak_scaling_value(FLOPS_BLOCK, e_steps, DD.max_over_ranks(sum(tot_e), dev) / 1e3, ws) / 1e12
     h2d = 2 * (x_h.numel() + res_h.numel())
     d2h = 2 * out_h.numel()
     del x_h, res_h, out_h, x_d, res_d
@@ -400,8 +389,7 @@ def run_ours(args):
         path = time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma, h, hg, r, rank,
                          args.path_steps, timed)
 
-    if ws > 1:
-        dist.barrier()
+    DD.barrier()
     C.poll_status()
 
     if rank == 0:
@@ -452,9 +440,7 @@ def run_ours(args):
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline_obj()
         print(json.dumps(line), flush=True)
-    if ws > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    DD.shutdown()
     return 0
 
 
@@ -483,7 +469,7 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
     del act, h2, p2
 
     # fused LM-head cross-entropy (8192 x 2048 x 128256)
-    H, Wv, labels = synth.lmhead_ce_inputs(seed=3 + 1000 * rank)
+    H, Wv, labels = synth.lmhead_ce_inputs(seed=3 + 1000 * rank)  # rank's own tokens
     H, Wv, labels = H.to(dev), Wv.to(dev), labels.to(dev)
     ws_ce = torch.empty(C.lmhead_ce_workspace_size(M_TOK, V_CE), dtype=torch.uint8, device=dev)
 
