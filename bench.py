@@ -248,7 +248,6 @@ def run_reference(args):
 
 def run_ours(args):
     import torch
-    import torch.distributed as dist
 
     from gemm_epilogue_transformer_02_b200 import binding as C
     from gemm_epilogue_transformer_02_b200 import dist as DD
