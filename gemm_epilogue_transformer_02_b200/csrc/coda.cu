@@ -143,10 +143,18 @@ constexpr int pair_stages() {
   return st > 8 ? 8 : st;
 }
 
-// Raster group of kAllRows: every M tile of a column block runs before the next
-// column block, so each weight column block is read from DRAM once while the
-// (smaller) activation operand stays resident in L2.
+// Raster order.  The tiles that run at the same time should share the operand
+// that stays resident in L2, so that the other operand streams from DRAM once:
+//   A (M x K) no larger than B (K x N): every M tile of a column block runs
+//     before the next column block (group = all rows): A stays resident and
+//     each column block of B is read once;
+//   otherwise row-major order (group = 1): B stays resident and each row
+//     block of A is read once.
 constexpr int kAllRows = 1 << 30;
+
+inline int raster_group(int64_t M, int64_t N, int64_t K) {
+  return (M * K <= N * K) ? kAllRows : 1;
+}
 
 struct KernelCache {
   bool attr = false;
@@ -304,7 +312,7 @@ coda_status_t coda_gemm_res_partialrms(const uint16_t* x, const uint16_t* W, con
   p.ep.has_out2 = hg_out != nullptr;
   const int n_nt = static_cast<int>((N + 255) / 256);
   return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), n_nt,
-                                            16, kKindResPartial, static_cast<cudaStream_t>(stream));
+      raster_group(M, N, K), kKindResPartial, static_cast<cudaStream_t>(stream));
 }
 
 coda_status_t coda_rms_reduce(const float* partial, int64_t M, int64_t T, int64_t N, float eps, float* r_out,
@@ -344,7 +352,7 @@ coda_status_t coda_gemm_rowscale(const uint16_t* A, const uint16_t* W, const flo
   p.ep.r = r;
   const int n_nt = static_cast<int>((N + 255) / 256);
   return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), n_nt,
-                                            kAllRows, kKindRowScale, static_cast<cudaStream_t>(stream));
+      raster_group(M, N, K), kKindRowScale, static_cast<cudaStream_t>(stream));
 }
 
 coda_status_t coda_gemm_rowscale_partial(const uint16_t* A, const uint16_t* W, const float* partial, int64_t T,
@@ -375,7 +383,7 @@ coda_status_t coda_gemm_rowscale_partial(const uint16_t* A, const uint16_t* W, c
   p.ep.r_out = r_out;
   const int n_nt = static_cast<int>((N + 255) / 256);
   return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), n_nt,
-                                            kAllRows, kKindRowScale, static_cast<cudaStream_t>(stream));
+      raster_group(M, N, K), kKindRowScale, static_cast<cudaStream_t>(stream));
 }
 
 coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const float* r, uint16_t* act_out,
@@ -402,7 +410,7 @@ coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const fl
   p.ep.has_save = gateup_save != nullptr;
   const int n_nt = static_cast<int>((F + 127) / 128);
   return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(F), static_cast<int>(K), n_nt,
-                                            kAllRows, kKindSwiGLU, static_cast<cudaStream_t>(stream));
+      raster_group(M, 2 * F, K), kKindSwiGLU, static_cast<cudaStream_t>(stream));
 }
 
 size_t coda_lmhead_ce_workspace_size(int64_t M, int64_t V) {
@@ -435,10 +443,9 @@ coda_status_t coda_lmhead_ce(const uint16_t* H, const uint16_t* W, const int64_t
   p.ep.zlab = reinterpret_cast<float*>(w + 2 * align256(static_cast<size_t>(n_nt) * M * 4));
   p.ep.labels = labels;
   p.ep.r = r;
-  const int n_mt = static_cast<int>((M + kBM - 1) / kBM);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   coda_status_t st = run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(V),
-                                                        static_cast<int>(K), n_nt, n_mt, kKindCE, s);
+                                                        static_cast<int>(K), n_nt, raster_group(M, V, K), kKindCE, s);
   if (st != CODA_OK) return st;
   ce_combine_kernel<<<static_cast<int>((M + 31) / 32), 32 * kCombWarps, 0, s>>>(
       p.ep.ws_m, p.ep.ws_s, p.ep.zlab, labels, static_cast<int>(M), n_nt, V, lse_out, loss_out);
@@ -491,7 +498,7 @@ coda_status_t coda_gemm_rowscale_bwd(const uint16_t* dOut, const uint16_t* hg, c
     p.ep.has_out2 = 1;
     coda_status_t st = run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(N),
                                                            static_cast<int>(N2), static_cast<int>((N + 255) / 256),
-                                                           16, kKindBwdP, s);
+                                                           raster_group(M, N, N2), kKindBwdP, s);
     if (st != CODA_OK) return st;
   }
   {
@@ -501,8 +508,8 @@ coda_status_t coda_gemm_rowscale_bwd(const uint16_t* dOut, const uint16_t* hg, c
     if (!(map_a(&p.tmA, y, true, N, M) && map_b(&p.tmB, dOut, true, N2, M, N2, 128) &&
           map_out_f32(&p.ep.tmOut, dW2_out, N, N2)))
       return CODA_ERR_INTERNAL;
-    return run_gemm<256, pair_stages<Epi>(), true, true, true, Epi>(dev, info, p, static_cast<int>(N), static_cast<int>(N2), static_cast<int>(M),
-                                             static_cast<int>((N2 + 255) / 256), 16, kKindF32MN, s);
+    return run_gemm<256, pair_stages<Epi>(), true, true, true, Epi>(dev, info, p, static_cast<int>(N), static_cast<int>(N2), static_cast<int>(M), static_cast<int>((N2 + 255) / 256),
+      raster_group(N, N2, M), kKindF32MN, s);
   }
 }
 
@@ -562,7 +569,7 @@ coda_status_t coda_gemm_res_partialrms_bwd(const uint16_t* dh, const uint16_t* x
     p.ep.r = nullptr;
     coda_status_t st = run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(K),
                                                            static_cast<int>(N), static_cast<int>((K + 255) / 256),
-                                                           16, kKindRowScaleKK, s);
+                                                           raster_group(M, K, N), kKindRowScaleKK, s);
     if (st != CODA_OK) return st;
   }
   if (dW1_out) {
@@ -572,8 +579,8 @@ coda_status_t coda_gemm_res_partialrms_bwd(const uint16_t* dh, const uint16_t* x
     if (!(map_a(&p.tmA, x, true, K, M) && map_b(&p.tmB, dh, true, N, M, N, 128) &&
           map_out_f32(&p.ep.tmOut, dW1_out, K, N)))
       return CODA_ERR_INTERNAL;
-    return run_gemm<256, pair_stages<Epi>(), true, true, true, Epi>(dev, info, p, static_cast<int>(K), static_cast<int>(N), static_cast<int>(M),
-                                             static_cast<int>((N + 255) / 256), 16, kKindF32MN, s);
+    return run_gemm<256, pair_stages<Epi>(), true, true, true, Epi>(dev, info, p, static_cast<int>(K), static_cast<int>(N), static_cast<int>(M), static_cast<int>((N + 255) / 256),
+      raster_group(K, N, M), kKindF32MN, s);
   }
   return CODA_OK;
 }
