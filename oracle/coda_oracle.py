@@ -83,6 +83,17 @@ def silu(v: np.ndarray) -> np.ndarray:
     return out
 
 
+def silu_grad(v: np.ndarray) -> np.ndarray:
+    """d silu / dv = s (1 + v (1 - s)) with s = 1 / (1 + exp(-v))."""
+    v = np.asarray(v, dtype=np.float64)
+    s = np.empty_like(v)
+    pos = v >= 0
+    s[pos] = 1.0 / (1.0 + np.exp(-v[pos]))
+    e = np.exp(v[~pos])
+    s[~pos] = e / (1.0 + e)
+    return s * (1.0 + v * (1.0 - s))
+
+
 # ---------------------------------------------------------------------------
 # 1. Unfused definitions
 # ---------------------------------------------------------------------------
@@ -111,6 +122,21 @@ def swiglu_down_unfused(y, W_gu, W_down, res) -> dict:
     a = silu(gate) * up
     h2 = matmul(a, W_down) + as_f64(res)
     return {"gate": gate, "up": up, "a": a, "h2": h2}
+
+
+def swiglu_mlp_backward_unfused(y, W_gu, W_down, res, d_h2) -> dict:
+    """Backward of h2 = (silu(y W_g) * (y W_u)) W_down + res for the loss
+    L = sum(d_h2 * h2), by the chain rule: d_a = d_h2 W_down^T;
+    dW_down = a^T d_h2; d_gate = d_a * up * silu'(gate); d_up = d_a * silu(gate);
+    dW_gu = y^T [d_gate | d_up]; d_y = [d_gate | d_up] W_gu^T; d_res = d_h2."""
+    f = swiglu_down_unfused(y, W_gu, W_down, res)
+    dH2 = as_f64(d_h2)
+    d_a = matmul(dH2, as_f64(W_down).T)
+    d_gate = d_a * f["up"] * silu_grad(f["gate"])
+    d_up = d_a * silu(f["gate"])
+    d_gu = np.hstack([d_gate, d_up])
+    return {"d_a": d_a, "d_gate": d_gate, "d_up": d_up, "dW_down": matmul(f["a"].T, dH2),
+            "dW_gu": matmul(as_f64(y).T, d_gu), "d_y": matmul(d_gu, as_f64(W_gu).T), "d_res": dH2.copy(), **f}
 
 
 def cross_entropy_unfused(H, W, labels) -> dict:
@@ -230,6 +256,17 @@ def gemm_swiglu(A, W_gu, r) -> dict:
     F = acc.shape[1] // 2
     g, u = acc[:, :F], acc[:, F:]
     return {"gate": g, "up": u, "act": silu(g) * u}
+
+
+def gemm_swiglu_bwd(d_out, W_down, gate, up) -> dict:
+    """SwiGLU backward in the down projection's dA GEMM epilogue: the product
+    d_act = d_out W_down^T meets the saved gate and up of the same tile, and
+    the epilogue emits d_gate = d_act * up * silu'(gate) and
+    d_up = d_act * silu(gate); d_act itself is not kept."""
+    d_act = matmul(d_out, as_f64(W_down).T)
+    g = as_f64(gate)
+    u = as_f64(up)
+    return {"d_act": d_act, "d_gate": d_act * u * silu_grad(g), "d_up": d_act * silu(g)}
 
 
 def lmhead_ce(H, W, labels, r=None, chunk_cols: int = 256) -> dict:

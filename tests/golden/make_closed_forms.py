@@ -22,6 +22,9 @@ def rows():
            "same with c = -3")
     yield ("silu_1", one / (one + (-one).exp()), "silu(1) = 1 / (1 + e^-1)")
     yield ("silu_m2", Decimal(-2) / (one + Decimal(2).exp()), "silu(-2) = -2 / (1 + e^2)")
+    sig2 = one / (one + Decimal(-2).exp())
+    yield ("silu_grad_2", sig2 * (one + 2 * (one - sig2)),
+           "silu'(2) = s (1 + 2 (1 - s)), s = 1 / (1 + e^-2)")
     yield ("ce_uniform_V128256", Decimal(128256).ln(),
            "cross-entropy with all logits equal (W = 0), V = 128256: loss = ln V")
     yield ("ce_uniform_V1000", Decimal(1000).ln(), "same with V = 1000")

@@ -353,3 +353,60 @@ def test_column_sampled_backward_equals_full_definition():
     np.testing.assert_array_equal(part["dW2_cols"], full["dW2"][:, cols])
     for k in ("dgamma", "dh", "dres", "dx", "dW1"):
         np.testing.assert_array_equal(part[k], full[k])
+
+
+# --------------------------------------------------------------- SwiGLU backward
+
+def test_silu_grad_closed_form_and_numerical_derivative():
+    g = golden()
+    v = O.silu_grad(np.array([0.0, 2.0]))
+    assert v[0] == 0.5
+    assert math.isclose(v[1], g["silu_grad_2"], rel_tol=1e-15)
+    z = np.linspace(-30, 30, 61)
+    h = 1e-6
+    num = (O.silu(z + h) - O.silu(z - h)) / (2 * h)
+    np.testing.assert_allclose(O.silu_grad(z), num, rtol=1e-7, atol=1e-9)
+
+
+def _swiglu_loss(y, Wgu, Wd, res, dh2):
+    return float((O.swiglu_down_unfused(y, Wgu, Wd, res)["h2"] * dh2).sum())
+
+
+def test_swiglu_mlp_backward_matches_finite_differences():
+    r = rng(18)
+    M, N, F = 3, 5, 4
+    y, Wgu, Wd, res = r.normal(size=(M, N)), r.normal(size=(N, 2 * F)) / 2, r.normal(size=(F, N)) / 2, \
+        r.normal(size=(M, N))
+    dh2 = r.normal(size=(M, N))
+    b = O.swiglu_mlp_backward_unfused(y, Wgu, Wd, res, dh2)
+    step = 1e-6
+    for arr, gname in ((y, "d_y"), (Wgu, "dW_gu"), (Wd, "dW_down"), (res, "d_res")):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            old = arr[idx]
+            arr[idx] = old + step
+            lp = _swiglu_loss(y, Wgu, Wd, res, dh2)
+            arr[idx] = old - step
+            lm = _swiglu_loss(y, Wgu, Wd, res, dh2)
+            arr[idx] = old
+            fd[idx] = (lp - lm) / (2 * step)
+        assert np.abs(fd - b[gname]).max() <= 1e-6 * np.abs(fd).max(), gname
+
+
+def test_swiglu_bwd_step_equals_chain_rule_and_brute_force():
+    r = rng(19)
+    M, N, F = 4, 6, 5
+    y, Wgu, Wd = r.normal(size=(M, N)), r.normal(size=(N, 2 * F)), r.normal(size=(F, N))
+    dh2 = r.normal(size=(M, N))
+    b = O.swiglu_mlp_backward_unfused(y, Wgu, Wd, np.zeros((M, N)), dh2)
+    st = O.gemm_swiglu_bwd(dh2, Wd, b["gate"], b["up"])
+    np.testing.assert_allclose(st["d_gate"], b["d_gate"], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(st["d_up"], b["d_up"], rtol=1e-13, atol=1e-14)
+    d_act = bf_matmul(dh2, Wd.T)
+    for i in range(M):
+        for j in range(F):
+            gv, uv = b["gate"][i, j], b["up"][i, j]
+            s = 1 / (1 + math.exp(-gv))
+            assert math.isclose(st["d_gate"][i, j], d_act[i, j] * uv * s * (1 + gv * (1 - s)), rel_tol=1e-11,
+                                abs_tol=1e-13)
+            assert math.isclose(st["d_up"][i, j], d_act[i, j] * gv * s, rel_tol=1e-11, abs_tol=1e-13)
