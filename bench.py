@@ -467,7 +467,31 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
     res["swiglu_down"] = {"ms": round(sum(tot) / len(tot), 4),
                           "gemm_swiglu_ms": round(k[0], 4), "gemm_swiglu_tflops": round(f_sw / k[0] / 1e9, 1),
                           "down_proj_ms": round(k[1], 4), "down_proj_tflops": round(f_dn / k[1] / 1e9, 1)}
-    del act, h2, p2
+
+    # SwiGLU backward: fused d_act epilogue -> d_gate|d_up, then d_y, dW_gu, dW_down
+    gu = torch.empty(M_TOK, N2, dtype=torch.bfloat16, device=dev)
+    C.gemm_swiglu(hg, W2, r, act_out=act, gateup_out=gu)
+    d_h2 = synth.block_backward_dout(M_TOK, D, seed=5 + 1000 * rank).to(dev)
+    d_gu = torch.empty(M_TOK, N2, dtype=torch.bfloat16, device=dev)
+
+    def swb(evs=None):
+        C.gemm_swiglu_bwd(d_h2, W_down, gu, out=d_gu)
+        if evs:
+            evs[0].record(stream)
+        C.gemm_res_partialrms_bwd(d_gu, hg, W2)
+        C.gemm_res_partialrms_bwd(d_h2, act, W_down, dx=False)
+
+    for _ in range(3):
+        swb(None)
+    tot, parts = timed(swb, steps, 0, inner_events=1)
+    k = [sum(p[i] for p in parts) / len(parts) for i in range(2)]
+    f_swb = 2.0 * M_TOK * F_SW * D
+    f_rest = 2 * 2.0 * M_TOK * D * N2 + 2.0 * M_TOK * F_SW * D
+    ms = sum(tot) / len(tot)
+    res["swiglu_backward"] = {"ms": round(ms, 4), "tflops": round((f_swb + f_rest) / ms / 1e9, 1),
+                              "gemm_swiglu_bwd_ms": round(k[0], 4),
+                              "gemm_swiglu_bwd_tflops": round(f_swb / k[0] / 1e9, 1)}
+    del act, h2, p2, gu, d_h2, d_gu
 
     # fused LM-head cross-entropy (8192 x 2048 x 128256)
     H, Wv, labels = synth.lmhead_ce_inputs(seed=3 + 1000 * rank)  # rank's own tokens

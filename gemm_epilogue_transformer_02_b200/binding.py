@@ -50,6 +50,7 @@ _SIGS = {
     "coda_gemm_rowscale": (_ST, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "coda_gemm_rowscale_partial": (_ST, [_P, _P, _P, _I64, _I64, _F, _P, _P, _I64, _I64, _I64, _P]),
     "coda_gemm_swiglu": (_ST, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "coda_gemm_swiglu_bwd": (_ST, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "coda_lmhead_ce_workspace_size": (_SZ, [_I64, _I64]),
     "coda_lmhead_ce": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _P]),
     "coda_gemm_rowscale_bwd_workspace_size": (_SZ, [_I64, _I64]),
@@ -220,8 +221,9 @@ def gemm_rowscale_partial(A, W, partial, N_norm: int, eps: float, out=None, r_ou
     return out, r_out
 
 
-def gemm_swiglu(A, W_gu, r=None, save=False, act_out=None):
-    """act = silu(r * A W_g) * (r * A W_u); returns (act, gateup or None)."""
+def gemm_swiglu(A, W_gu, r=None, save=False, act_out=None, gateup_out=None):
+    """act = silu(r * A W_g) * (r * A W_u); returns (act, gateup or None).
+    With save (or gateup_out given) the bf16 gate and up are kept for the backward."""
     M, K = A.shape
     F = W_gu.shape[1] // 2
     _need(A, BF16, "A")
@@ -230,9 +232,35 @@ def gemm_swiglu(A, W_gu, r=None, save=False, act_out=None):
         _need(r, F32, "r", (M,))
     if act_out is None:
         act_out = _empty((M, F), BF16, A)
-    gu = _empty((M, 2 * F), BF16, A) if save else None
+    gu = gateup_out
+    if gu is not None:
+        _need(gu, BF16, "gateup_out", (M, 2 * F))
+    elif save:
+        gu = _empty((M, 2 * F), BF16, A)
     _call("coda_gemm_swiglu", _ptr(A), _ptr(W_gu), _ptr(r), _ptr(act_out), _ptr(gu), M, F, K, _stream())
     return act_out, gu
+
+
+def gemm_swiglu_bwd(d_out, W_down, gateup, out=None):
+    """[d_gate | d_up] from d_act = d_out W_down^T and the saved gate/up."""
+    M, N = d_out.shape
+    F = W_down.shape[0]
+    _need(d_out, BF16, "d_out")
+    _need(W_down, BF16, "W_down", (F, N))
+    _need(gateup, BF16, "gateup", (M, 2 * F))
+    if out is None:
+        out = _empty((M, 2 * F), BF16, d_out)
+    _call("coda_gemm_swiglu_bwd", _ptr(d_out), _ptr(W_down), _ptr(gateup), _ptr(out), M, F, N, _stream())
+    return out
+
+
+def swiglu_mlp_backward(d_h2, y, W_gu, W_down, act, gateup):
+    """Backward of h2 = (silu(y W_g) * (y W_u)) W_down + res from the saved
+    gate/up and act: returns dict(d_gateup, d_y, dW_gu, dW_down, d_res)."""
+    d_gu = gemm_swiglu_bwd(d_h2, W_down, gateup)
+    d_y, dW_gu = gemm_res_partialrms_bwd(d_gu, y, W_gu)
+    _, dW_down = gemm_res_partialrms_bwd(d_h2, act, W_down, dx=False)
+    return {"d_gateup": d_gu, "d_y": d_y, "dW_gu": dW_gu, "dW_down": dW_down, "d_res": d_h2}
 
 
 def lmhead_ce_workspace_size(M: int, V: int) -> int:

@@ -132,6 +132,7 @@ enum KernelKind : uint32_t {
   kKindCE,
   kKindBwdP,
   kKindF32MN,
+  kKindSwiGLUBwd,
 };
 
 // Pipeline depth of the pair kernels: as many 32 KB stages (this CTA's halves
@@ -411,6 +412,32 @@ coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const fl
   const int n_nt = static_cast<int>((F + 127) / 128);
   return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(F), static_cast<int>(K), n_nt,
       raster_group(M, 2 * F, K), kKindSwiGLU, static_cast<cudaStream_t>(stream));
+}
+
+coda_status_t coda_gemm_swiglu_bwd(const uint16_t* d_out, const uint16_t* W_down, const uint16_t* gateup,
+                                   uint16_t* d_gateup_out, int64_t M, int64_t F, int64_t N, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(F) && dim_ok(N), CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(d_out && W_down && gateup && d_gateup_out, CODA_ERR_NULL);
+  CODA_CHECK(al16(d_out) && al16(W_down) && al16(gateup) && al16(d_gateup_out), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  using Epi = EpiSwiGLUBwd;
+  GemmParams<Epi> p{};
+  // d_act = d_out W_down^T: W_down [F, N] read as [F rows of length N] (K-major), GEMM K = N.
+  if (!(map_a(&p.tmA, d_out, false, M, N) && map_b(&p.tmB, W_down, false, F, N, N, 128) &&
+        map_out_bf16(&p.ep.tmDG, d_gateup_out, M, F, 2 * F) &&
+        map_out_bf16(&p.ep.tmDU, d_gateup_out + F, M, F, 2 * F)))
+    return CODA_ERR_INTERNAL;
+  p.ep.gu = reinterpret_cast<const __nv_bfloat16*>(gateup);
+  const int n_nt = static_cast<int>((F + 255) / 256);
+  return run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(
+      dev, info, p, static_cast<int>(M), static_cast<int>(F), static_cast<int>(N), n_nt, raster_group(M, F, N),
+      kKindSwiGLUBwd, static_cast<cudaStream_t>(stream));
 }
 
 size_t coda_lmhead_ce_workspace_size(int64_t M, int64_t V) {

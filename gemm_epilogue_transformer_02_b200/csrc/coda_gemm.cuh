@@ -778,6 +778,120 @@ struct EpiSwiGLU {
 };
 
 // ---------------------------------------------------------------------------
+// SwiGLU backward in the down projection's dA GEMM: acc = d_act = d_out W_down^T
+// for output columns j of this tile; the saved gate g and up u of the same
+// columns are read into registers and
+//   d_gate = d_act * u * silu'(g),  d_up = d_act * silu(g)
+// (silu'(g) = s (1 + g (1 - s)), s = 1 / (1 + exp(-g))) are written to the
+// [M, 2F] gradient (gate half, up half).  d_act never reaches memory.
+// ---------------------------------------------------------------------------
+struct EpiSwiGLUBwd {
+  static constexpr int kSmemPerWarp = 2 * 8192;  // double-buffered (d_gate 4 KB + d_up 4 KB)
+  static constexpr int kBarsPerWarp = 0;
+  static constexpr bool kPairedB = false;
+
+  struct Params {
+    CUtensorMap tmDG;           // gate view of d_gateup [M, F], row stride 2F, box 64 x 32
+    CUtensorMap tmDU;           // up view of d_gateup
+    const __nv_bfloat16* gu;    // saved [M, 2F]: gate columns [0, F), up columns [F, 2F)
+  };
+  struct State {
+    uint32_t cnt;
+  };
+  __device__ static void init_state(State& s) { s.cnt = 0; }
+
+  // 32 saved gate and 32 saved up values of this thread's row from column col.
+  __device__ static __forceinline__ void load32(const __nv_bfloat16* grow, bool live, int F, int col, uint4 (&g)[4],
+                                                uint4 (&u)[4]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      g[j] = make_uint4(0, 0, 0, 0);
+      u[j] = make_uint4(0, 0, 0, 0);
+      if (live && col + j * 8 < F) {
+        g[j] = __ldg(reinterpret_cast<const uint4*>(grow + col + j * 8));
+        u[j] = __ldg(reinterpret_cast<const uint4*>(grow + F + col + j * 8));
+      }
+    }
+  }
+
+  template <int BN>
+  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
+    const int col0 = c.nb * BN;
+    const int row = c.row0 + c.lane;
+    const int F = c.N;
+    int nch = (F - col0 + 63) / 64;
+    if (nch > BN / 64) nch = BN / 64;
+    const bool live = row < c.M;
+    const __nv_bfloat16* grow = ep.gu + static_cast<size_t>(live ? row : 0) * (2 * static_cast<size_t>(F));
+    // 32-column sub-chunks; the saved gate/up of the next sub-chunk are in
+    // flight while this one is computed
+    uint4 pg[4], pu[4];
+    load32(grow, live, F, col0, pg, pu);
+    for (int ch = 0; ch < nch; ++ch) {
+      const int cc = col0 + ch * 64;
+      uint8_t* DG = c.wsmem + (st.cnt & 1) * 8192;
+      uint8_t* DU = DG + 4096;
+      if (c.lane == 0) bulk_wait_read<1>();
+      __syncwarp();
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint4 gv[4], uv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          gv[j] = pg[j];
+          uv[j] = pu[j];
+        }
+        const int nxt = cc + hh * 32 + 32;
+        if (nxt < col0 + nch * 64) load32(grow, live, F, nxt, pg, pu);
+        uint32_t v[32];
+        tmem_ld32(c.taddr + ch * 64 + hh * 32, v);
+        tmem_ld_wait(v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t gw[4] = {gv[j].x, gv[j].y, gv[j].z, gv[j].w};
+          const uint32_t uw[4] = {uv[j].x, uv[j].y, uv[j].z, uv[j].w};
+          uint32_t og[4], ou[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float dg2[2], du2[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float da = __uint_as_float(v[j * 8 + 2 * e + h]);
+              const float g = h ? bf16hi(gw[e]) : bf16lo(gw[e]);
+              const float u = h ? bf16hi(uw[e]) : bf16lo(uw[e]);
+              const float sg = __fdividef(1.0f, 1.0f + __expf(-g));  // sigmoid; 0 when exp overflows
+              dg2[h] = da * u * (sg * (1.0f + g * (1.0f - sg)));
+              du2[h] = da * (g * sg);
+            }
+            og[e] = pack_bf16x2(dg2[0], dg2[1]);
+            ou[e] = pack_bf16x2(du2[0], du2[1]);
+          }
+          const uint32_t off = sw128_off(c.lane, hh * 4 + j);
+          st_shared_v4(DG + off, make_uint4(og[0], og[1], og[2], og[3]));
+          st_shared_v4(DU + off, make_uint4(ou[0], ou[1], ou[2], ou[3]));
+        }
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (c.lane == 0) {
+        if (c.row0 < c.M) {
+          tma_store_2d(&ep.tmDG, DG, cc, c.row0);
+          tma_store_2d(&ep.tmDU, DU, cc, c.row0);
+        }
+        bulk_commit();
+      }
+      ++st.cnt;
+    }
+    return true;
+  }
+
+  __device__ static void finish(const Params&, State&, uint64_t*, int lane, uint64_t) {
+    if (lane == 0) bulk_wait_all<0>();
+    __syncwarp();
+  }
+};
+
+// ---------------------------------------------------------------------------
 // LM-head cross-entropy: block log-sum-exp of the tile with an online
 // (running max, running sum-exp) state over 32-column chunks.  Logits stay in
 // fp32 registers and never reach memory.  Per (column tile, row) the tile's

@@ -136,6 +136,21 @@ coda_status_t coda_gemm_rowscale_partial(const uint16_t* A, const uint16_t* W, c
 coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const float* r, uint16_t* act_out,
                                uint16_t* gateup_save, int64_t M, int64_t F, int64_t K, void* stream);
 
+/* SwiGLU backward, block-local in the down projection's dA GEMM (section "CODA:
+ * the secret in the epilogue": the backward of a block-local epilogue is
+ * block-local too).  The GEMM forms d_act = d_out W_down^T tile by tile; its
+ * epilogue reads the saved gate g and up u of the same tile (gateup, as saved
+ * by coda_gemm_swiglu) and writes
+ *   d_gateup[:, j]     = bf16(d_act_j * u_j * silu'(g_j))   (gate half)
+ *   d_gateup[:, F + j] = bf16(d_act_j * silu(g_j))           (up half)
+ * with silu'(g) = s (1 + g (1 - s)), s = 1 / (1 + exp(-g)); d_act is not
+ * stored.  d_out [M, N] bf16 (gradient of the down projection's output),
+ * W_down [F, N] bf16, gateup and d_gateup_out [M, 2F] bf16.  The rest of the
+ * MLP backward are plain GEMMs: coda_gemm_res_partialrms_bwd(d_gateup, y, W_gu)
+ * gives d_y and dW_gu; with x = act it gives dW_down. */
+coda_status_t coda_gemm_swiglu_bwd(const uint16_t* d_out, const uint16_t* W_down, const uint16_t* gateup,
+                                   uint16_t* d_gateup_out, int64_t M, int64_t F, int64_t N, void* stream);
+
 /* Bytes of workspace coda_lmhead_ce needs for M tokens and vocabulary V. */
 size_t coda_lmhead_ce_workspace_size(int64_t M, int64_t V);
 

@@ -100,3 +100,22 @@ def test_block_backward(block):
     check("dres", g["dres"], ref["dres"])
     check("dx", g["dx"], ref["dx"])
     check("dW1", g["dW1"], ref["dW1"])
+
+
+def test_swiglu_backward_sampled_rows(block):
+    """SwiGLU backward on the SwiGLU-chain workload: d_h2 std 0.01 (seed 5)."""
+    inp, d, f = block
+    s = C.swiglu_down(f["hg"], f["r"], f["h"], d["W2"], d["W_down"], save=True)
+    d_h2 = synth.block_backward_dout(M, D, seed=5)
+    y = f["hg"]  # the gate/up GEMM's operand (r is applied in its epilogue)
+    d_gu = C.gemm_swiglu_bwd(dev(d_h2), d["W_down"], s["gateup"])
+    C.poll_status()
+    rows = sample_rows(24, M, 6)
+    u = O.rmsnorm_block_unfused(b(inp.x)[rows], b(inp.res)[rows], b(inp.W1), b(inp.W2), b(inp.gamma), inp.eps)
+    ref = O.swiglu_mlp_backward_unfused(u["y"], b(inp.W2), b(inp.W_down), u["h"], b(d_h2)[rows])
+    ri = torch.as_tensor(rows, device="cuda")
+    F = N2 // 2
+    # intermediates of a chain whose gate/up come from the bf16-stored hg (see the act check)
+    check("d_gate", d_gu[ri][:, :F], ref["d_gate"], rel=5e-2, storage_rounding=2.0 ** -7)
+    check("d_up", d_gu[ri][:, F:], ref["d_up"], rel=5e-2, storage_rounding=2.0 ** -7)
+    del y

@@ -296,3 +296,38 @@ def test_bounded_wait_gives_up_and_reports_timeout():
     C.poll_status()   # cleared
     # the context is still usable
     test_rms_reduce()
+
+
+# ------------------------------------------------------------ SwiGLU backward
+
+@pytest.mark.parametrize("M,N,F", [(300, 136, 200), (256, 512, 384)])
+def test_gemm_swiglu_bwd(M, N, F):
+    g = gen(500 + F)
+    d_out = synth.normal_bf16(g, (M, N))
+    W_down = synth.normal_bf16(g, (F, N), std=1 / math.sqrt(N))
+    gu = synth.normal_bf16(g, (M, 2 * F), std=1.5)
+    d_gu = C.gemm_swiglu_bwd(dev(d_out), dev(W_down), dev(gu))
+    ref = O.gemm_swiglu_bwd(b(d_out), b(W_down), b(gu)[:, :F], b(gu)[:, F:])
+    check("d_gate", d_gu[:, :F], ref["d_gate"])
+    check("d_up", d_gu[:, F:], ref["d_up"])
+
+
+def test_swiglu_mlp_backward_chain():
+    g = gen(31)
+    M, N, F = 260, 256, 320
+    y = synth.normal_bf16(g, (M, N))
+    W_gu = synth.normal_bf16(g, (N, 2 * F), std=1 / math.sqrt(N))
+    W_down = synth.normal_bf16(g, (F, N), std=1 / math.sqrt(F))
+    res = synth.normal_bf16(g, (M, N))
+    d_h2 = synth.normal_bf16(g, (M, N), std=0.01)
+    act, gu = C.gemm_swiglu(dev(y), dev(W_gu), None, save=True)
+    bw = C.swiglu_mlp_backward(dev(d_h2), dev(y), dev(W_gu), dev(W_down), act, gu)
+    C.poll_status()
+    ref = O.swiglu_mlp_backward_unfused(b(y), b(W_gu), b(W_down), b(res), b(d_h2))
+    # d_gate and d_up are intermediates built from the bf16-saved gate/up (a
+    # product of three factors, like act): looser bar; the chain's outputs keep it
+    check("d_gate", bw["d_gateup"][:, :F], ref["d_gate"], rel=5e-2, storage_rounding=2.0 ** -7)
+    check("d_up", bw["d_gateup"][:, F:], ref["d_up"], rel=5e-2, storage_rounding=2.0 ** -7)
+    check("d_y", bw["d_y"], ref["d_y"])
+    check("dW_gu", bw["dW_gu"], ref["dW_gu"])
+    check("dW_down", bw["dW_down"], ref["dW_down"])
