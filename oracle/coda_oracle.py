@@ -156,6 +156,23 @@ def cross_entropy_unfused(H, W, labels) -> dict:
     return {"z": z, "lse": lse, "loss": loss, "mean": loss.sum() / loss.shape[0]}
 
 
+def cross_entropy_backward_unfused(H, W, labels, d_loss=None) -> dict:
+    """Backward of the per-token losses loss_i = lse_i - z_i,label with z = H W,
+    for L = sum_i d_loss_i loss_i (d_loss defaults to 1/M: the mean):
+    G = d_loss_i (softmax(z)_i - onehot(label_i));  dH = G W^T;  dW = H^T G."""
+    z = matmul(H, W)
+    M, V = z.shape
+    m = z.max(axis=1)
+    p = np.exp(z - m[:, None])
+    p /= p.sum(axis=1)[:, None]
+    lab = np.asarray(labels, dtype=np.int64)
+    G = p.copy()
+    G[np.arange(M), lab] -= 1.0
+    dl = np.full(M, 1.0 / M) if d_loss is None else np.asarray(d_loss, dtype=np.float64)
+    G *= dl[:, None]
+    return {"G": G, "dH": matmul(G, as_f64(W).T), "dW": matmul(as_f64(H).T, G)}
+
+
 def rmsnorm_block_backward_unfused(x, res, W1, W2, gamma, eps: float, dOut) -> dict:
     """Backward of out = (gamma * h * r) W2 with h = x W1 + res, by the chain
     rule on the unfused definition, for the loss L = sum(dOut * out):
@@ -296,6 +313,37 @@ def lmhead_ce(H, W, labels, r=None, chunk_cols: int = 256) -> dict:
     zl[idx] = z[idx, lab[idx]]
     loss = lse - zl
     return {"lse": lse, "loss": loss, "mean": loss.sum() / M}
+
+
+def lmhead_ce_grad_chunk(H, W_chunk, labels, lse, col0: int, d_loss) -> np.ndarray:
+    """Block-local cross-entropy gradient of one vocabulary chunk: the logits
+    z = H W_chunk are recomputed and, with the forward's saved lse,
+    G = d_loss_i (exp(z - lse_i) - [col0 + j == label_i])."""
+    z = matmul(H, W_chunk)
+    M, Vc = z.shape
+    G = np.exp(z - np.asarray(lse, dtype=np.float64)[:, None])
+    lab = np.asarray(labels, dtype=np.int64) - col0
+    hit = (lab >= 0) & (lab < Vc)
+    G[np.nonzero(hit)[0], lab[hit]] -= 1.0
+    return G * np.asarray(d_loss, dtype=np.float64)[:, None]
+
+
+def lmhead_ce_bwd(H, W, labels, lse, d_loss=None, chunk_cols: int = 4096) -> dict:
+    """The chunked block-local backward: per vocabulary chunk, G_c from the
+    recomputed logits, dH += G_c W_c^T, dW_c = H^T G_c."""
+    Hf = as_f64(H)
+    Wf = as_f64(W)
+    M = Hf.shape[0]
+    V = Wf.shape[1]
+    dl = np.full(M, 1.0 / M) if d_loss is None else np.asarray(d_loss, dtype=np.float64)
+    dH = np.zeros_like(Hf)
+    dW = np.zeros_like(Wf)
+    for c0 in range(0, V, chunk_cols):
+        Wc = Wf[:, c0:c0 + chunk_cols]
+        G = lmhead_ce_grad_chunk(Hf, Wc, labels, lse, c0, dl)
+        dH += G @ Wc.T
+        dW[:, c0:c0 + chunk_cols] = Hf.T @ G
+    return {"dH": dH, "dW": dW}
 
 
 def gemm_rowscale_bwd(dOut, hg, W2, r, tile_cols: int) -> dict:
