@@ -507,7 +507,20 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
     f_ce = 2.0 * M_TOK * D * V_CE
     ms = sum(tot) / len(tot)
     res["lmhead_ce"] = {"ms": round(ms, 4), "tflops": round(f_ce / ms / 1e9, 1)}
-    del H, Wv, labels, ws_ce
+
+    # fused LM-head cross-entropy backward from the saved lse (three GEMMs per vocabulary chunk)
+    _, lse, _ = C.lmhead_ce(H, Wv, labels, ws=ws_ce)
+    ws_ceb = torch.empty(C.load_library().coda_lmhead_ce_bwd_workspace_size(M_TOK, V_CE), dtype=torch.uint8,
+                         device=dev)
+
+    def ceb():
+        C.lmhead_ce_bwd(H, Wv, labels, lse, ws=ws_ceb)
+
+    ceb()
+    tot, _ = timed(ceb, max(2, steps // 4), 0)
+    ms = sum(tot) / len(tot)
+    res["lmhead_ce_backward"] = {"ms": round(ms, 4), "tflops": round(3 * f_ce / ms / 1e9, 1)}
+    del H, Wv, labels, ws_ce, ws_ceb, lse
 
     # backward of the block (dOut std 0.01)
     dOut = synth.block_backward_dout(seed=4 + 1000 * rank).to(dev)

@@ -53,6 +53,8 @@ _SIGS = {
     "coda_gemm_swiglu_bwd": (_ST, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "coda_lmhead_ce_workspace_size": (_SZ, [_I64, _I64]),
     "coda_lmhead_ce": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _P]),
+    "coda_lmhead_ce_bwd_workspace_size": (_SZ, [_I64, _I64]),
+    "coda_lmhead_ce_bwd": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _P]),
     "coda_gemm_rowscale_bwd_workspace_size": (_SZ, [_I64, _I64]),
     "coda_gemm_rowscale_bwd": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _P]),
     "coda_rms_reduce_bwd_workspace_size": (_SZ, [_I64, _I64]),
@@ -285,6 +287,29 @@ def lmhead_ce(H, W, labels, r=None, ws=None):
     _call("coda_lmhead_ce", _ptr(H), _ptr(W), _ptr(labels), _ptr(r), _ptr(loss), _ptr(lse), _ptr(mean),
           _ptr(ws), ws.numel(), M, V, K, _stream())
     return loss, lse, mean
+
+
+def lmhead_ce_bwd(H, W, labels, lse, d_loss=None, r=None, ws=None):
+    """Backward of the fused cross-entropy from the saved lse; returns (dH, dW) fp32.
+    d_loss None weights every token by 1/M (the mean)."""
+    M, K = H.shape
+    V = W.shape[1]
+    _need(H, BF16, "H")
+    _need(W, BF16, "W", (K, V))
+    _need(labels, torch.int64, "labels", (M,))
+    _need(lse, F32, "lse", (M,))
+    if d_loss is not None:
+        _need(d_loss, F32, "d_loss", (M,))
+    if r is not None:
+        _need(r, F32, "r", (M,))
+    dH = _empty((M, K), F32, H)
+    dW = _empty((K, V), F32, H)
+    nb = int(load_library().coda_lmhead_ce_bwd_workspace_size(M, V))
+    if ws is None:
+        ws = _empty((max(nb, 16),), torch.uint8, H)
+    _call("coda_lmhead_ce_bwd", _ptr(H), _ptr(W), _ptr(labels), _ptr(lse), _ptr(d_loss), _ptr(r), _ptr(dH), _ptr(dW),
+          _ptr(ws), ws.numel(), M, V, K, _stream())
+    return dH, dW
 
 
 # ---------------------------------------------------------------- backward

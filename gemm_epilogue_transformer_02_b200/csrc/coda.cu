@@ -121,6 +121,9 @@ bool map_out_bf16(CUtensorMap* m, const void* p, uint64_t rows, uint64_t cols, u
 bool map_out_f32(CUtensorMap* m, const void* p, uint64_t rows, uint64_t cols) {
   return tmap2d(m, p, true, cols, rows, cols, 32, 32);
 }
+bool map_out_f32_ld(CUtensorMap* m, const void* p, uint64_t rows, uint64_t cols, uint64_t stride) {
+  return tmap2d(m, p, true, cols, rows, stride, 32, 32);
+}
 
 // ------------------------------------------------------------------ launch
 
@@ -133,7 +136,13 @@ enum KernelKind : uint32_t {
   kKindBwdP,
   kKindF32MN,
   kKindSwiGLUBwd,
+  kKindCEGrad,
+  kKindF32KK,
 };
+
+// Vocabulary columns per chunk of the cross-entropy backward: the chunk's
+// bf16 gradient (M x 4096) is written once and read by two GEMMs right after.
+constexpr int64_t kCEBwdChunk = 4096;
 
 // Pipeline depth of the pair kernels: as many 32 KB stages (this CTA's halves
 // of A and B) as fit next to the epilogue's shared memory, at most 8.
@@ -485,6 +494,89 @@ coda_status_t coda_lmhead_ce(const uint16_t* H, const uint16_t* W, const int64_t
 }
 
 // ----------------------------------------------------------------- backward
+
+size_t coda_lmhead_ce_bwd_workspace_size(int64_t M, int64_t V) {
+  if (M < 0 || V <= 0) return 0;
+  const int64_t vc = V < kCEBwdChunk ? V : kCEBwdChunk;
+  return align256(static_cast<size_t>(M) * static_cast<size_t>(vc) * 2) + align256(static_cast<size_t>(M) * 4);
+}
+
+coda_status_t coda_lmhead_ce_bwd(const uint16_t* H, const uint16_t* W, const int64_t* labels, const float* lse,
+                                 const float* d_loss, const float* r, float* dH_out, float* dW_out, void* ws,
+                                 size_t ws_bytes, int64_t M, int64_t V, int64_t K, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(V) && dim_ok(K), CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(H && W && labels && lse && dH_out && dW_out, CODA_ERR_NULL);
+  CODA_CHECK(al16(H) && al16(W) && al16(labels) && al16(lse) && al16(d_loss) && al16(r) && al16(dH_out) &&
+                 al16(dW_out) && al16(ws),
+             CODA_ERR_ALIGN);
+  CODA_CHECK(ws != nullptr && ws_bytes >= coda_lmhead_ce_bwd_workspace_size(M, V), CODA_ERR_WORKSPACE);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint16_t* G = static_cast<uint16_t*>(ws);
+  const int64_t vmax = V < kCEBwdChunk ? V : kCEBwdChunk;
+  float* resid = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(static_cast<size_t>(M) * vmax * 2));
+  for (int64_t c0 = 0; c0 < V; c0 += kCEBwdChunk) {
+    const int64_t vc = (V - c0) < kCEBwdChunk ? (V - c0) : kCEBwdChunk;
+    {
+      // G = d (exp(z - lse) - onehot) for z = r (H W[:, c0:c0+vc]), bf16 [M, vc]
+      using Epi = EpiCEGrad;
+      GemmParams<Epi> p{};
+      if (!(map_a(&p.tmA, H, false, M, K) && map_b(&p.tmB, W + c0, true, vc, K, V, 128) &&
+            map_out_bf16(&p.ep.tmG, G, M, vc, vc)))
+        return CODA_ERR_INTERNAL;
+      p.ep.labels = labels;
+      p.ep.lse = lse;
+      p.ep.d_loss = d_loss;
+      p.ep.r = r;
+      p.ep.scale = 1.0f / static_cast<float>(M);
+      p.ep.col_offset = c0;
+      p.ep.resid = resid;
+      const coda_status_t st = run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(
+          dev, info, p, static_cast<int>(M), static_cast<int>(vc), static_cast<int>(K),
+          static_cast<int>((vc + 255) / 256), raster_group(M, vc, K), kKindCEGrad, s);
+      if (st != CODA_OK) return st;
+    }
+    {
+      // dH (+)= G W[:, chunk]^T: B = the chunk of W read as [K rows of length vc] (K-major)
+      using Epi = EpiStoreF32;
+      GemmParams<Epi> p{};
+      if (!(map_a(&p.tmA, G, false, M, vc) && map_b(&p.tmB, W + c0, false, K, vc, V, 128) &&
+            map_out_f32(&p.ep.tmOut, dH_out, M, K)))
+        return CODA_ERR_INTERNAL;
+      p.ep.accum = c0 == 0 ? nullptr : dH_out;
+      p.ep.ld = K;
+      const coda_status_t st = run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(
+          dev, info, p, static_cast<int>(M), static_cast<int>(K), static_cast<int>(vc),
+          static_cast<int>((K + 255) / 256), raster_group(M, K, vc), kKindF32KK, s);
+      if (st != CODA_OK) return st;
+    }
+    {
+      // dW[:, chunk] = H^T G: A = H read transposed (MN-major), B = G (MN-major), K = tokens
+      using Epi = EpiStoreF32;
+      GemmParams<Epi> p{};
+      if (!(map_a(&p.tmA, H, true, K, M) && map_b(&p.tmB, G, true, vc, M, vc, 128) &&
+            map_out_f32_ld(&p.ep.tmOut, dW_out + c0, K, vc, V)))
+        return CODA_ERR_INTERNAL;
+      p.ep.accum = nullptr;
+      p.ep.ld = V;
+      const coda_status_t st = run_gemm<256, pair_stages<Epi>(), true, true, true, Epi>(
+          dev, info, p, static_cast<int>(K), static_cast<int>(vc), static_cast<int>(M),
+          static_cast<int>((vc + 255) / 256), raster_group(K, vc, M), kKindF32MN, s);
+      if (st != CODA_OK) return st;
+    }
+  }
+  // the label entries, exact: add back what the bf16 gradient dropped there
+  ce_bwd_label_fix_kernel<<<static_cast<int>(M), kFixThreads, 0, s>>>(
+      labels, resid, reinterpret_cast<const __nv_bfloat16*>(H), reinterpret_cast<const __nv_bfloat16*>(W), dH_out,
+      dW_out, static_cast<int>(M), static_cast<int>(K), V);
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}
 
 size_t coda_gemm_rowscale_bwd_workspace_size(int64_t M, int64_t N) {
   if (M < 0 || N <= 0) return 0;

@@ -641,7 +641,9 @@ struct EpiStoreF32 {
   static constexpr bool kPairedB = false;
 
   struct Params {
-    CUtensorMap tmOut;  // [M, N] fp32, box 32 x 32
+    CUtensorMap tmOut;   // [M, N] fp32, box 32 x 32
+    const float* accum;  // null, or the output itself: out = acc + out (accumulation over calls)
+    long long ld;        // row stride (elements) of `accum`
   };
   struct State {
     uint32_t cnt;
@@ -651,22 +653,42 @@ struct EpiStoreF32 {
   template <int BN>
   __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
     const int col0 = c.nb * BN;
+    const int row = c.row0 + c.lane;
     int nch = (c.N - col0 + 31) / 32;
     if (nch > BN / 32) nch = BN / 32;
     for (int ch = 0; ch < nch; ++ch) {
+      const int cc = col0 + ch * 32;
+      uint4 old[8];
+      if (ep.accum != nullptr) {
+        const float* src = ep.accum + static_cast<size_t>(row < c.M ? row : 0) * ep.ld + cc;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          old[j] = make_uint4(0, 0, 0, 0);
+          if (row < c.M && cc + 4 * j < c.N) old[j] = *reinterpret_cast<const uint4*>(src + 4 * j);
+        }
+      }
       uint8_t* O = c.wsmem + (st.cnt & 1) * 4096;
       if (c.lane == 0) bulk_wait_read<1>();
       __syncwarp();
       uint32_t v[32];
       tmem_ld32(c.taddr + ch * 32, v);
       tmem_ld_wait(v);
+      if (ep.accum != nullptr) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + __uint_as_float(old[j].x));
+          v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + __uint_as_float(old[j].y));
+          v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + __uint_as_float(old[j].z));
+          v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + __uint_as_float(old[j].w));
+        }
+      }
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         st_shared_v4(O + sw128_off(c.lane, j), make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
       fence_async_smem();
       __syncwarp();
       if (c.lane == 0) {
-        if (c.row0 < c.M) tma_store_2d(&ep.tmOut, O, col0 + ch * 32, c.row0);
+        if (c.row0 < c.M) tma_store_2d(&ep.tmOut, O, cc, c.row0);
         bulk_commit();
       }
       ++st.cnt;
@@ -963,6 +985,93 @@ struct EpiCE {
   }
 
   __device__ static void finish(const Params&, State&, uint64_t*, int, uint64_t) {}
+};
+
+// ---------------------------------------------------------------------------
+// Cross-entropy backward, block-local: the logits of one vocabulary chunk are
+// recomputed in the accumulator and, with the forward's saved log-sum-exp,
+// turned into the gradient
+//   G_ij = d_i (exp(z_ij - lse_i) - [col0 + j == label_i]),   z = r_i (H W_chunk)_ij
+// (d_i = d_loss_i, or `scale` for every token when d_loss is null), stored in
+// bf16 for the two GEMMs that consume the chunk (dH += G W_chunk^T and
+// dW_chunk = H^T G).  The logits themselves are never stored.
+// ---------------------------------------------------------------------------
+struct EpiCEGrad {
+  static constexpr int kSmemPerWarp = 2 * 4096;
+  static constexpr int kBarsPerWarp = 0;
+  static constexpr bool kPairedB = false;
+
+  struct Params {
+    CUtensorMap tmG;        // [M, Vc] bf16, box 64 x 32
+    const int64_t* labels;  // [M]
+    const float* lse;       // [M] from the forward
+    const float* d_loss;    // [M] or null
+    const float* r;         // [M] or null
+    float scale;            // weight of every token when d_loss is null (1/M: the mean)
+    float* resid;           // [M]: G - bf16(G) at each row's label entry (or null)
+    long long col_offset;   // vocabulary index of this chunk's column 0
+  };
+  struct State {
+    uint32_t cnt;
+  };
+  __device__ static void init_state(State& s) { s.cnt = 0; }
+
+  template <int BN>
+  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
+    constexpr float kL2E = 1.4426950408889634f;
+    const int col0 = c.nb * BN;
+    const int row = c.row0 + c.lane;
+    const bool live = row < c.M;
+    int nch = (c.N - col0 + 63) / 64;
+    if (nch > BN / 64) nch = BN / 64;
+    const float rs = (ep.r != nullptr && live) ? __ldg(ep.r + row) : 1.f;
+    const float lse2 = live ? __ldg(ep.lse + row) * kL2E : 0.f;
+    const float d = live ? (ep.d_loss != nullptr ? __ldg(ep.d_loss + row) : ep.scale) : 0.f;
+    const long long lab = live ? ep.labels[row] - ep.col_offset : -1;
+    for (int ch = 0; ch < nch; ++ch) {
+      const int cc = col0 + ch * 64;
+      uint8_t* O = c.wsmem + (st.cnt & 1) * 4096;
+      if (c.lane == 0) bulk_wait_read<1>();
+      __syncwarp();
+      uint32_t v0[32], v1[32];
+      tmem_ld64(c.taddr + ch * 64, v0, v1);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float gg[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int jj = j * 8 + 2 * e + h;
+            const float z = rs * acc_at(v0, v1, jj);
+            const float p = exp2f(fmaf(z, kL2E, -lse2));
+            const bool hit = lab == static_cast<long long>(cc + jj);
+            gg[h] = d * (p - (hit ? 1.0f : 0.0f));
+            if (hit && ep.resid != nullptr) {
+              // the label entry dominates its dW column: keep what bf16 rounding drops
+              ep.resid[row] = gg[h] - __bfloat162float(__float2bfloat16_rn(gg[h]));
+            }
+          }
+          o[e] = pack_bf16x2(gg[0], gg[1]);
+        }
+        st_shared_v4(O + sw128_off(c.lane, j), make_uint4(o[0], o[1], o[2], o[3]));
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (c.lane == 0) {
+        if (c.row0 < c.M) tma_store_2d(&ep.tmG, O, cc, c.row0);
+        bulk_commit();
+      }
+      ++st.cnt;
+    }
+    return true;
+  }
+
+  __device__ static void finish(const Params&, State&, uint64_t*, int lane, uint64_t) {
+    if (lane == 0) bulk_wait_all<0>();
+    __syncwarp();
+  }
 };
 
 }  // namespace coda

@@ -153,6 +153,82 @@ __global__ void __launch_bounds__(1024) mean_kernel(const float* __restrict__ lo
   if (threadIdx.x == 0) *mean = red[0] / static_cast<float>(M);
 }
 
+// Cross-entropy backward: exact label entries.  The chunked backward stores the
+// gradient G in bf16; at each row's label entry G = d (p - 1) dominates its dW
+// column, so the rounding dropped there (resid_i, recorded in fp32 by the
+// gradient epilogue) is added back:
+//   dH[i, :] += resid_i W[:, label_i]
+//   dW[:, v] += sum over rows i with label_i = v (in increasing i) of resid_i H[i, :]
+// Block i handles row i; the first row carrying a label owns that dW column,
+// so every column is updated by one block in a fixed order (no atomics).
+constexpr int kFixThreads = 256;
+constexpr int kFixCols = 8;  // columns of dW per thread per pass
+
+__global__ void __launch_bounds__(kFixThreads) ce_bwd_label_fix_kernel(
+    const int64_t* __restrict__ labels, const float* __restrict__ resid, const __nv_bfloat16* __restrict__ H,
+    const __nv_bfloat16* __restrict__ W, float* __restrict__ dH, float* __restrict__ dW, int M, int K,
+    long long V) {
+  __shared__ int rows[kFixThreads];
+  __shared__ int warp_count[kFixThreads / 32];
+  __shared__ int nrows;
+  const int i = blockIdx.x;
+  const long long lab = labels[i];
+  if (lab < 0 || lab >= V) return;  // such a row has no label entry (and no residual)
+  const float ri = resid[i];
+  for (int k = threadIdx.x; k < K; k += kFixThreads)
+    dH[static_cast<size_t>(i) * K + k] += ri * __bfloat162float(W[static_cast<size_t>(k) * V + lab]);
+  int earlier = 0;
+  for (int j = threadIdx.x; j < i; j += kFixThreads) earlier |= (labels[j] == lab);
+  if (__syncthreads_or(earlier)) return;  // an earlier row owns this column
+  // This block owns column `lab`.  Usually no later row repeats the label:
+  // then the column gets resid_i H[i, :] alone.
+  int later = 0;
+  for (int j = i + 1 + static_cast<int>(threadIdx.x); j < M; j += kFixThreads) later |= (labels[j] == lab);
+  if (!__syncthreads_or(later)) {
+    for (int k = threadIdx.x; k < K; k += kFixThreads)
+      dW[static_cast<size_t>(k) * V + lab] += ri * __bfloat162float(H[static_cast<size_t>(i) * K + k]);
+    return;
+  }
+  // Otherwise add the residuals of rows j >= i carrying the same label, in
+  // increasing j, kFixThreads * kFixCols columns per pass.
+  for (int kbase = 0; kbase < K; kbase += kFixThreads * kFixCols) {
+    float acc[kFixCols];
+#pragma unroll
+    for (int q = 0; q < kFixCols; ++q) acc[q] = 0.f;
+    for (int j0 = i; j0 < M; j0 += kFixThreads) {
+      const int j = j0 + threadIdx.x;
+      const bool match = j < M && labels[j] == lab;
+      const unsigned ballot = __ballot_sync(0xffffffffu, match);
+      if ((threadIdx.x & 31) == 0) warp_count[threadIdx.x >> 5] = __popc(ballot);
+      __syncthreads();
+      int base = 0;
+      for (int w = 0; w < (threadIdx.x >> 5); ++w) base += warp_count[w];
+      if (match) rows[base + __popc(ballot & ((1u << (threadIdx.x & 31)) - 1u))] = j;
+      if (threadIdx.x == 0) {
+        int t = 0;
+        for (int w = 0; w < kFixThreads / 32; ++w) t += warp_count[w];
+        nrows = t;
+      }
+      __syncthreads();
+      for (int q = 0; q < nrows; ++q) {
+        const int jr = rows[q];
+        const float rj = resid[jr];
+#pragma unroll
+        for (int s2 = 0; s2 < kFixCols; ++s2) {
+          const int k = kbase + s2 * kFixThreads + threadIdx.x;
+          if (k < K) acc[s2] += rj * __bfloat162float(H[static_cast<size_t>(jr) * K + k]);
+        }
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int s2 = 0; s2 < kFixCols; ++s2) {
+      const int k = kbase + s2 * kFixThreads + threadIdx.x;
+      if (k < K) dW[static_cast<size_t>(k) * V + lab] += acc[s2];
+    }
+  }
+}
+
 // ------------------------------------------------------ unfused comparison chain
 
 // out = a + b (bf16, 8 elements per thread).

@@ -166,6 +166,29 @@ coda_status_t coda_lmhead_ce(const uint16_t* H, const uint16_t* W, const int64_t
                              float* loss_out, float* lse_out, float* mean_out, void* ws, size_t ws_bytes,
                              int64_t M, int64_t V, int64_t K, void* stream);
 
+/* Bytes of workspace coda_lmhead_ce_bwd needs (one bf16 gradient chunk of
+ * M x min(V, 4096) and M fp32 residuals). */
+size_t coda_lmhead_ce_bwd_workspace_size(int64_t M, int64_t V);
+
+/* Backward of coda_lmhead_ce, block-local (section "CODA: the secret in the
+ * epilogue": the backward inherits the block-local structure).  For the loss
+ * L = sum_i d_i loss_i (d = d_loss, or 1/M for every token when d_loss is
+ * NULL: the mean), with the forward's saved lse:
+ *   G_ij = d_i (exp(z_ij - lse_i) - [j == label_i]),  z = r_i (H W)_ij
+ *   dH_out = G W^T  [M, K] fp32;   dW_out = H^T G  [K, V] fp32.
+ * The vocabulary is processed in chunks of 4096 columns: a GEMM recomputes the
+ * chunk's logits and its epilogue writes G_chunk (bf16, in the workspace;
+ * the logits are never stored), then dH += G_chunk W_chunk^T and
+ * dW_chunk = H^T G_chunk.  The label entry d_i (p - 1) dominates its dW
+ * column, so the part of it that bf16 drops is kept in fp32 and added back
+ * afterwards (deterministically, without atomics).  A label outside [0, V)
+ * contributes no onehot term.  H [M, K] bf16,
+ * W [K, V] bf16, labels [M] int64, lse [M] fp32, d_loss and r [M] fp32 or NULL,
+ * ws >= coda_lmhead_ce_bwd_workspace_size(M, V). */
+coda_status_t coda_lmhead_ce_bwd(const uint16_t* H, const uint16_t* W, const int64_t* labels, const float* lse,
+                                 const float* d_loss, const float* r, float* dH_out, float* dW_out, void* ws,
+                                 size_t ws_bytes, int64_t M, int64_t V, int64_t K, void* stream);
+
 /* ---------------------------------------------------------------- backward */
 
 /* Bytes of workspace coda_gemm_rowscale_bwd needs (holds y = r * hg, bf16 [M, N]). */
