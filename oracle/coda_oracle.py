@@ -139,6 +139,36 @@ def swiglu_mlp_backward_unfused(y, W_gu, W_down, res, d_h2) -> dict:
             "dW_gu": matmul(as_f64(y).T, d_gu), "d_y": matmul(d_gu, as_f64(W_gu).T), "d_res": dH2.copy(), **f}
 
 
+def rope_rotate(t, positions, head_dim: int, theta: float) -> np.ndarray:
+    """Rotary position encoding of the heads of t ([M, n_heads * head_dim]),
+    rotate-half form: for i < head_dim / 2 the columns i and i + head_dim / 2 of
+    every head form a pair rotated by the angle pos * theta^(-2 i / head_dim):
+    (a, b) -> (a cos - b sin, b cos + a sin)."""
+    t = as_f64(t)
+    M, W_ = t.shape
+    half = head_dim // 2
+    pos = np.asarray(positions, dtype=np.float64)
+    inv = theta ** (-2.0 * np.arange(half) / head_dim)
+    ang = pos[:, None] * inv[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    out = t.copy()
+    for h0 in range(0, W_, head_dim):
+        a = t[:, h0:h0 + half]
+        b = t[:, h0 + half:h0 + head_dim]
+        out[:, h0:h0 + half] = a * c - b * s
+        out[:, h0 + half:h0 + head_dim] = b * c + a * s
+    return out
+
+
+def qkv_rope_unfused(x, W_qkv, positions, head_dim: int, rope_cols: int, theta: float) -> np.ndarray:
+    """QKV projection followed by RoPE on its first rope_cols columns (the q and
+    k heads); the remaining (v) columns pass through."""
+    qkv = matmul(x, W_qkv)
+    out = qkv.copy()
+    out[:, :rope_cols] = rope_rotate(qkv[:, :rope_cols], positions, head_dim, theta)
+    return out
+
+
 def cross_entropy_unfused(H, W, labels) -> dict:
     """Softmax cross-entropy over the vocabulary with materialised logits:
     z = H W; lse_i = log sum_j exp(z_ij); loss_i = lse_i - z_i,label; mean over

@@ -1,0 +1,65 @@
+"""Pins of the oracle's RoPE in the QKV projection (CPU only).
+
+Source: KuCoin news flash "CODA: new research optimizes transformer training
+with GEMM epilogue programming", section "CODA: the secret in the epilogue"
+(RoPE, rotary position encoding, takes the same re-parameterisation) and
+section "Five kinds of building blocks" (RoPE as an elementwise transform).
+The rotate-half form with angle pos * theta^(-2i/d) is the plain reading.
+Pins: position 0 is the identity; every rotated pair keeps its norm; the
+q.k product of two rotated vectors depends only on the position difference;
+brute force with Python's math on a tiny case.
+"""
+import math
+
+import numpy as np
+
+from oracle import coda_oracle as O
+
+
+def test_position_zero_is_identity_and_pairs_keep_norm():
+    r = np.random.default_rng(31)
+    t = r.normal(size=(3, 16))
+    np.testing.assert_allclose(O.rope_rotate(t, [0, 0, 0], 8, 10000.0), t, rtol=0, atol=0)
+    pos = [5, 1000, 8191]
+    out = O.rope_rotate(t, pos, 8, 500000.0)
+    for h0 in (0, 8):
+        n_in = t[:, h0:h0 + 4] ** 2 + t[:, h0 + 4:h0 + 8] ** 2
+        n_out = out[:, h0:h0 + 4] ** 2 + out[:, h0 + 4:h0 + 8] ** 2
+        np.testing.assert_allclose(n_out, n_in, rtol=1e-12)
+
+
+def test_relative_position_property():
+    r = np.random.default_rng(32)
+    q, k = r.normal(size=(1, 8)), r.normal(size=(1, 8))
+    dots = []
+    for p in (3, 40, 1000):
+        qr = O.rope_rotate(q, [p + 7], 8, 10000.0)
+        kr = O.rope_rotate(k, [p], 8, 10000.0)
+        dots.append(float((qr * kr).sum()))
+    np.testing.assert_allclose(dots, dots[0], rtol=1e-10)
+
+
+def test_brute_force_tiny():
+    r = np.random.default_rng(33)
+    d, theta = 4, 100.0
+    t = r.normal(size=(2, 2 * d))
+    pos = [3, 11]
+    out = O.rope_rotate(t, pos, d, theta)
+    for m in range(2):
+        for h0 in (0, d):
+            for i in range(d // 2):
+                ang = pos[m] * theta ** (-2 * i / d)
+                a, b = t[m, h0 + i], t[m, h0 + i + d // 2]
+                assert math.isclose(out[m, h0 + i], a * math.cos(ang) - b * math.sin(ang), rel_tol=1e-12,
+                                    abs_tol=1e-14)
+                assert math.isclose(out[m, h0 + i + d // 2], b * math.cos(ang) + a * math.sin(ang),
+                                    rel_tol=1e-12, abs_tol=1e-14)
+
+
+def test_qkv_rope_leaves_v_columns():
+    r = np.random.default_rng(34)
+    x, W = r.normal(size=(4, 6)), r.normal(size=(6, 24))
+    out = O.qkv_rope_unfused(x, W, [0, 1, 2, 3], 8, 16, 10000.0)
+    qkv = x @ W
+    np.testing.assert_allclose(out[:, 16:], qkv[:, 16:], rtol=1e-14)
+    np.testing.assert_allclose(out[:, :16], O.rope_rotate(qkv[:, :16], [0, 1, 2, 3], 8, 10000.0), rtol=1e-14)
