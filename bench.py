@@ -493,6 +493,22 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
                               "gemm_swiglu_bwd_tflops": round(f_swb / k[0] / 1e9, 1)}
     del act, h2, p2, gu, d_h2, d_gu
 
+    # QKV projection with RoPE in its epilogue (1B attention input: 32 q + 8 k + 8 v heads of 64)
+    n_qkv, rope_cols = 48 * 64, 40 * 64
+    W_qkv = synth.normal_bf16(synth.make_gen(8 + 1000 * rank), (D, n_qkv), std=0.02).to(dev)
+    pos = (torch.arange(M_TOK, dtype=torch.int32, device=dev) % 2048)
+    qkv = torch.empty(M_TOK, n_qkv, dtype=torch.bfloat16, device=dev)
+
+    def qr():
+        C.gemm_qkv_rope(x, W_qkv, pos, 64, rope_cols, out=qkv)
+
+    for _ in range(3):
+        qr()
+    tot, _ = timed(qr, steps, 0)
+    ms = sum(tot) / len(tot)
+    res["qkv_rope"] = {"ms": round(ms, 4), "tflops": round(2.0 * M_TOK * D * n_qkv / ms / 1e9, 1)}
+    del W_qkv, pos, qkv
+
     # fused LM-head cross-entropy (8192 x 2048 x 128256)
     H, Wv, labels = synth.lmhead_ce_inputs(seed=3 + 1000 * rank)  # rank's own tokens
     H, Wv, labels = H.to(dev), Wv.to(dev), labels.to(dev)

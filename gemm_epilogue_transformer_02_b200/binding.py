@@ -50,6 +50,7 @@ _SIGS = {
     "coda_gemm_rowscale": (_ST, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "coda_gemm_rowscale_partial": (_ST, [_P, _P, _P, _I64, _I64, _F, _P, _P, _I64, _I64, _I64, _P]),
     "coda_gemm_swiglu": (_ST, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "coda_gemm_qkv_rope": (_ST, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _F, _P]),
     "coda_gemm_swiglu_bwd": (_ST, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "coda_lmhead_ce_workspace_size": (_SZ, [_I64, _I64]),
     "coda_lmhead_ce": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _P]),
@@ -241,6 +242,20 @@ def gemm_swiglu(A, W_gu, r=None, save=False, act_out=None, gateup_out=None):
         gu = _empty((M, 2 * F), BF16, A)
     _call("coda_gemm_swiglu", _ptr(A), _ptr(W_gu), _ptr(r), _ptr(act_out), _ptr(gu), M, F, K, _stream())
     return act_out, gu
+
+
+def gemm_qkv_rope(x, W_qkv, positions, head_dim: int, rope_cols: int, theta: float = 500000.0, out=None):
+    """qkv = x W_qkv with RoPE applied to the first rope_cols columns (q and k heads)."""
+    M, K = x.shape
+    N = W_qkv.shape[1]
+    _need(x, BF16, "x")
+    _need(W_qkv, BF16, "W_qkv", (K, N))
+    _need(positions, torch.int32, "positions", (M,))
+    if out is None:
+        out = _empty((M, N), BF16, x)
+    _call("coda_gemm_qkv_rope", _ptr(x), _ptr(W_qkv), _ptr(positions), _ptr(out), M, N, K, int(head_dim),
+          int(rope_cols), float(theta), _stream())
+    return out
 
 
 def gemm_swiglu_bwd(d_out, W_down, gateup, out=None):

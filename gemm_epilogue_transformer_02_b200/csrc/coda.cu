@@ -138,6 +138,7 @@ enum KernelKind : uint32_t {
   kKindSwiGLUBwd,
   kKindCEGrad,
   kKindF32KK,
+  kKindRope,
 };
 
 // Vocabulary columns per chunk of the cross-entropy backward: the chunk's
@@ -421,6 +422,36 @@ coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const fl
   const int n_nt = static_cast<int>((F + 127) / 128);
   return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(F), static_cast<int>(K), n_nt,
       raster_group(M, 2 * F, K), kKindSwiGLU, static_cast<cudaStream_t>(stream));
+}
+
+coda_status_t coda_gemm_qkv_rope(const uint16_t* x, const uint16_t* W_qkv, const int32_t* positions, uint16_t* out,
+                                 int64_t M, int64_t N, int64_t K, int64_t head_dim, int64_t rope_cols, float theta,
+                                 void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(N) && dim_ok(K) && (head_dim == 64 || head_dim == 128) &&
+                 N % head_dim == 0 && rope_cols >= 0 && rope_cols <= N && rope_cols % head_dim == 0 &&
+                 theta > 1.0f,
+             CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(x && W_qkv && positions && out, CODA_ERR_NULL);
+  CODA_CHECK(al16(x) && al16(W_qkv) && al16(positions) && al16(out), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  using Epi = EpiRope;
+  GemmParams<Epi> p{};
+  if (!(map_a(&p.tmA, x, false, M, K) && map_b(&p.tmB, W_qkv, true, N, K, N, 128) &&
+        map_out_bf16(&p.ep.tmOut, out, M, N, N)))
+    return CODA_ERR_INTERNAL;
+  p.ep.positions = positions;
+  p.ep.head_dim = static_cast<int>(head_dim);
+  p.ep.rope_cols = static_cast<int>(rope_cols);
+  p.ep.log2_theta = log2f(theta);
+  return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(
+      dev, info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>((N + 255) / 256),
+      raster_group(M, N, K), kKindRope, static_cast<cudaStream_t>(stream));
 }
 
 coda_status_t coda_gemm_swiglu_bwd(const uint16_t* d_out, const uint16_t* W_down, const uint16_t* gateup,

@@ -86,6 +86,7 @@ struct GemmSmem {
   static constexpr int kEpiBytes = kEpiWarps * Epi::kSmemPerWarp;
   static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1 + kEpiWarps * Epi::kBarsPerWarp;
   static constexpr int kBytes = 1024 /*align slack*/ + STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 16;
+  static_assert(Epi::kSmemPerWarp % 1024 == 0, "per-warp epilogue buffers keep the 128-byte swizzle alignment");
 };
 
 // Bounded wait that ignores the abort flag (used to drain copies in flight
@@ -985,6 +986,120 @@ struct EpiCE {
   }
 
   __device__ static void finish(const Params&, State&, uint64_t*, int, uint64_t) {}
+};
+
+// ---------------------------------------------------------------------------
+// RoPE in the QKV projection's epilogue (rotate-half form).  For every head of
+// head_dim columns that lies below rope_cols (the q and k heads), columns i and
+// i + head_dim/2 form a pair rotated by the angle pos * theta^(-2 i / head_dim):
+//   (a, b) -> (a cos - b sin, b cos + a sin);
+// heads at or beyond rope_cols (v) are stored unrotated.  One thread owns one
+// row, so both columns of every pair are in its registers, and the sines and
+// cosines of its row are computed once per 32 frequencies and reused for every
+// head of the tile.  The angle is taken in turns, pos * theta^(-2i/d) / (2 pi),
+// in fp64; only its fractional part goes to sincospif, so large positions
+// keep their accuracy without a range reduction.
+// ---------------------------------------------------------------------------
+struct EpiRope {
+  // one 256-column x 32-row bf16 staging tile (four 64-column boxes) + 1 KB of
+  // per-frequency turns; a multiple of 1024 keeps the 128-byte swizzle alignment
+  static constexpr int kSmemPerWarp = 16384 + 1024;
+  static constexpr int kBarsPerWarp = 0;
+  static constexpr bool kPairedB = false;
+
+  struct Params {
+    CUtensorMap tmOut;      // [M, N] bf16, box 64 x 32
+    const int* positions;   // [M]
+    int head_dim;           // 64 or 128
+    int rope_cols;          // columns [0, rope_cols) are rotated; a multiple of head_dim
+    float log2_theta;
+  };
+  struct State {
+    bool freq_ready;
+  };
+  __device__ static void init_state(State& s) { s.freq_ready = false; }
+
+  template <int BN>
+  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
+    constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+    const int col0 = c.nb * BN;
+    const int row = c.row0 + c.lane;
+    const int dh = ep.head_dim;
+    const int half = dh >> 1;
+    double* turn = reinterpret_cast<double*>(c.wsmem + 16384);
+    if (!st.freq_ready) {
+      for (int i = c.lane; i < half; i += 32)
+        turn[i] = exp2(-(2.0 * i / dh) * static_cast<double>(ep.log2_theta)) * kInvTwoPi;
+      __syncwarp();
+      st.freq_ready = true;
+    }
+    const double pos = (row < c.M) ? static_cast<double>(ep.positions[row]) : 0.0;
+    int ncols = c.N - col0;
+    if (ncols > BN) ncols = BN;
+    const int nheads = ncols / dh;
+    const bool any_rot = col0 < ep.rope_cols;
+    uint8_t* S = c.wsmem;
+    if (c.lane == 0) bulk_wait_read<0>();  // the previous tile's stores have read the staging
+    __syncwarp();
+    for (int s = 0; s < half / 32; ++s) {
+      float cs[32], sn[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        cs[e] = 1.f;
+        sn[e] = 0.f;
+        if (any_rot) {
+          const double t = pos * turn[s * 32 + e];
+          sincospif(static_cast<float>(2.0 * (t - rint(t))), &sn[e], &cs[e]);
+        }
+      }
+      for (int hd = 0; hd < nheads; ++hd) {
+        const int hc0 = hd * dh;  // head's first column within the tile
+        const bool rot = col0 + hc0 < ep.rope_cols;
+        uint32_t va[32], vb[32];
+        tmem_ld32(c.taddr + hc0 + s * 32, va);
+        tmem_ld32(c.taddr + hc0 + half + s * 32, vb);
+        tmem_ld_wait(va);
+        reg_pin(vb);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t pa[4], pb[4];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            float oa[2], ob[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int e = q * 8 + 2 * e2 + h;
+              const float a = __uint_as_float(va[e]);
+              const float bb = __uint_as_float(vb[e]);
+              oa[h] = rot ? a * cs[e] - bb * sn[e] : a;
+              ob[h] = rot ? bb * cs[e] + a * sn[e] : bb;
+            }
+            pa[e2] = pack_bf16x2(oa[0], oa[1]);
+            pb[e2] = pack_bf16x2(ob[0], ob[1]);
+          }
+          const int ca = hc0 + s * 32 + q * 8;
+          const int cb = hc0 + half + s * 32 + q * 8;
+          st_shared_v4(S + (ca >> 6) * 4096 + sw128_off(c.lane, (ca & 63) >> 3),
+                       make_uint4(pa[0], pa[1], pa[2], pa[3]));
+          st_shared_v4(S + (cb >> 6) * 4096 + sw128_off(c.lane, (cb & 63) >> 3),
+                       make_uint4(pb[0], pb[1], pb[2], pb[3]));
+        }
+      }
+    }
+    fence_async_smem();
+    __syncwarp();
+    if (c.lane == 0) {
+      if (c.row0 < c.M)
+        for (int bx = 0; bx < (ncols + 63) / 64; ++bx) tma_store_2d(&ep.tmOut, S + bx * 4096, col0 + bx * 64, c.row0);
+      bulk_commit();
+    }
+    return true;
+  }
+
+  __device__ static void finish(const Params&, State&, uint64_t*, int lane, uint64_t) {
+    if (lane == 0) bulk_wait_all<0>();
+    __syncwarp();
+  }
 };
 
 // ---------------------------------------------------------------------------

@@ -136,6 +136,21 @@ coda_status_t coda_gemm_rowscale_partial(const uint16_t* A, const uint16_t* W, c
 coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const float* r, uint16_t* act_out,
                                uint16_t* gateup_save, int64_t M, int64_t F, int64_t K, void* stream);
 
+/* QKV projection with RoPE in its epilogue (section "CODA: the secret in the
+ * epilogue" lists RoPE, rotary position encoding, among the re-parameterised
+ * operations; section "Five kinds of building blocks": an elementwise
+ * transform).  acc = x W_qkv (fp32); for every head of head_dim columns below
+ * rope_cols (the q and k heads), columns i and i + head_dim/2 of the head are
+ * rotated by the angle positions[m] * theta^(-2 i / head_dim):
+ *   (a, b) -> (a cos - b sin, b cos + a sin);
+ * columns from rope_cols on (v) are stored unrotated; out = bf16.
+ * x [M, K] bf16, W_qkv [K, N] bf16 (q heads, then k heads, then v heads),
+ * positions [M] int32, out [M, N] bf16; head_dim 64 or 128, N and rope_cols
+ * multiples of head_dim, theta > 1 (LLaMA-3: 500000). */
+coda_status_t coda_gemm_qkv_rope(const uint16_t* x, const uint16_t* W_qkv, const int32_t* positions, uint16_t* out,
+                                 int64_t M, int64_t N, int64_t K, int64_t head_dim, int64_t rope_cols, float theta,
+                                 void* stream);
+
 /* SwiGLU backward, block-local in the down projection's dA GEMM (section "CODA:
  * the secret in the epilogue": the backward of a block-local epilogue is
  * block-local too).  The GEMM forms d_act = d_out W_down^T tile by tile; its
