@@ -282,6 +282,14 @@ def run_ours(args):
             evs[0].record(stream)
         C.gemm_rowscale_partial(hg, W2, part, D, EPS, out=out, r_out=r)
 
+    ws_block = torch.empty(max(int(C.load_library().coda_rmsnorm_block_workspace_size(M_TOK)), 16),
+                           dtype=torch.uint8, device=dev)
+
+    def block1():
+        # the same block as one persistent launch (both GEMMs on the same CTA pairs)
+        C.rmsnorm_block(x, res, W1, W2, gamma, EPS, out=out,
+                        bufs={"h": h, "hg": hg, "partial": part, "r": r, "ws": ws_block})
+
     def block3():
         # the same block with the light reduction as its own kernel
         C.gemm_res_partialrms(x, W1, res, gamma, h_out=h, hg_out=hg, partial_out=part)
@@ -337,17 +345,18 @@ def run_ours(args):
     # ---- unfused chain, same protocol
     # ---- fused vs unfused chain (and the three-launch block), interleaved
     # step by step so that all three see the same clocks and power state
-    ms_unfused = ms_fused_il = ms_block3 = None
+    ms_unfused = ms_fused_il = ms_block3 = ms_block1 = None
     if not args.no_unfused:
         u_steps = max(20, min(args.steps, 200))
         for _ in range(5):
             unfused()
             block3()
+            block1()
         torch.cuda.synchronize()
         rec = []
         for _ in range(u_steps):
             evs = []
-            for fn in (block, unfused, block3):
+            for fn in (block, unfused, block3, block1):
                 flush.zero_()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
@@ -356,8 +365,8 @@ def run_ours(args):
                 evs.append((e0, e1))
             rec.append(evs)
         torch.cuda.synchronize()
-        avg = [sum(r_[i][0].elapsed_time(r_[i][1]) for r_ in rec) / len(rec) for i in range(3)]
-        ms_fused_il, ms_unfused, ms_block3 = avg
+        avg = [sum(r_[i][0].elapsed_time(r_[i][1]) for r_ in rec) / len(rec) for i in range(4)]
+        ms_fused_il, ms_unfused, ms_block3, ms_block1 = avg
 
     # ---- end-to-end through the public API with host buffers (pinned)
     x_h = inp.x.pin_memory()
@@ -424,7 +433,7 @@ def run_ours(args):
                 "gemm_res_partialrms_gbs": round(BYTES_G1 / (k_ms[0] / 1e3) / 1e9, 1),
                 "interleaved": None if ms_unfused is None else {
                     "steps": u_steps, "fused_ms": round(ms_fused_il, 4), "unfused_chain_ms": round(ms_unfused, 4),
-                    "three_launch_block_ms": round(ms_block3, 4)},
+                    "three_launch_block_ms": round(ms_block3, 4), "one_launch_block_ms": round(ms_block1, 4)},
                 "unfused_chain_ms": None if ms_unfused is None else round(ms_unfused, 4),
                 "speedup_vs_unfused": None if ms_unfused is None else round(ms_unfused / ms_fused_il, 4),
                 "hbm_bytes_fused_alg": BYTES_FUSED, "hbm_bytes_unfused_alg": BYTES_UNFUSED,

@@ -49,6 +49,8 @@ _SIGS = {
     "coda_rms_reduce": (_ST, [_P, _I64, _I64, _I64, _F, _P, _P]),
     "coda_gemm_rowscale": (_ST, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "coda_gemm_rowscale_partial": (_ST, [_P, _P, _P, _I64, _I64, _F, _P, _P, _I64, _I64, _I64, _P]),
+    "coda_rmsnorm_block_workspace_size": (_SZ, [_I64]),
+    "coda_rmsnorm_block": (_ST, [_P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _I64, _P]),
     "coda_gemm_swiglu": (_ST, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "coda_gemm_qkv_rope": (_ST, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _F, _P]),
     "coda_gemm_swiglu_bwd": (_ST, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
@@ -415,11 +417,44 @@ def selftest_bounded_wait(limit_ns: int) -> int:
 # -------------------------------------------------- call sequences of the path
 
 
-def gemm_rmsnorm_gemm(x, res, W1, W2, gamma, eps: float, out=None, bufs=None, fold_reduce=True):
+def rmsnorm_block(x, res, W1, W2, gamma, eps: float, out=None, bufs=None):
+    """The whole block in one persistent launch (coda_rmsnorm_block).
+    Returns dict(out, h, hg, partial, r)."""
+    M, K = x.shape
+    N = W1.shape[1]
+    N2 = W2.shape[1]
+    _need(x, BF16, "x")
+    if res is not None:
+        _need(res, BF16, "res", (M, N))
+    _need(W1, BF16, "W1", (K, N))
+    _need(W2, BF16, "W2", (N, N2))
+    _need(gamma, BF16, "gamma", (N,))
+    b = bufs or {}
+    h = b.get("h") if b.get("h") is not None else _empty((M, N), BF16, x)
+    hg = b.get("hg") if b.get("hg") is not None else _empty((M, N), BF16, x)
+    partial = b.get("partial") if b.get("partial") is not None else _empty((partial_cols(N), M), F32, x)
+    r = b.get("r") if b.get("r") is not None else _empty((M,), F32, x)
+    if out is None:
+        out = _empty((M, N2), BF16, x)
+    ws = b.get("ws")
+    if ws is None:
+        ws = _empty((max(int(load_library().coda_rmsnorm_block_workspace_size(M)), 16),), torch.uint8, x)
+    _call("coda_rmsnorm_block", _ptr(x), _ptr(res), _ptr(W1), _ptr(W2), _ptr(gamma), float(eps), _ptr(h), _ptr(hg),
+          _ptr(partial), _ptr(r), _ptr(out), _ptr(ws), ws.numel(), M, K, N, N2, _stream())
+    return {"out": out, "h": h, "hg": hg, "partial": partial, "r": r}
+
+
+def gemm_rmsnorm_gemm(x, res, W1, W2, gamma, eps: float, out=None, bufs=None, fold_reduce=True, launches=None):
     """The fused block: first GEMM + residual + partial RMS, the light
-    reduction, and the row-scaled second GEMM.  With fold_reduce (default) the
-    reduction runs inside the second GEMM's epilogue (two launches); without
-    it, as its own kernel (three launches).  Returns dict(out, h, hg, partial, r)."""
+    reduction, and the row-scaled second GEMM.  launches=1: one persistent
+    launch (coda_rmsnorm_block); 2 (the default, or fold_reduce): the reduction
+    inside the second GEMM's epilogue; 3 (fold_reduce=False): the reduction as
+    its own kernel.  Returns dict(out, h, hg, partial, r)."""
+    if launches is None:
+        launches = 2 if fold_reduce else 3
+    if launches == 1:
+        return rmsnorm_block(x, res, W1, W2, gamma, eps, out=out, bufs=bufs)
+    fold_reduce = launches == 2
     N = W1.shape[1]
     b = bufs or {}
     h, hg, partial = gemm_res_partialrms(x, W1, res, gamma, h_out=b.get("h"), hg_out=b.get("hg"),

@@ -6,6 +6,7 @@
 
 #include "coda.h"
 #include "coda_device.cuh"
+#include "coda_block.cuh"
 #include "coda_gemm.cuh"
 #include "coda_rowops.cuh"
 
@@ -139,6 +140,7 @@ enum KernelKind : uint32_t {
   kKindCEGrad,
   kKindF32KK,
   kKindRope,
+  kKindBlock,
 };
 
 // Vocabulary columns per chunk of the cross-entropy backward: the chunk's
@@ -364,6 +366,108 @@ coda_status_t coda_gemm_rowscale(const uint16_t* A, const uint16_t* W, const flo
   const int n_nt = static_cast<int>((N + 255) / 256);
   return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), n_nt,
       raster_group(M, N, K), kKindRowScale, static_cast<cudaStream_t>(stream));
+}
+
+size_t coda_rmsnorm_block_workspace_size(int64_t M) {
+  if (M < 0) return 0;
+  return align256(static_cast<size_t>((M + 255) / 256) * 4);
+}
+
+coda_status_t coda_rmsnorm_block(const uint16_t* x, const uint16_t* res, const uint16_t* W1, const uint16_t* W2,
+                                 const uint16_t* gamma, float eps, uint16_t* h_out, uint16_t* hg_out,
+                                 float* partial_out, float* r_out, uint16_t* out, void* ws, size_t ws_bytes,
+                                 int64_t M, int64_t K, int64_t N, int64_t N2, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(K) && dim_ok(N) && dim_ok(N2) && eps >= 0.f,
+             CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(x && W1 && W2 && gamma && h_out && hg_out && partial_out && out, CODA_ERR_NULL);
+  CODA_CHECK(al16(x) && al16(res) && al16(W1) && al16(W2) && al16(gamma) && al16(h_out) && al16(hg_out) &&
+                 al16(partial_out) && al16(r_out) && al16(out) && al16(ws),
+             CODA_ERR_ALIGN);
+  CODA_CHECK(ws != nullptr && ws_bytes >= coda_rmsnorm_block_workspace_size(M), CODA_ERR_WORKSPACE);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  constexpr int kStages = 5;
+  auto kern = coda_block_kernel<kStages>;
+  constexpr int smem = BlockSmem<kStages>::kBytes;
+  KernelCache& kc = g_kcache[dev][kKindBlock];
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!kc.attr) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return CODA_ERR_LAUNCH;
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * (info->sms / 2), 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = info->sms / 2;
+      }
+      kc.max_clusters = n;
+      kc.attr = true;
+    }
+  }
+  BlockParams p{};
+  bool ok = map_a(&p.tmA1, x, false, M, K) && map_b(&p.tmB1, W1, true, N, K, N, 128) &&
+            map_a(&p.tmA2, hg_out, false, M, N) && map_b(&p.tmB2, W2, true, N2, N, N2, 128) &&
+            map_out_bf16(&p.ep1.tmOut1, h_out, M, N, N) && map_out_bf16(&p.ep1.tmOut2, hg_out, M, N, N) &&
+            map_out_bf16(&p.ep2.tmOut, out, M, N2, N2);
+  if (!ok) return CODA_ERR_INTERNAL;
+  p.ep1.in = reinterpret_cast<const __nv_bfloat16*>(res);
+  p.ep1.gamma = reinterpret_cast<const __nv_bfloat16*>(gamma);
+  p.ep1.r = nullptr;
+  p.ep1.partial = partial_out;
+  p.ep1.has_out1 = 1;
+  p.ep1.has_out2 = 1;
+  p.ep2.r = nullptr;
+  p.ep2.partial = partial_out;
+  p.ep2.T = static_cast<int>((N + 255) / 256);
+  p.ep2.inv_n = 1.0f / static_cast<float>(N);
+  p.ep2.eps = eps;
+  p.ep2.r_out = r_out;
+  p.ready = static_cast<int*>(ws);
+  p.M = static_cast<int>(M);
+  p.K1 = static_cast<int>(K);
+  p.N1 = static_cast<int>(N);
+  p.N2 = static_cast<int>(N2);
+  p.n_mt = static_cast<int>((M + 255) / 256);
+  p.n_nt1 = static_cast<int>((N + 255) / 256);
+  p.n_nt2 = static_cast<int>((N2 + 255) / 256);
+  p.n1 = p.n_mt * p.n_nt1;
+  p.n2 = p.n_mt * p.n_nt2;
+  p.ready_target = p.n_nt1 * 2 * kEpiWarps;
+  p.wait_ns = static_cast<uint64_t>(g_wait_ns);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, static_cast<size_t>(p.n_mt) * 4, s) != cudaSuccess) return CODA_ERR_LAUNCH;
+  const int total = p.n1 + p.n2;
+  const int clusters = total < kc.max_clusters ? total : kc.max_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return CODA_ERR_LAUNCH;
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
 }
 
 coda_status_t coda_gemm_rowscale_partial(const uint16_t* A, const uint16_t* W, const float* partial, int64_t T,

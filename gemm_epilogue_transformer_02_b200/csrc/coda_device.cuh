@@ -329,6 +329,43 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
                : "memory");
 }
 
+// ------------------------------------------- cross-CTA completion counters
+
+// Order this thread's completed async-proxy (TMA) global writes before its
+// later generic-proxy operations, and the reverse for later TMA reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ void red_release_add(int* addr, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire(const int* addr) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+  return v;
+}
+
+// Wait (bounded) until *addr >= target.  Returns false after recording a
+// timeout, or when another role of the CTA aborted.
+__device__ __noinline__ bool counter_wait(const int* addr, int target, const WaitCtx& w) {
+  if (ld_acquire(addr) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(64);
+    if (ld_acquire(addr) >= target) return true;
+    if ((i & 15u) == 0) {
+      if (*w.abort_flag) return false;
+      if (globaltimer_ns() - t0 > w.limit_ns) {
+        *w.abort_flag = 1;
+        atomicCAS(&g_coda_status, 0, kDevTimeout);
+        return false;
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------- small helpers
 
 __device__ __forceinline__ uint4 ld_shared_v4(const void* p) {

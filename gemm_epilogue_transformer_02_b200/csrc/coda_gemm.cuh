@@ -595,7 +595,9 @@ struct EpiRowScale {
       rs = 0.f;
       if (row < c.M) {
         float sum = 0.f;
-        for (int t = 0; t < ep.T; ++t) sum += __ldg(ep.partial + static_cast<size_t>(t) * c.M + row);
+        // coherent (L2) loads: in the one-launch block the partials are written
+        // by other CTAs of the same kernel
+        for (int t = 0; t < ep.T; ++t) sum += __ldcg(ep.partial + static_cast<size_t>(t) * c.M + row);
         rs = rsqrtf(sum * ep.inv_n + ep.eps);
         if (ep.r_out != nullptr && c.nb == 0) ep.r_out[row] = rs;
       }

@@ -126,6 +126,29 @@ coda_status_t coda_gemm_rowscale_partial(const uint16_t* A, const uint16_t* W, c
                                          int64_t N_norm, float eps, float* r_out, uint16_t* out, int64_t M,
                                          int64_t N, int64_t K, void* stream);
 
+/* Bytes of workspace coda_rmsnorm_block needs (one int per 256-row block). */
+size_t coda_rmsnorm_block_workspace_size(int64_t M);
+
+/* The whole GEMM-RMSNorm-GEMM block in one persistent launch: the work of
+ * coda_gemm_res_partialrms (h, hg, partial) followed by that of
+ * coda_gemm_rowscale_partial (out, r), with the same results.  Both GEMMs run
+ * on the same CTA pairs: every pair first computes its share of first-GEMM
+ * tiles, then second-GEMM tiles, each of which starts once all first-GEMM
+ * tiles of its 256-row block have published their outputs (a counter per row
+ * block in the workspace, zeroed by this call with a memset on `stream`).  The
+ * second GEMM's tiles thereby fill the SMs the first GEMM's last wave leaves
+ * idle.  The kernel needs all of its clusters resident at once (its grid is
+ * the occupancy limit); kernels running concurrently on other streams that
+ * keep part of it from becoming resident make its bounded waits expire
+ * (CODA_ERR_DEVICE_TIMEOUT from coda_poll_status), so run it alone.
+ * x [M, K], res [M, N] (or NULL), W1 [K, N], W2 [N, N2], gamma [N] bf16;
+ * h_out, hg_out [M, N] bf16; partial_out [T, M] fp32 (T = coda_partial_cols(N));
+ * r_out [M] fp32 (or NULL); out [M, N2] bf16. */
+coda_status_t coda_rmsnorm_block(const uint16_t* x, const uint16_t* res, const uint16_t* W1, const uint16_t* W2,
+                                 const uint16_t* gamma, float eps, uint16_t* h_out, uint16_t* hg_out,
+                                 float* partial_out, float* r_out, uint16_t* out, void* ws, size_t ws_bytes,
+                                 int64_t M, int64_t K, int64_t N, int64_t N2, void* stream);
+
 /* Gate/up GEMM with SwiGLU in its epilogue (section "CODA: the secret in the
  * epilogue" lists SwiGLU among the re-parameterised operations):
  *   g = r_i (A W_gu[:, :F])_ij,  u = r_i (A W_gu[:, F:])_ij,  act = bf16(silu(g) * u)
