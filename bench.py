@@ -70,6 +70,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-unfused", action="store_true", help="skip timing the unfused comparison chain")
+    ap.add_argument("--sweep", action="store_true",
+                    help="also time the block at hidden 4096 (gate/up 28672) and 8192 (gate/up 57344)")
     return ap.parse_args()
 
 
@@ -398,6 +400,8 @@ def run_ours(args):
     if not args.no_path:
         path = time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma, h, hg, r, rank,
                          args.path_steps, timed)
+    if args.sweep:
+        path["hidden_sweep"] = time_sweep(C, synth, torch, dev, stream, flush, rank, args.path_steps)
 
     DD.barrier()
     C.poll_status()
@@ -452,6 +456,48 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     DD.shutdown()
     return 0
+
+
+def time_sweep(C, synth, torch, dev, stream, flush, rank, steps):
+    """The fused block and the unfused chain at larger widths, timed interleaved."""
+    out = {}
+    for d, n2 in ((4096, 28672), (8192, 57344)):
+        inp = synth.block_inputs(M_TOK, d, d, n2, seed=50 + d // 1024 + 1000 * rank, w_std=0.02)
+        t = [v.to(dev) for v in (inp.x, inp.res, inp.W1, inp.W2, inp.gamma)]
+        o = torch.empty(M_TOK, n2, dtype=torch.bfloat16, device=dev)
+        bf = {"h": torch.empty(M_TOK, d, dtype=torch.bfloat16, device=dev),
+              "hg": torch.empty(M_TOK, d, dtype=torch.bfloat16, device=dev),
+              "partial": torch.empty(C.partial_cols(d), M_TOK, dtype=torch.float32, device=dev),
+              "r": torch.empty(M_TOK, dtype=torch.float32, device=dev)}
+        bu = {"t": torch.empty(M_TOK, d, dtype=torch.bfloat16, device=dev),
+              "h": torch.empty(M_TOK, d, dtype=torch.bfloat16, device=dev),
+              "y": torch.empty(M_TOK, d, dtype=torch.bfloat16, device=dev)}
+        fns = (lambda: C.gemm_rmsnorm_gemm(*t, EPS, out=o, bufs=bf),
+               lambda: C.unfused_block(*t, EPS, out=o, bufs=bu))
+        for _ in range(3):
+            for fn in fns:
+                fn()
+        torch.cuda.synchronize()
+        rec = []
+        for _ in range(max(3, steps)):
+            row = []
+            for fn in fns:
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                row.append((e0, e1))
+            rec.append(row)
+        torch.cuda.synchronize()
+        fused, unf = [sum(r_[i][0].elapsed_time(r_[i][1]) for r_ in rec) / len(rec) for i in range(2)]
+        flops = 2.0 * M_TOK * d * (d + n2)
+        out[f"hidden{d}"] = {"n2": n2, "fused_ms": round(fused, 4), "unfused_ms": round(unf, 4),
+                             "tflops": round(flops / fused / 1e9, 1), "frac_of_nominal_2250": round(
+                                 flops / (fused / 1e3) / 2.25e15, 4), "speedup_vs_unfused": round(unf / fused, 4)}
+        del t, o, bf, bu
+        torch.cuda.empty_cache()
+    return out
 
 
 def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma, h, hg, r, rank, steps, timed):
