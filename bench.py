@@ -479,15 +479,15 @@ def time_sweep(C, synth, torch, dev, stream, flush, rank, steps):
                 fn()
         torch.cuda.synchronize()
         rec = []
-        for _ in range(max(3, steps)):
-            row = []
-            for fn in fns:
+        for it in range(max(3, 5 * steps)):
+            row = [None, None]
+            for i in ((0, 1) if it % 2 == 0 else (1, 0)):  # alternate the order: no position bias
                 flush.zero_()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-                fn()
+                fns[i]()
                 e1.record(stream)
-                row.append((e0, e1))
+                row[i] = (e0, e1)
             rec.append(row)
         torch.cuda.synchronize()
         fused, unf = [sum(r_[i][0].elapsed_time(r_[i][1]) for r_ in rec) / len(rec) for i in range(2)]
