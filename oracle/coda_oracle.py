@@ -189,7 +189,8 @@ def cross_entropy_unfused(H, W, labels) -> dict:
 def cross_entropy_backward_unfused(H, W, labels, d_loss=None) -> dict:
     """Backward of the per-token losses loss_i = lse_i - z_i,label with z = H W,
     for L = sum_i d_loss_i loss_i (d_loss defaults to 1/M: the mean):
-    G = d_loss_i (softmax(z)_i - onehot(label_i));  dH = G W^T;  dW = H^T G."""
+    G = d_loss_i (softmax(z)_i - onehot(label_i));  dH = G W^T;  dW = H^T G.
+    A label outside [0, V) has no onehot term (its row of G is d_i softmax)."""
     z = matmul(H, W)
     M, V = z.shape
     m = z.max(axis=1)
@@ -197,7 +198,8 @@ def cross_entropy_backward_unfused(H, W, labels, d_loss=None) -> dict:
     p /= p.sum(axis=1)[:, None]
     lab = np.asarray(labels, dtype=np.int64)
     G = p.copy()
-    G[np.arange(M), lab] -= 1.0
+    idx = np.nonzero((lab >= 0) & (lab < V))[0]  # a label outside [0, V) has no onehot term
+    G[idx, lab[idx]] -= 1.0
     dl = np.full(M, 1.0 / M) if d_loss is None else np.asarray(d_loss, dtype=np.float64)
     G *= dl[:, None]
     return {"G": G, "dH": matmul(G, as_f64(W).T), "dW": matmul(as_f64(H).T, G)}

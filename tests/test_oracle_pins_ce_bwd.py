@@ -62,3 +62,24 @@ def test_chunked_block_local_backward_equals_definition():
         got = O.lmhead_ce_bwd(H, W, labels, lse, d, chunk_cols=chunk)
         np.testing.assert_allclose(got["dH"], ref["dH"], rtol=0, atol=1e-13 * np.abs(ref["dH"]).max())
         np.testing.assert_allclose(got["dW"], ref["dW"], rtol=0, atol=1e-13 * np.abs(ref["dW"]).max())
+
+
+def test_out_of_range_label_has_no_onehot_term():
+    """A token whose label lies outside [0, V) keeps only the softmax part of
+    its gradient: its row of G sums to d_i (a valid row sums to 0), equals
+    d_i softmax(z_i) computed directly, and the chunked backward agrees."""
+    r = np.random.default_rng(24)
+    M, K, V = 4, 5, 9
+    H, W = r.normal(size=(M, K)), r.normal(size=(K, V))
+    labels = np.array([3, -1, V, 0])
+    d = np.array([0.25, 0.5, 0.75, 1.0])
+    b = O.cross_entropy_backward_unfused(H, W, labels, d)
+    np.testing.assert_allclose(b["G"].sum(axis=1), [0.0, 0.5, 0.75, 0.0], atol=1e-15)
+    z = H @ W
+    for i in (1, 2):
+        e = np.exp(z[i] - z[i].max())
+        np.testing.assert_allclose(b["G"][i], d[i] * e / e.sum(), rtol=1e-13)
+    lse = np.log(np.exp(z).sum(axis=1))
+    got = O.lmhead_ce_bwd(H, W, labels, lse, d, chunk_cols=4)
+    np.testing.assert_allclose(got["dW"], b["dW"], rtol=0, atol=1e-13 * np.abs(b["dW"]).max())
+    np.testing.assert_allclose(got["dH"], b["dH"], rtol=0, atol=1e-13 * np.abs(b["dH"]).max())
