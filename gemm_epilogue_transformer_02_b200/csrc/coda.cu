@@ -391,9 +391,10 @@ coda_status_t coda_rmsnorm_block(const uint16_t* x, const uint16_t* res, const u
     const coda_status_t ds = current_device(&dev, &info);
     if (ds != CODA_OK) return ds;
   }
-  constexpr int kStages = 5;
+  constexpr int kStages = 6;
   auto kern = coda_block_kernel<kStages>;
   constexpr int smem = BlockSmem<kStages>::kBytes;
+  static_assert(smem <= 232448, "the block kernel's shared memory exceeds one SM's opt-in limit");
   KernelCache& kc = g_kcache[dev][kKindBlock];
   {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -633,7 +634,11 @@ coda_status_t coda_lmhead_ce(const uint16_t* H, const uint16_t* W, const int64_t
 size_t coda_lmhead_ce_bwd_workspace_size(int64_t M, int64_t V) {
   if (M < 0 || V <= 0) return 0;
   const int64_t vc = V < kCEBwdChunk ? V : kCEBwdChunk;
-  return align256(static_cast<size_t>(M) * static_cast<size_t>(vc) * 2) + align256(static_cast<size_t>(M) * 4);
+  const size_t nb = static_cast<size_t>((V + kLabelTile - 1) / kLabelTile);
+  return align256(static_cast<size_t>(M) * static_cast<size_t>(vc) * 2)  // G chunk (bf16)
+         + align256(static_cast<size_t>(M) * 4)                           // label residuals
+         + 2 * align256(nb * 4) + align256((nb + 1) * 4)                  // bucket counts, cursors, offsets
+         + 2 * align256(static_cast<size_t>(M) * 8);                      // (label, row) entries, two copies
 }
 
 coda_status_t coda_lmhead_ce_bwd(const uint16_t* H, const uint16_t* W, const int64_t* labels, const float* lse,
@@ -653,9 +658,33 @@ coda_status_t coda_lmhead_ce_bwd(const uint16_t* H, const uint16_t* W, const int
     if (ds != CODA_OK) return ds;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint16_t* G = static_cast<uint16_t*>(ws);
   const int64_t vmax = V < kCEBwdChunk ? V : kCEBwdChunk;
-  float* resid = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(static_cast<size_t>(M) * vmax * 2));
+  const int nbk = static_cast<int>((V + kLabelTile - 1) / kLabelTile);
+  uint8_t* wp = static_cast<uint8_t*>(ws);
+  uint16_t* G = reinterpret_cast<uint16_t*>(wp);
+  wp += align256(static_cast<size_t>(M) * vmax * 2);
+  float* resid = reinterpret_cast<float*>(wp);
+  wp += align256(static_cast<size_t>(M) * 4);
+  int* counts = reinterpret_cast<int*>(wp);
+  wp += align256(static_cast<size_t>(nbk) * 4);
+  int* cursor = reinterpret_cast<int*>(wp);
+  wp += align256(static_cast<size_t>(nbk) * 4);
+  int* start = reinterpret_cast<int*>(wp);
+  wp += align256(static_cast<size_t>(nbk + 1) * 4);
+  int2* unsorted = reinterpret_cast<int2*>(wp);
+  wp += align256(static_cast<size_t>(M) * 8);
+  int2* entries = reinterpret_cast<int2*>(wp);
+  {
+    // rows bucketed by the 256-column vocabulary tile of their label, sorted by (label, row)
+    const int mi = static_cast<int>(M);
+    const int g = (mi + 255) / 256;
+    if (cudaMemsetAsync(counts, 0, static_cast<size_t>(nbk) * 4, s) != cudaSuccess) return CODA_ERR_LAUNCH;
+    ce_label_count_kernel<<<g, 256, 0, s>>>(labels, mi, V, counts);
+    ce_label_scan_kernel<<<1, 1024, 0, s>>>(counts, nbk, start, cursor);
+    ce_label_fill_kernel<<<g, 256, 0, s>>>(labels, mi, V, cursor, unsorted);
+    ce_label_sort_kernel<<<g, 256, 0, s>>>(unsorted, start, nbk, entries);
+    if (cudaGetLastError() != cudaSuccess) return CODA_ERR_LAUNCH;
+  }
   for (int64_t c0 = 0; c0 < V; c0 += kCEBwdChunk) {
     const int64_t vc = (V - c0) < kCEBwdChunk ? (V - c0) : kCEBwdChunk;
     {
@@ -700,17 +729,24 @@ coda_status_t coda_lmhead_ce_bwd(const uint16_t* H, const uint16_t* W, const int
         return CODA_ERR_INTERNAL;
       p.ep.accum = nullptr;
       p.ep.ld = V;
+      p.ep.fix_resid = resid;
+      p.ep.fix_col0 = c0;
+      p.ep.fix_start = start;
+      p.ep.fix_entries = entries;
+      p.ep.fix_H = reinterpret_cast<const __nv_bfloat16*>(H);
+      p.ep.fix_tile0 = static_cast<int>(c0 / kLabelTile);
       const coda_status_t st = run_gemm<256, pair_stages<Epi>(), true, true, true, Epi>(
           dev, info, p, static_cast<int>(K), static_cast<int>(vc), static_cast<int>(M),
           static_cast<int>((vc + 255) / 256), raster_group(K, vc, M), kKindF32MN, s);
       if (st != CODA_OK) return st;
     }
+    // dH's label entries of this chunk, while the chunk of W is still in L2
+    ce_label_dh_fix_kernel<<<info->sms * 4, 256, 0, s>>>(
+        entries, start, static_cast<int>(c0 / kLabelTile), static_cast<int>((c0 + vc + kLabelTile - 1) / kLabelTile),
+        resid, reinterpret_cast<const __nv_bfloat16*>(W), V, static_cast<int>(K), dH_out);
+    if (cudaGetLastError() != cudaSuccess) return CODA_ERR_LAUNCH;
   }
-  // the label entries, exact: add back what the bf16 gradient dropped there
-  ce_bwd_label_fix_kernel<<<static_cast<int>(M), kFixThreads, 0, s>>>(
-      labels, resid, reinterpret_cast<const __nv_bfloat16*>(H), reinterpret_cast<const __nv_bfloat16*>(W), dH_out,
-      dW_out, static_cast<int>(M), static_cast<int>(K), V);
-  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+  return CODA_OK;
 }
 
 size_t coda_gemm_rowscale_bwd_workspace_size(int64_t M, int64_t N) {

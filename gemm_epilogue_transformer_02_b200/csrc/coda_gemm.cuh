@@ -403,13 +403,14 @@ __device__ __forceinline__ float acc_at(const uint32_t (&v0)[32], const uint32_t
 // 128 bytes per 64-column chunk) one chunk ahead, and the first chunk of the
 // next tile is requested before this tile's last chunk is processed, so its
 // latency hides behind the epilogue math.  Outputs are staged in shared
-// memory (128-byte swizzle) and written by TMA stores; MODE 0 double-buffers
-// the staging, MODE 1 (whose mainloop is long) uses one buffer.
+// memory (128-byte swizzle) and written by TMA stores from one staging buffer
+// per warp (a second buffer would cost the mainloop its sixth pipeline stage,
+// which is worth more: 63.5 against 65.5 us on the 1B block's first GEMM).
 // partial is laid out [column tile][row] (fp32).
 // ---------------------------------------------------------------------------
 template <int MODE>
 struct EpiLoadStore2 {
-  static constexpr int kNBuf = MODE == 0 ? 2 : 1;
+  static constexpr int kNBuf = 1;
   static constexpr int kOut2Bytes = MODE == 0 ? 4096 : 8192;  // 32 x 64 bf16, or 32 x 64 fp32 as two 32 x 32 boxes
   static constexpr int kBufBytes = 4096 + kOut2Bytes;
   static constexpr int kSmemPerWarp = kNBuf * kBufBytes;
@@ -636,7 +637,14 @@ struct EpiRowScale {
 };
 
 // ---------------------------------------------------------------------------
-// fp32 output (weight gradients): out = acc.
+// fp32 output (weight gradients): out = acc, or out = acc + out (accumulation
+// over calls).  An optional correction serves the cross-entropy backward,
+// whose gradient G is stored in bf16 and whose label entries' rounding
+// residuals resid_i are kept in fp32: in dW_c = H^T G (output rows = hidden,
+// columns = vocabulary), column v adds resid_i H[i, k] for every row i
+// labelled v, in increasing i.  The rows come bucketed per 256-column
+// vocabulary tile and sorted by (label, row), and are added to the staged
+// tile in shared memory before it is stored.
 // ---------------------------------------------------------------------------
 struct EpiStoreF32 {
   static constexpr int kSmemPerWarp = 2 * 4096;
@@ -647,6 +655,12 @@ struct EpiStoreF32 {
     CUtensorMap tmOut;   // [M, N] fp32, box 32 x 32
     const float* accum;  // null, or the output itself: out = acc + out (accumulation over calls)
     long long ld;        // row stride (elements) of `accum`
+    const float* fix_resid;            // [tokens] label-entry residuals
+    long long fix_col0;                // vocabulary index of this chunk's column 0
+    const int* fix_start;              // [tiles + 1] bucket offsets, or null (no correction)
+    const int2* fix_entries;           // (label, row) sorted within each bucket
+    const __nv_bfloat16* fix_H;        // [tokens, M]: the hidden states
+    int fix_tile0;                     // bucket of this chunk's column 0 (chunk start / 256)
   };
   struct State {
     uint32_t cnt;
@@ -655,10 +669,40 @@ struct EpiStoreF32 {
 
   template <int BN>
   __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
+    static_assert(BN <= 256 && 256 % BN == 0, "a tile lies within one 256-column label bucket");
     const int col0 = c.nb * BN;
     const int row = c.row0 + c.lane;
     int nch = (c.N - col0 + 31) / 32;
     if (nch > BN / 32) nch = BN / 32;
+    // this tile's run of (label, row) entries
+    int e0 = 0, e1 = 0;
+    if (ep.fix_start != nullptr) {
+      const int bkt = ep.fix_tile0 + col0 / 256;
+      e0 = ep.fix_start[bkt];
+      e1 = ep.fix_start[bkt + 1];
+    }
+    // The run is fetched 32 entries at a time: lane l holds entry e0 + l, its
+    // residual, and (for its own output row) H[row of entry j, row] for every
+    // j of the batch, so the whole batch costs three rounds of loads.
+    int2 fe = make_int2(-1, 0);
+    float fr = 0.f;
+    float hv[32];
+    int nfe = 0;
+    auto fetch_batch = [&](int first) {
+      nfe = min(32, e1 - first);
+      fe = make_int2(-1, 0);
+      fr = 0.f;
+      if (c.lane < nfe) {
+        fe = ep.fix_entries[first + c.lane];
+        fr = ep.fix_resid[fe.y];
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int tok = __shfl_sync(0xffffffffu, fe.y, j);
+        hv[j] = (j < nfe && row < c.M) ? __bfloat162float(ep.fix_H[static_cast<size_t>(tok) * c.M + row]) : 0.f;
+      }
+    };
+    if (e0 < e1) fetch_batch(e0);
     for (int ch = 0; ch < nch; ++ch) {
       const int cc = col0 + ch * 32;
       uint4 old[8];
@@ -688,6 +732,27 @@ struct EpiStoreF32 {
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         st_shared_v4(O + sw128_off(c.lane, j), make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+      // entries are sorted by label, so the batch's entries of this 32-column
+      // chunk are consecutive; add them in order (all branches warp-uniform).
+      while (e0 < e1) {
+        const long long vbase = ep.fix_col0 + cc;  // vocabulary index of this chunk's column 0
+        int done = 0;  // entries of the batch left of the next chunk
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (j >= nfe) break;
+          const long long q = static_cast<long long>(__shfl_sync(0xffffffffu, fe.x, j)) - vbase;
+          if (q >= 32) break;
+          ++done;
+          const float rj = __shfl_sync(0xffffffffu, fr, j);
+          if (q >= 0 && row < c.M) {
+            float* sp = reinterpret_cast<float*>(O + sw128_off(c.lane, static_cast<int>(q >> 2))) + (q & 3);
+            *sp += rj * hv[j];
+          }
+        }
+        if (done < nfe) break;      // the rest of the batch lies right of this chunk
+        e0 += nfe;                  // batch used up: fetch the next one
+        if (e0 < e1) fetch_batch(e0);
+      }
       fence_async_smem();
       __syncwarp();
       if (c.lane == 0) {

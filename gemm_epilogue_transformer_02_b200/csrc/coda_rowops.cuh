@@ -156,75 +156,129 @@ __global__ void __launch_bounds__(1024) mean_kernel(const float* __restrict__ lo
 // Cross-entropy backward: exact label entries.  The chunked backward stores the
 // gradient G in bf16; at each row's label entry G = d (p - 1) dominates its dW
 // column, so the rounding dropped there (resid_i, recorded in fp32 by the
-// gradient epilogue) is added back:
-//   dH[i, :] += resid_i W[:, label_i]
+// gradient epilogue) is added back, chunk by chunk:
+//   dH[i, :] += resid_i W[:, label_i]        (ce_label_dh_fix_kernel)
 //   dW[:, v] += sum over rows i with label_i = v (in increasing i) of resid_i H[i, :]
-// Block i handles row i; the first row carrying a label owns that dW column,
-// so every column is updated by one block in a fixed order (no atomics).
-constexpr int kFixThreads = 256;
-constexpr int kFixCols = 8;  // columns of dW per thread per pass
+//                                             (in the dW GEMM's epilogue)
+// The rows are bucketed by the 256-column vocabulary tile of their label and
+// sorted within a bucket by (label, row): a chunk's rows are then one run of
+// the sorted array, a dW tile's label columns one ordered run within it, and
+// every column sums its rows in a fixed order (deterministic, no
+// floating-point atomics).
+constexpr int kLabelTile = 256;  // vocabulary columns per bucket (the GEMM tile width)
 
-__global__ void __launch_bounds__(kFixThreads) ce_bwd_label_fix_kernel(
-    const int64_t* __restrict__ labels, const float* __restrict__ resid, const __nv_bfloat16* __restrict__ H,
-    const __nv_bfloat16* __restrict__ W, float* __restrict__ dH, float* __restrict__ dW, int M, int K,
-    long long V) {
-  __shared__ int rows[kFixThreads];
-  __shared__ int warp_count[kFixThreads / 32];
-  __shared__ int nrows;
-  const int i = blockIdx.x;
+// counts[b] = number of rows whose label lies in vocabulary tile b.
+__global__ void ce_label_count_kernel(const int64_t* __restrict__ labels, int M, long long V, int* counts) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= M) return;
   const long long lab = labels[i];
-  if (lab < 0 || lab >= V) return;  // such a row has no label entry (and no residual)
-  const float ri = resid[i];
-  for (int k = threadIdx.x; k < K; k += kFixThreads)
-    dH[static_cast<size_t>(i) * K + k] += ri * __bfloat162float(W[static_cast<size_t>(k) * V + lab]);
-  int earlier = 0;
-  for (int j = threadIdx.x; j < i; j += kFixThreads) earlier |= (labels[j] == lab);
-  if (__syncthreads_or(earlier)) return;  // an earlier row owns this column
-  // This block owns column `lab`.  Usually no later row repeats the label:
-  // then the column gets resid_i H[i, :] alone.
-  int later = 0;
-  for (int j = i + 1 + static_cast<int>(threadIdx.x); j < M; j += kFixThreads) later |= (labels[j] == lab);
-  if (!__syncthreads_or(later)) {
-    for (int k = threadIdx.x; k < K; k += kFixThreads)
-      dW[static_cast<size_t>(k) * V + lab] += ri * __bfloat162float(H[static_cast<size_t>(i) * K + k]);
-    return;
-  }
-  // Otherwise add the residuals of rows j >= i carrying the same label, in
-  // increasing j, kFixThreads * kFixCols columns per pass.
-  for (int kbase = 0; kbase < K; kbase += kFixThreads * kFixCols) {
-    float acc[kFixCols];
+  if (lab >= 0 && lab < V) atomicAdd(&counts[lab / kLabelTile], 1);
+}
+
+// Exclusive scan of counts[0, n) into start[0, n] (start[n] = total) and a copy
+// of it into cursor[0, n).  One block of 1024 threads walks the array.
+__global__ void __launch_bounds__(1024) ce_label_scan_kernel(const int* __restrict__ counts, int n, int* start,
+                                                             int* cursor) {
+  __shared__ int warp_sums[32];
+  __shared__ int carry;
+  const int lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < n; base += 1024) {
+    const int i = base + static_cast<int>(threadIdx.x);
+    const int v = i < n ? counts[i] : 0;
+    int x = v;  // inclusive scan within the warp
 #pragma unroll
-    for (int q = 0; q < kFixCols; ++q) acc[q] = 0.f;
-    for (int j0 = i; j0 < M; j0 += kFixThreads) {
-      const int j = j0 + threadIdx.x;
-      const bool match = j < M && labels[j] == lab;
-      const unsigned ballot = __ballot_sync(0xffffffffu, match);
-      if ((threadIdx.x & 31) == 0) warp_count[threadIdx.x >> 5] = __popc(ballot);
-      __syncthreads();
-      int base = 0;
-      for (int w = 0; w < (threadIdx.x >> 5); ++w) base += warp_count[w];
-      if (match) rows[base + __popc(ballot & ((1u << (threadIdx.x & 31)) - 1u))] = j;
-      if (threadIdx.x == 0) {
-        int t = 0;
-        for (int w = 0; w < kFixThreads / 32; ++w) t += warp_count[w];
-        nrows = t;
-      }
-      __syncthreads();
-      for (int q = 0; q < nrows; ++q) {
-        const int jr = rows[q];
-        const float rj = resid[jr];
-#pragma unroll
-        for (int s2 = 0; s2 < kFixCols; ++s2) {
-          const int k = kbase + s2 * kFixThreads + threadIdx.x;
-          if (k < K) acc[s2] += rj * __bfloat162float(H[static_cast<size_t>(jr) * K + k]);
-        }
-      }
-      __syncthreads();
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
     }
+    if (lane == 31) warp_sums[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+      int w = warp_sums[lane];
 #pragma unroll
-    for (int s2 = 0; s2 < kFixCols; ++s2) {
-      const int k = kbase + s2 * kFixThreads + threadIdx.x;
-      if (k < K) dW[static_cast<size_t>(k) * V + lab] += acc[s2];
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      warp_sums[lane] = w;
+    }
+    __syncthreads();
+    const int excl = carry + (wid > 0 ? warp_sums[wid - 1] : 0) + x - v;
+    if (i < n) {
+      start[i] = excl;
+      cursor[i] = excl;
+    }
+    __syncthreads();
+    if (threadIdx.x == 1023) carry = excl + v;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) start[n] = carry;
+}
+
+// Drops (label, row) of every row with a label in [0, V) into its bucket, in
+// arrival order.
+__global__ void ce_label_fill_kernel(const int64_t* __restrict__ labels, int M, long long V, int* cursor,
+                                     int2* __restrict__ unsorted) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= M) return;
+  const long long lab = labels[i];
+  if (lab < 0 || lab >= V) return;
+  const int pos = atomicAdd(&cursor[lab / kLabelTile], 1);
+  unsorted[pos] = make_int2(static_cast<int>(lab), i);
+}
+
+// Places every entry at its rank by (label, row) within its bucket (the keys
+// are distinct, so the result does not depend on the arrival order).
+__global__ void ce_label_sort_kernel(const int2* __restrict__ unsorted, const int* __restrict__ start, int n,
+                                     int2* __restrict__ sorted) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= start[n]) return;
+  const int2 me = unsorted[e];
+  const int b = me.x / kLabelTile;
+  const int s0 = start[b];
+  const int s1 = start[b + 1];
+  int rank = 0;
+  for (int f = s0; f < s1; ++f) {
+    const int2 o = unsorted[f];
+    rank += (o.x < me.x || (o.x == me.x && o.y < me.y)) ? 1 : 0;
+  }
+  sorted[s0 + rank] = me;
+}
+
+// dH[i, :] += resid_i W[:, label_i] for the rows whose label lies in buckets
+// [b0, b1) (one vocabulary chunk), run right after that chunk's GEMMs, which
+// leave the chunk of W in L2.  One warp per (row, 256 columns of dH): each
+// lane gathers its 8 elements of W's label column at once, then updates 8
+// coalesced 128-byte segments of the dH row; every element is written by one
+// thread once.
+constexpr int kDhFixSpan = 8;  // 32-column slices per warp item
+__global__ void ce_label_dh_fix_kernel(const int2* __restrict__ entries, const int* __restrict__ start, int b0,
+                                       int b1, const float* __restrict__ resid, const __nv_bfloat16* __restrict__ W,
+                                       long long V, int K, float* __restrict__ dH) {
+  const int first = start[b0];
+  const long long n = start[b1] - first;
+  const int groups = (K + 32 * kDhFixSpan - 1) / (32 * kDhFixSpan);
+  const int lane = threadIdx.x & 31;
+  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; w < n * groups;
+       w += nwarps) {
+    const int2 en = entries[first + static_cast<int>(w / groups)];
+    const int kbase = static_cast<int>(w % groups) * 32 * kDhFixSpan + lane;
+    const float ri = resid[en.y];
+    float wv[kDhFixSpan];
+#pragma unroll
+    for (int u = 0; u < kDhFixSpan; ++u) {
+      const int k = kbase + 32 * u;
+      wv[u] = k < K ? __bfloat162float(W[static_cast<size_t>(k) * V + en.x]) : 0.f;
+    }
+    float* d = dH + static_cast<size_t>(en.y) * K;
+#pragma unroll
+    for (int u = 0; u < kDhFixSpan; ++u) {
+      const int k = kbase + 32 * u;
+      if (k < K) d[k] += ri * wv[u];
     }
   }
 }

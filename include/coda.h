@@ -204,8 +204,9 @@ coda_status_t coda_lmhead_ce(const uint16_t* H, const uint16_t* W, const int64_t
                              float* loss_out, float* lse_out, float* mean_out, void* ws, size_t ws_bytes,
                              int64_t M, int64_t V, int64_t K, void* stream);
 
-/* Bytes of workspace coda_lmhead_ce_bwd needs (one bf16 gradient chunk of
- * M x min(V, 4096) and M fp32 residuals). */
+/* Bytes of workspace coda_lmhead_ce_bwd needs: one bf16 gradient chunk of
+ * M x min(V, 4096), M fp32 residuals, and the rows bucketed by label (three
+ * int arrays of ceil(V / 256) entries and two of M (label, row) pairs). */
 size_t coda_lmhead_ce_bwd_workspace_size(int64_t M, int64_t V);
 
 /* Backward of coda_lmhead_ce, block-local (section "CODA: the secret in the
@@ -218,9 +219,10 @@ size_t coda_lmhead_ce_bwd_workspace_size(int64_t M, int64_t V);
  * chunk's logits and its epilogue writes G_chunk (bf16, in the workspace;
  * the logits are never stored), then dH += G_chunk W_chunk^T and
  * dW_chunk = H^T G_chunk.  The label entry d_i (p - 1) dominates its dW
- * column, so the part of it that bf16 drops is kept in fp32 and added back
- * afterwards (deterministically, without atomics).  A label outside [0, V)
- * contributes no onehot term.  H [M, K] bf16,
+ * column, so the part of it that bf16 drops is kept in fp32 and added back in
+ * the epilogues of the dH and dW GEMMs (rows bucketed by label beforehand;
+ * each dW column sums its rows in increasing row order, so the result is
+ * deterministic).  A label outside [0, V) contributes no onehot term.  H [M, K] bf16,
  * W [K, V] bf16, labels [M] int64, lse [M] fp32, d_loss and r [M] fp32 or NULL,
  * ws >= coda_lmhead_ce_bwd_workspace_size(M, V). */
 coda_status_t coda_lmhead_ce_bwd(const uint16_t* H, const uint16_t* W, const int64_t* labels, const float* lse,

@@ -65,3 +65,29 @@ def test_lmhead_ce_bwd_fullsize_sampled():
     dW_ref = np.stack([O.matmul(Hb.T, O.lmhead_ce_grad_chunk(Hb, Wb[:, [v]], lab, lse_ref, int(v), d))[:, 0]
                        for v in cols], axis=1)
     check("dW (sampled columns)", dW[:, torch.as_tensor(cols, device="cuda")], dW_ref)
+
+
+def test_lmhead_ce_bwd_repeated_labels_and_determinism():
+    """Many tokens share a few labels, placed on both sides of 256-column
+    bucket and 4096-column chunk boundaries; two tokens carry labels outside
+    [0, V) (no onehot term).  Every dW label column sums its tokens' exact
+    label entries in a fixed order, so two calls agree bit for bit."""
+    M, K, V = 300, 136, 5000
+    g = synth.make_gen(650)
+    H = synth.normal_bf16(g, (M, K))
+    W = synth.normal_bf16(g, (K, V), std=1.5 / math.sqrt(K))
+    pool = torch.tensor([0, 1, 255, 256, 4095, 4096, 4999], dtype=torch.int64)
+    labels = pool[torch.randint(0, len(pool), (M,), generator=g)]
+    Hd, Wd, Ld = dev(H), dev(W), dev(labels)
+    _, lse, _ = C.lmhead_ce(Hd, Wd, Ld)  # lse of every token (labels do not enter it)
+    bad = labels.clone()
+    bad[5], bad[200] = -1, V
+    Bd = dev(bad)
+    dH, dW = C.lmhead_ce_bwd(Hd, Wd, Bd, lse)
+    dH2, dW2 = C.lmhead_ce_bwd(Hd, Wd, Bd, lse)
+    C.poll_status()
+    assert torch.equal(dH, dH2) and torch.equal(dW, dW2)
+    ref = O.cross_entropy_backward_unfused(b(H), b(W), bad.numpy())
+    check("dH", dH, ref["dH"])
+    check("dW", dW, ref["dW"])
+    check("dW label columns", dW[:, dev(pool)], ref["dW"][:, pool.numpy()])
