@@ -548,6 +548,54 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
                               "gemm_swiglu_bwd_tflops": round(f_swb / k[0] / 1e9, 1)}
     del act, h2, p2, gu, d_h2, d_gu
 
+    # FP8 (e4m3) block on the same workload, timed step by step beside the bf16
+    # block (an L2 flush between them): per-tensor scales, hg8's scale from the
+    # previous step's amax (delayed scaling; the update is part of the step)
+    res_d = inp.res.to(dev)
+    x8, _, sx = C.fp8_quantize(x)
+    W1t8, _, sw1 = C.fp8_quantize(W1, transpose=True)
+    W2t8, _, sw2 = C.fp8_quantize(W2, transpose=True)
+    s_hg = torch.ones(1, dtype=torch.float32, device=dev)
+    b8 = {"h": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
+          "hg8": torch.empty(M_TOK, D, dtype=torch.uint8, device=dev),
+          "amax": torch.empty(1, dtype=torch.float32, device=dev),
+          "partial": torch.empty(C.partial_cols(D), M_TOK, dtype=torch.float32, device=dev),
+          "r": torch.empty(M_TOK, dtype=torch.float32, device=dev)}
+    out8 = torch.empty(M_TOK, N2, dtype=torch.bfloat16, device=dev)
+    out16 = torch.empty(M_TOK, N2, dtype=torch.bfloat16, device=dev)
+    b16 = {"h": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
+           "hg": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
+           "partial": torch.empty(C.partial_cols(D), M_TOK, dtype=torch.float32, device=dev),
+           "r": torch.empty(M_TOK, dtype=torch.float32, device=dev)}
+
+    def f8(evs=None):
+        C.gemm_rmsnorm_gemm(x, res_d, W1, W2, gamma, EPS, out=out16, bufs=b16)
+        if evs:
+            evs[0].record(stream)
+            flush.zero_()
+            evs[1].record(stream)
+        C.gemm_res_partialrms_fp8(x8, sx, W1t8, sw1, res_d, gamma, s_hg, h_out=b8["h"], hg8_out=b8["hg8"],
+                                  amax_out=b8["amax"], partial_out=b8["partial"])
+        if evs:
+            evs[2].record(stream)
+        C.gemm_rowscale_partial_fp8(b8["hg8"], s_hg, W2t8, sw2, b8["partial"], D, EPS, out=out8, r_out=b8["r"])
+        C.fp8_scale_from_amax(b8["amax"], scale_out=s_hg)
+
+    for _ in range(3):
+        f8(None)
+    _, parts = timed(f8, steps, 0, inner_events=3)
+    k = [sum(p[i] for p in parts) / len(parts) for i in range(4)]
+    f_blk = 2.0 * M_TOK * D * (D + N2)
+    ms8 = k[2] + k[3]
+    res["fp8_block"] = {"ms": round(ms8, 4), "tflops": round(f_blk / ms8 / 1e9, 1),
+                        "frac_of_nominal_fp8_4500": round(f_blk / (ms8 / 1e3) / 4.5e15, 4),
+                        "gemm_res_partialrms_fp8_ms": round(k[2], 4),
+                        "gemm_rowscale_partial_fp8_ms": round(k[3], 4),
+                        "gemm_rowscale_partial_fp8_tflops": round(2.0 * M_TOK * D * N2 / k[3] / 1e9, 1),
+                        "bf16_block_ms_same_steps": round(k[0], 4), "speedup_vs_bf16_block": round(k[0] / ms8, 4),
+                        "scaling": "per-tensor e4m3; hg8 scale from the previous step's amax"}
+    del res_d, x8, W1t8, W2t8, b8, out8, out16, b16
+
     # QKV projection with RoPE in its epilogue (1B attention input: 32 q + 8 k + 8 v heads of 64)
     n_qkv, rope_cols = 48 * 64, 40 * 64
     W_qkv = synth.normal_bf16(synth.make_gen(8 + 1000 * rank), (D, n_qkv), std=0.02).to(dev)

@@ -67,6 +67,10 @@ _SIGS = {
     "coda_unfused_add": (_ST, [_P, _P, _P, _I64, _P]),
     "coda_unfused_rmsnorm": (_ST, [_P, _P, _F, _P, _P, _I64, _I64, _P]),
     "coda_selftest_bounded_wait": (_ST, [_I64, _P, _P]),
+    "coda_fp8_quantize": (_ST, [_P, _I64, _I64, ctypes.c_int, _P, _P, _P, _P]),
+    "coda_fp8_scale_from_amax": (_ST, [_P, _P, _P]),
+    "coda_gemm_res_partialrms_fp8": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "coda_gemm_rowscale_partial_fp8": (_ST, [_P, _P, _P, _P, _P, _I64, _I64, _F, _P, _P, _I64, _I64, _I64, _P]),
 }
 
 _lib = None
@@ -465,6 +469,88 @@ def gemm_rmsnorm_gemm(x, res, W1, W2, gamma, eps: float, out=None, bufs=None, fo
         r = rms_reduce(partial, N, eps, r_out=b.get("r"))
         out = gemm_rowscale(hg, W2, r, out=out)
     return {"out": out, "h": h, "hg": hg, "partial": partial, "r": r}
+
+
+# ---------------------------------------------------------------- FP8 (e4m3)
+
+U8 = torch.uint8
+
+
+def fp8_quantize(src, transpose: bool = False, dst=None, amax=None, scale=None):
+    """Per-tensor e4m3 quantisation of a bf16 [rows, cols] tensor (its own
+    scale = amax / 448).  Returns (codes uint8 [rows, cols] or, transposed,
+    [cols, rows]; amax [1] fp32; scale [1] fp32)."""
+    rows, cols = src.shape
+    _need(src, BF16, "src")
+    if dst is None:
+        dst = _empty((cols, rows) if transpose else (rows, cols), U8, src)
+    amax = _empty((1,), F32, src) if amax is None else amax
+    scale = _empty((1,), F32, src) if scale is None else scale
+    _call("coda_fp8_quantize", _ptr(src), rows, cols, 1 if transpose else 0, _ptr(dst), _ptr(amax), _ptr(scale),
+          _stream())
+    return dst, amax, scale
+
+
+def fp8_scale_from_amax(amax, scale_out=None):
+    """scale = amax / 448 (1 for 0), on the device."""
+    _need(amax, F32, "amax", (1,))
+    scale_out = _empty((1,), F32, amax) if scale_out is None else scale_out
+    _call("coda_fp8_scale_from_amax", _ptr(amax), _ptr(scale_out), _stream())
+    return scale_out
+
+
+def gemm_res_partialrms_fp8(x8, sx, Wt8, sw, res, gamma, s_hg, *, h=True, h_out=None, hg8_out=None,
+                            amax_out=None, partial_out=None):
+    """First GEMM of the FP8 block.  Returns (h bf16 or None, hg8 e4m3 codes,
+    amax [1] = max |gamma * h|, partial [T, M])."""
+    M, K = x8.shape
+    N = Wt8.shape[0]
+    _need(x8, U8, "x8")
+    _need(Wt8, U8, "Wt8", (N, K))
+    for t, nm in ((sx, "sx"), (sw, "sw"), (s_hg, "s_hg")):
+        _need(t, F32, nm, (1,))
+    if res is not None:
+        _need(res, BF16, "res", (M, N))
+    _need(gamma, BF16, "gamma", (N,))
+    if h and h_out is None:
+        h_out = _empty((M, N), BF16, x8)
+    hg8_out = _empty((M, N), U8, x8) if hg8_out is None else hg8_out
+    amax_out = _empty((1,), F32, x8) if amax_out is None else amax_out
+    partial_out = _empty((partial_cols(N), M), F32, x8) if partial_out is None else partial_out
+    _call("coda_gemm_res_partialrms_fp8", _ptr(x8), _ptr(sx), _ptr(Wt8), _ptr(sw), _ptr(res), _ptr(gamma),
+          _ptr(s_hg), _ptr(h_out if h else None), _ptr(hg8_out), _ptr(amax_out), _ptr(partial_out), M, N, K,
+          _stream())
+    return (h_out if h else None), hg8_out, amax_out, partial_out
+
+
+def gemm_rowscale_partial_fp8(A8, sa, Wt8, sw, partial, N_norm: int, eps: float, out=None, r_out=None):
+    """Second GEMM of the FP8 block: out = r * sa * sw * (A8 Wt8^T), r from
+    the partials.  Returns (out bf16, r)."""
+    M, K = A8.shape
+    N = Wt8.shape[0]
+    _need(A8, U8, "A8")
+    _need(Wt8, U8, "Wt8", (N, K))
+    _need(sa, F32, "sa", (1,))
+    _need(sw, F32, "sw", (1,))
+    _need(partial, F32, "partial", (partial.shape[0], M))
+    out = _empty((M, N), BF16, A8) if out is None else out
+    r_out = _empty((M,), F32, A8) if r_out is None else r_out
+    _call("coda_gemm_rowscale_partial_fp8", _ptr(A8), _ptr(sa), _ptr(Wt8), _ptr(sw), _ptr(partial),
+          partial.shape[0], N_norm, float(eps), _ptr(r_out), _ptr(out), M, N, K, _stream())
+    return out, r_out
+
+
+def gemm_rmsnorm_gemm_fp8(x8, sx, W1t8, sw1, res, gamma, s_hg, W2t8, sw2, eps: float, out=None, bufs=None):
+    """The FP8 block in two launches (plus the zeroing of amax): returns
+    dict(out, h, hg8, amax, partial, r).  s_hg is the scale hg8 is quantised
+    with (delayed scaling: fp8_scale_from_amax of an earlier call's amax)."""
+    N = W1t8.shape[0]
+    b = bufs or {}
+    h, hg8, amax, partial = gemm_res_partialrms_fp8(x8, sx, W1t8, sw1, res, gamma, s_hg, h_out=b.get("h"),
+                                                    hg8_out=b.get("hg8"), amax_out=b.get("amax"),
+                                                    partial_out=b.get("partial"))
+    out, r = gemm_rowscale_partial_fp8(hg8, s_hg, W2t8, sw2, partial, N, eps, out=out, r_out=b.get("r"))
+    return {"out": out, "h": h, "hg8": hg8, "amax": amax, "partial": partial, "r": r}
 
 
 def unfused_block(x, res, W1, W2, gamma, eps: float, out=None, bufs=None):

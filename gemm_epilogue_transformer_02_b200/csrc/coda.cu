@@ -106,6 +106,21 @@ bool tmap2d(CUtensorMap* m, const void* base, bool f32, uint64_t cols, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
+// e4m3 operands and outputs: 1-byte elements, 128-byte inner boxes (one swizzle row).
+bool tmap2d_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t stride,
+               uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {stride};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Operand maps of the mainloop.  A: [M, K] K-major (box 64 x 128) or stored
 // transposed as [K, M] (MN-major, box 64 x 64).  B: [K, N] MN-major (box 64 x 64)
 // or stored transposed as [N, K] (K-major, box 64 x BN).
@@ -141,6 +156,8 @@ enum KernelKind : uint32_t {
   kKindF32KK,
   kKindRope,
   kKindBlock,
+  kKindResPartialF8,
+  kKindRowScaleF8,
 };
 
 // Vocabulary columns per chunk of the cross-entropy backward: the chunk's
@@ -925,6 +942,130 @@ coda_status_t coda_selftest_bounded_wait(int64_t limit_ns, int* gave_up_dev, voi
   bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_ns),
                                                                                 gave_up_dev);
   return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}
+
+// ------------------------------------------------------------- FP8 (e4m3)
+
+coda_status_t coda_fp8_quantize(const uint16_t* src, int64_t rows, int64_t cols, int transpose, uint8_t* dst,
+                                float* amax_out, float* scale_out, void* stream) {
+  CODA_CHECK(rows >= 0 && rows < (int64_t(1) << 31) && dim_ok(cols) && (!transpose || rows % 4 == 0) &&
+                 (!transpose || rows <= int64_t(65535) * kQT),
+             CODA_ERR_SHAPE);
+  CODA_CHECK(src && dst && amax_out && scale_out, CODA_ERR_NULL);
+  CODA_CHECK(al16(src) && al16(dst) && al16(amax_out) && al16(scale_out), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(amax_out, 0, sizeof(float), s) != cudaSuccess) return CODA_ERR_LAUNCH;
+  const size_t n8 = static_cast<size_t>(rows) * static_cast<size_t>(cols) / 8;
+  if (n8 > 0) {
+    const int grid = info->sms * 4;
+    amax_bf16_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(src), n8,
+                                          reinterpret_cast<unsigned*>(amax_out));
+    if (transpose) {
+      const dim3 g(static_cast<unsigned>((cols + kQT - 1) / kQT), static_cast<unsigned>((rows + kQT - 1) / kQT));
+      quantize_e4m3_t_kernel<<<g, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(src), static_cast<int>(rows),
+                                               static_cast<int>(cols), amax_out, dst);
+    } else {
+      quantize_e4m3_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(src), n8, amax_out, dst);
+    }
+  }
+  fp8_scale_kernel<<<1, 1, 0, s>>>(amax_out, scale_out);
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}
+
+coda_status_t coda_fp8_scale_from_amax(const float* amax, float* scale_out, void* stream) {
+  CODA_CHECK(amax && scale_out, CODA_ERR_NULL);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  fp8_scale_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(amax, scale_out);
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}
+
+namespace {
+inline bool fp8_dim_ok(int64_t v) { return dim_ok(v) && v % 16 == 0; }
+}  // namespace
+
+coda_status_t coda_gemm_res_partialrms_fp8(const uint8_t* x8, const float* sx, const uint8_t* Wt8, const float* sw,
+                                           const uint16_t* res, const uint16_t* gamma, const float* s_hg,
+                                           uint16_t* h_out, uint8_t* hg8_out, float* amax_out, float* partial,
+                                           int64_t M, int64_t N, int64_t K, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && fp8_dim_ok(N) && fp8_dim_ok(K), CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(x8 && sx && Wt8 && sw && gamma && s_hg && hg8_out && amax_out && partial, CODA_ERR_NULL);
+  CODA_CHECK(al16(x8) && al16(Wt8) && al16(res) && al16(gamma) && al16(h_out) && al16(hg8_out) && al16(partial) &&
+                 al16(amax_out),
+             CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  using Epi = EpiLoadStore2<2>;
+  GemmParams<Epi> p{};
+  bool ok = tmap2d_u8(&p.tmA, x8, K, M, K, 128, kBM) && tmap2d_u8(&p.tmB, Wt8, K, N, K, 128, 128) &&
+            tmap2d_u8(&p.ep.tmOut2, hg8_out, N, M, N, 128, 32);
+  if (h_out) ok = ok && map_out_bf16(&p.ep.tmOut1, h_out, M, N, N);
+  if (!ok) return CODA_ERR_INTERNAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(amax_out, 0, sizeof(float), s) != cudaSuccess) return CODA_ERR_LAUNCH;
+  p.ep.in = reinterpret_cast<const __nv_bfloat16*>(res);
+  p.ep.gamma = reinterpret_cast<const __nv_bfloat16*>(gamma);
+  p.ep.partial = partial;
+  p.ep.has_out1 = h_out != nullptr;
+  p.ep.has_out2 = 1;
+  p.ep.sa = sx;
+  p.ep.sb = sw;
+  p.ep.s_out = s_hg;
+  p.ep.amax = reinterpret_cast<unsigned*>(amax_out);
+  const int n_nt = static_cast<int>((N + 255) / 256);
+  return run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M),
+                                                                    static_cast<int>(N), static_cast<int>(K), n_nt,
+                                                                    raster_group(M, N, K), kKindResPartialF8, s);
+}
+
+coda_status_t coda_gemm_rowscale_partial_fp8(const uint8_t* A8, const float* sa, const uint8_t* Wt8, const float* sw,
+                                             const float* partial, int64_t T, int64_t N_norm, float eps,
+                                             float* r_out, uint16_t* out, int64_t M, int64_t N, int64_t K,
+                                             void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(N) && fp8_dim_ok(K) && T > 0 && T <= 1 << 20 &&
+                 N_norm > 0 && eps >= 0.f,
+             CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(A8 && sa && Wt8 && sw && partial && out, CODA_ERR_NULL);
+  CODA_CHECK(al16(A8) && al16(Wt8) && al16(partial) && al16(r_out) && al16(out), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  using Epi = EpiRowScaleF8;
+  GemmParams<Epi> p{};
+  if (!(tmap2d_u8(&p.tmA, A8, K, M, K, 128, kBM) && tmap2d_u8(&p.tmB, Wt8, K, N, K, 128, 128) &&
+        map_out_bf16(&p.ep.tmOut, out, M, N, N)))
+    return CODA_ERR_INTERNAL;
+  p.ep.partial = partial;
+  p.ep.T = static_cast<int>(T);
+  p.ep.inv_n = 1.0f / static_cast<float>(N_norm);
+  p.ep.eps = eps;
+  p.ep.r_out = r_out;
+  p.ep.sa = sa;
+  p.ep.sb = sw;
+  const int n_nt = static_cast<int>((N + 255) / 256);
+  return run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M),
+                                                                    static_cast<int>(N), static_cast<int>(K), n_nt,
+                                                                    raster_group(M, N, K), kKindRowScaleF8,
+                                                                    static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -54,6 +54,18 @@ struct TileSched {
   }
 };
 
+// Operand type of the mainloop: bf16 (kind::f16) unless the epilogue declares
+// kFp8 = true (e4m3 operands, kind::f8f6f4).  A k-block is 128 bytes of K per
+// row either way: 64 bf16 or 128 e4m3 elements.
+template <class E, class = void>
+struct epi_fp8 {
+  static constexpr bool value = false;
+};
+template <class E>
+struct epi_fp8<E, decltype(void(E::kFp8))> {
+  static constexpr bool value = E::kFp8;
+};
+
 template <class Epi>
 struct GemmParams {
   CUtensorMap tmA;
@@ -111,6 +123,9 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
   static_assert(!PAIR || BN == 256, "pair tiles are 256 x 256");
   constexpr int kTileM = PAIR ? 2 * kBM : kBM;   // rows per tile
   constexpr int kBCols = PAIR ? BN / 2 : BN;     // B columns loaded by this CTA
+  constexpr bool kF8 = epi_fp8<Epi>::value;
+  constexpr int kKb = kF8 ? 2 * kBK : kBK;       // K elements per k-block (128 bytes per row)
+  static_assert(!kF8 || (!A_MN && !B_MN && PAIR), "e4m3 operands: K-major A and B, CTA pairs");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -166,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const WaitCtx w{abort_flag, p.wait_ns};
-  const int nkb = (p.K + kBK - 1) / kBK;
+  const int nkb = (p.K + kKb - 1) / kKb;
   const int ntiles = p.sched.ntiles;
 
   if (warp == 0) {
@@ -193,14 +208,14 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
             if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * S::kStageBytes);
             const uint32_t fb = full0 + stage * 8;
             if (!A_MN) {
-              tma_load_2d_pair(a, &p.tmA, fb, kb * kBK, arow);
+              tma_load_2d_pair(a, &p.tmA, fb, kb * kKb, arow);
             } else {
 #pragma unroll
               for (int j = 0; j < kBM / 64; ++j)
                 tma_load_2d_pair(a + j * (64 * kBK * 2), &p.tmA, fb, arow + j * 64, kb * kBK);
             }
             if (!B_MN) {
-              tma_load_2d_pair(b, &p.tmB, fb, kb * kBK, bcol);
+              tma_load_2d_pair(b, &p.tmB, fb, kb * kKb, bcol);
             } else if (Epi::kPairedB) {
               // rank 0 holds the gate half, rank 1 the up half of the accumulator columns
               const CUtensorMap* m = rank == 0 ? &p.tmB : &p.tmB2;
@@ -261,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, BN, A_MN, B_MN);
+      constexpr uint32_t kIdesc = kF8 ? idesc_e4m3_f32(kTileM, BN) : idesc_bf16_f32(kTileM, BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -286,7 +301,9 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
                                      : sdesc_sw128(a0 + kk * 32, 16, 1024);
             const uint64_t bd = B_MN ? sdesc_sw128(b0 + kk * 16 * 128, 64 * kBK * 2, 1024)
                                      : sdesc_sw128(b0 + kk * 32, 16, 1024);
-            if (PAIR)
+            if (kF8)
+              tc_mma_f8_pair(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            else if (PAIR)
               tc_mma_bf16_pair(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
             else
               tc_mma_bf16(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
@@ -399,6 +416,10 @@ __device__ __forceinline__ float acc_at(const uint32_t (&v0)[32], const uint32_t
 //     h = acc + res;  out1 = bf16(h);  out2 = hg = bf16(gamma * h);  partial += h^2
 //   MODE 1 (backward of the row-scaled second GEMM, acc = P = dOut W2^T):
 //     in = hg;  out1 = y = bf16(r * hg);  out2 = d_hg = r * P (fp32);  partial += hg * P
+//   MODE 2 (first GEMM of the FP8 block, e4m3 operands with per-tensor scales):
+//     h = acc * sa * sb + res;  out1 = bf16(h);  partial += h^2;
+//     out2 = hg8 = e4m3(gamma * h / s_out) (round to nearest even, saturating);
+//     amax = max |gamma * h| (the next call's scale, by atomic max on its bits)
 // The input tile is read straight into registers (each thread its own row,
 // 128 bytes per 64-column chunk) one chunk ahead, and the first chunk of the
 // next tile is requested before this tile's last chunk is processed, so its
@@ -411,7 +432,9 @@ __device__ __forceinline__ float acc_at(const uint32_t (&v0)[32], const uint32_t
 template <int MODE>
 struct EpiLoadStore2 {
   static constexpr int kNBuf = 1;
-  static constexpr int kOut2Bytes = MODE == 0 ? 4096 : 8192;  // 32 x 64 bf16, or 32 x 64 fp32 as two 32 x 32 boxes
+  static constexpr bool kFp8 = MODE == 2;
+  // out2 staging: 32 x 64 bf16; 32 x 64 fp32 as two 32 x 32 boxes; or 32 x 128 e4m3 (two chunks)
+  static constexpr int kOut2Bytes = MODE == 1 ? 8192 : 4096;
   static constexpr int kBufBytes = 4096 + kOut2Bytes;
   static constexpr int kSmemPerWarp = kNBuf * kBufBytes;
   static constexpr int kBarsPerWarp = 0;
@@ -425,6 +448,10 @@ struct EpiLoadStore2 {
     const float* r;              // MODE 1
     float* partial;              // [T, M] or null
     int has_out1, has_out2;
+    const float* sa;             // MODE 2: scales of the e4m3 operands A and B
+    const float* sb;
+    const float* s_out;          // MODE 2: scale hg8 is quantised with
+    unsigned* amax;              // MODE 2: running max |hg| (fp32 bits; zeroed by the caller)
   };
 
   struct State {
@@ -458,6 +485,11 @@ struct EpiLoadStore2 {
     const bool rows_live = c.row0 < c.M;
     float rs = 1.f;
     if (MODE == 1) rs = (row < c.M) ? __ldg(ep.r + row) : 0.f;
+    float asc = 1.f, inv_s = 1.f, amx = 0.f;
+    if (MODE == 2) {
+      asc = __ldg(ep.sa) * __ldg(ep.sb);
+      inv_s = 1.0f / __ldg(ep.s_out);
+    }
 
     if (st.pre_col != col0 || st.pre_row != row) load_chunk(ep, c.M, c.N, row, col0, st.pre);
     float ss = 0.f;
@@ -491,12 +523,38 @@ struct EpiLoadStore2 {
       __syncwarp();
       uint32_t v0[32], v1[32];
       tmem_ld64(c.taddr + ch * 64, v0, v1);
+      uint32_t q8lo = 0, q8hi = 0;  // MODE 2: codes of the even j, stored with the odd j
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const uint32_t off = sw128_off(c.lane, j);
         const uint32_t inw[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
         uint32_t o1[4];
-        if (MODE == 0) {
+        if (MODE == 2) {
+          const uint4 g4 = cc + j * 8 < c.N ? __ldg(reinterpret_cast<const uint4*>(ep.gamma + cc + j * 8))
+                                            : make_uint4(0, 0, 0, 0);
+          const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
+          uint32_t q[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float h0 = fmaf(acc_at(v0, v1, j * 8 + 2 * e), asc, bf16lo(inw[e]));
+            const float h1 = fmaf(acc_at(v0, v1, j * 8 + 2 * e + 1), asc, bf16hi(inw[e]));
+            ss = fmaf(h0, h0, ss);
+            ss = fmaf(h1, h1, ss);
+            o1[e] = pack_bf16x2(h0, h1);
+            const float g0 = h0 * bf16lo(gw[e]);
+            const float g1 = h1 * bf16hi(gw[e]);
+            amx = fmaxf(amx, fmaxf(fabsf(g0), fabsf(g1)));
+            q[e] = pack_e4m3x2(g0 * inv_s, g1 * inv_s);
+          }
+          // 8 codes per j; two j make one 16-byte unit of the 128-column e4m3 row
+          const uint32_t lo = q[0] | (q[1] << 16), hi = q[2] | (q[3] << 16);
+          if (j & 1) {
+            st_shared_v4(G + sw128_off(c.lane, (ch & 1) * 4 + (j >> 1)), make_uint4(q8lo, q8hi, lo, hi));
+          } else {
+            q8lo = lo;
+            q8hi = hi;
+          }
+        } else if (MODE == 0) {
           uint32_t o2[4];
           uint4 g4 = make_uint4(0, 0, 0, 0);  // gamma absent: hg is neither formed nor stored
           if (ep.gamma != nullptr && cc + j * 8 < c.N)
@@ -542,14 +600,23 @@ struct EpiLoadStore2 {
       if (c.lane == 0 && rows_live) {
         if (ep.has_out1) tma_store_2d(&ep.tmOut1, R, cc, c.row0);
         if (ep.has_out2) {
-          tma_store_2d(&ep.tmOut2, G, cc, c.row0);
-          if (MODE == 1 && cc + 32 < c.N) tma_store_2d(&ep.tmOut2, G + 4096, cc + 32, c.row0);
+          if (MODE == 2) {
+            // the e4m3 row holds two chunks: store after the odd one (or a lone last one)
+            if ((ch & 1) || ch + 1 == nch) tma_store_2d(&ep.tmOut2, G, col0 + (ch & ~1) * 64, c.row0);
+          } else {
+            tma_store_2d(&ep.tmOut2, G, cc, c.row0);
+            if (MODE == 1 && cc + 32 < c.N) tma_store_2d(&ep.tmOut2, G + 4096, cc + 32, c.row0);
+          }
         }
       }
       if (c.lane == 0) bulk_commit();
       ++st.cnt;
     }
     if (ep.partial != nullptr && row < c.M) ep.partial[static_cast<size_t>(c.nb) * c.M + row] = ss;
+    if (MODE == 2) {
+      const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(amx));  // |hg| >= 0: bits order as values
+      if (c.lane == 0 && m != 0u) atomicMax(ep.amax, m);
+    }
     return true;
   }
 
@@ -579,6 +646,8 @@ struct EpiRowScale {
     int T;
     float inv_n, eps;
     float* r_out;          // [M] or null (written when partial is given)
+    const float* sa;       // e4m3 operands: per-tensor scales of A and B (both null otherwise)
+    const float* sb;
   };
   struct State {
     uint32_t cnt;
@@ -605,6 +674,7 @@ struct EpiRowScale {
     } else if (ep.r != nullptr) {
       rs = (row < c.M) ? __ldg(ep.r + row) : 0.f;
     }
+    if (ep.sa != nullptr) rs *= __ldg(ep.sa) * __ldg(ep.sb);  // dequantise with the row scale
     for (int ch = 0; ch < nch; ++ch) {
       uint8_t* O = c.wsmem + (st.cnt & 1) * 4096;
       if (c.lane == 0) bulk_wait_read<1>();
@@ -634,6 +704,13 @@ struct EpiRowScale {
     if (lane == 0) bulk_wait_all<0>();
     __syncwarp();
   }
+};
+
+// The second GEMM of the FP8 block: e4m3 A (hg8) and B (W2 stored [N2, K]),
+// out = r * sa * sb * acc in bf16, with the light reduction folded in as in
+// the bf16 block.
+struct EpiRowScaleF8 : EpiRowScale {
+  static constexpr bool kFp8 = true;
 };
 
 // ---------------------------------------------------------------------------

@@ -283,6 +283,93 @@ __global__ void ce_label_dh_fix_kernel(const int2* __restrict__ entries, const i
   }
 }
 
+// ------------------------------------------------------------- FP8 (e4m3)
+// Per-tensor scaling for the FP8 block: s = amax / 448 (1 for an all-zero
+// tensor) and codes = e4m3(t * (1 / s)), rounded to nearest even and
+// saturated to +-448 (the KuCoin news flash "CODA: new research optimizes
+// transformer training with GEMM epilogue programming" names FP8 in section
+// "The lazy cost of training large models" only as the reason the non-GEMM
+// share grows; the scaling scheme is this library's).
+
+__device__ __forceinline__ float e4m3_scale(float amax) { return amax > 0.f ? amax / 448.0f : 1.0f; }
+
+// amax |src| of n8 * 8 bf16 values, as fp32 bits by atomic max (non-negative
+// floats order like their bits); *amax must be zero before the launch.
+__global__ void __launch_bounds__(256) amax_bf16_kernel(const __nv_bfloat16* __restrict__ src, size_t n8,
+                                                        unsigned* amax) {
+  __shared__ unsigned wm[8];
+  float m = 0.f;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const uint4 v = reinterpret_cast<const uint4*>(src)[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) m = fmaxf(m, fmaxf(fabsf(bf16lo(w[e])), fabsf(bf16hi(w[e]))));
+  }
+  const unsigned u = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = u;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const unsigned v = __reduce_max_sync(0xffffffffu, threadIdx.x < 8 ? wm[threadIdx.x] : 0u);
+    if (threadIdx.x == 0 && v != 0u) atomicMax(amax, v);
+  }
+}
+
+__global__ void fp8_scale_kernel(const float* amax, float* scale) { *scale = e4m3_scale(*amax); }
+
+// codes of n8 * 8 bf16 values, row-major as the source.
+__global__ void __launch_bounds__(256) quantize_e4m3_kernel(const __nv_bfloat16* __restrict__ src, size_t n8,
+                                                            const float* __restrict__ amax, uint8_t* __restrict__ dst) {
+  const float inv = 1.0f / e4m3_scale(*amax);
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const uint4 v = reinterpret_cast<const uint4*>(src)[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t q[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) q[e] = pack_e4m3x2(bf16lo(w[e]) * inv, bf16hi(w[e]) * inv);
+    reinterpret_cast<uint2*>(dst)[i] = make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
+  }
+}
+
+// Transposing form: src [rows, cols] -> dst [cols, rows] (a weight stored
+// K-major for the e4m3 mainloop), 64 x 64 tiles through shared memory.
+// Needs cols % 8 == 0 and rows % 4 == 0.
+constexpr int kQT = 64;
+__global__ void __launch_bounds__(256) quantize_e4m3_t_kernel(const __nv_bfloat16* __restrict__ src, int rows,
+                                                              int cols, const float* __restrict__ amax,
+                                                              uint8_t* __restrict__ dst) {
+  __shared__ uint8_t tile[kQT][kQT + 4];
+  const float inv = 1.0f / e4m3_scale(*amax);
+  const int r0 = blockIdx.y * kQT;
+  const int c0 = blockIdx.x * kQT;
+  for (int i = threadIdx.x; i < kQT * kQT / 8; i += blockDim.x) {
+    const int rr = i >> 3;
+    const int cc = (i & 7) * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r0 + rr < rows && c0 + cc < cols)
+      v = *reinterpret_cast<const uint4*>(src + static_cast<size_t>(r0 + rr) * cols + c0 + cc);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t q = pack_e4m3x2(bf16lo(w[e]) * inv, bf16hi(w[e]) * inv);
+      tile[rr][cc + 2 * e] = static_cast<uint8_t>(q & 0xffu);
+      tile[rr][cc + 2 * e + 1] = static_cast<uint8_t>(q >> 8);
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kQT * kQT / 4; i += blockDim.x) {
+    const int cc = i >> 4;
+    const int rr = (i & 15) * 4;
+    if (c0 + cc < cols && r0 + rr < rows) {
+      const uint32_t q = static_cast<uint32_t>(tile[rr][cc]) | (static_cast<uint32_t>(tile[rr + 1][cc]) << 8) |
+                         (static_cast<uint32_t>(tile[rr + 2][cc]) << 16) |
+                         (static_cast<uint32_t>(tile[rr + 3][cc]) << 24);
+      *reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(c0 + cc) * rows + r0 + rr) = q;
+    }
+  }
+}
+
 // ------------------------------------------------------ unfused comparison chain
 
 // out = a + b (bf16, 8 elements per thread).

@@ -294,6 +294,55 @@ coda_status_t coda_unfused_add(const uint16_t* a, const uint16_t* b, uint16_t* o
 coda_status_t coda_unfused_rmsnorm(const uint16_t* h, const uint16_t* gamma, float eps, uint16_t* y_out,
                                    float* r_out, int64_t M, int64_t N, void* stream);
 
+/* ------------------------------------------------------------ FP8 (e4m3)
+ *
+ * The block with FP8 GEMM operands.  The KuCoin news flash "CODA: new research
+ * optimizes transformer training with GEMM epilogue programming" names FP8 in
+ * section "The lazy cost of training large models" only as the reason the
+ * non-GEMM share of training time grows (faster matrix products, unchanged
+ * data movement); it gives no FP8 recipe.  This library's: OCP E4M3 codes
+ * (max 448, no infinities), round to nearest even with saturation, one fp32
+ * scale per tensor (t ~ s * decode(code)), both GEMM operands K-major, fp32
+ * accumulation, and the epilogue programs of the bf16 block.  Scales live in
+ * device memory so that no call synchronises with the host. */
+
+/* Quantises a bf16 tensor src [rows, cols] to e4m3 with its own per-tensor
+ * scale: amax_out = max |src|, scale_out = amax / 448 (1 if amax is 0), codes
+ * = e4m3(src * (1 / scale)).  transpose = 0: dst [rows, cols]; transpose = 1:
+ * dst [cols, rows] (a weight [K, N] stored K-major for the FP8 GEMMs).
+ * cols % 8 == 0; with transpose, rows % 4 == 0.  amax_out and scale_out are
+ * single device floats. */
+coda_status_t coda_fp8_quantize(const uint16_t* src, int64_t rows, int64_t cols, int transpose, uint8_t* dst,
+                                float* amax_out, float* scale_out, void* stream);
+
+/* scale_out = amax / 448 (1 if amax is 0): the next call's scale from this
+ * call's amax (delayed scaling of the block's hg8). */
+coda_status_t coda_fp8_scale_from_amax(const float* amax, float* scale_out, void* stream);
+
+/* First GEMM of the FP8 block: acc = x8 Wt8^T (e4m3 x e4m3 -> fp32), then in
+ * the epilogue h = acc * sx * sw + res, partial[t, i] = sum over 256-column
+ * tile t of h^2 (from the fp32 h), h_out = bf16(h),
+ * hg8_out = e4m3(gamma * h / s_hg), and amax_out = max |gamma * h| over the
+ * whole output (zeroed by this call, then raised by atomic max).
+ * x8 [M, K], Wt8 [N, K] (the weight transposed), hg8_out [M, N] e4m3;
+ * res [M, N] bf16 or NULL; gamma [N] bf16; h_out [M, N] bf16 or NULL;
+ * sx, sw, s_hg, amax_out single device floats; partial [T, M] fp32.
+ * N and K multiples of 16. */
+coda_status_t coda_gemm_res_partialrms_fp8(const uint8_t* x8, const float* sx, const uint8_t* Wt8, const float* sw,
+                                           const uint16_t* res, const uint16_t* gamma, const float* s_hg,
+                                           uint16_t* h_out, uint8_t* hg8_out, float* amax_out, float* partial,
+                                           int64_t M, int64_t N, int64_t K, void* stream);
+
+/* Second GEMM of the FP8 block, with the light reduction folded in as in
+ * coda_gemm_rowscale_partial: r_i = 1/sqrt(sum_t partial[t, i] / N_norm + eps),
+ * out = bf16(r_i * sa * sw * (A8 Wt8^T)_ij).  A8 [M, K] e4m3 (hg8 of the first
+ * GEMM), Wt8 [N, K] e4m3 (W2 transposed), sa, sw single device floats;
+ * r_out [M] or NULL; out [M, N] bf16.  K a multiple of 16. */
+coda_status_t coda_gemm_rowscale_partial_fp8(const uint8_t* A8, const float* sa, const uint8_t* Wt8, const float* sw,
+                                             const float* partial, int64_t T, int64_t N_norm, float eps,
+                                             float* r_out, uint16_t* out, int64_t M, int64_t N, int64_t K,
+                                             void* stream);
+
 /* ---------------------------------------------------------------- testing */
 
 /* Launches one block that waits on a barrier nothing ever signals, with time

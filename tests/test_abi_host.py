@@ -100,11 +100,30 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert lib.coda_unfused_rmsnorm(A, B, 1e-6, None, None, 16, 64, None) == NULL
     assert lib.coda_selftest_bounded_wait(0, A, None) == SHAPE
 
+    q = lib.coda_fp8_quantize
+    assert q(A, 16, 12, 0, B, C, D, None) == SHAPE        # cols not a multiple of 8
+    assert q(A, 6, 16, 1, B, C, D, None) == SHAPE         # transposed: rows not a multiple of 4
+    assert q(A, 16, 16, 0, None, C, D, None) == NULL
+    assert q(A, 16, 16, 0, MIS, C, D, None) == ALIGN
+    assert lib.coda_fp8_scale_from_amax(None, B, None) == NULL
+    p8 = lib.coda_gemm_res_partialrms_fp8
+    assert p8(A, B, C, D, None, A, B, None, C, D, A, 16, 64, 24, None) == SHAPE   # K not a multiple of 16
+    assert p8(A, B, C, D, None, A, B, None, C, D, A, 16, 72, 64, None) == SHAPE   # N not a multiple of 16
+    assert p8(A, B, C, D, None, None, B, None, C, D, A, 16, 64, 64, None) == NULL  # gamma
+    assert p8(A, B, C, D, None, A, B, None, MIS, D, A, 16, 64, 64, None) == ALIGN
+    assert p8(A, B, C, D, None, A, B, None, C, D, A, 0, 64, 64, None) == OK       # empty batch
+    r8 = lib.coda_gemm_rowscale_partial_fp8
+    assert r8(A, B, C, D, A, 1, 64, 1e-6, None, B, 16, 64, 40, None) == SHAPE     # K
+    assert r8(A, B, C, D, A, 0, 64, 1e-6, None, B, 16, 64, 64, None) == SHAPE     # T
+    assert r8(A, B, C, D, A, 1, 64, 1e-6, None, None, 16, 64, 64, None) == NULL   # out
+
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_valid_arguments_without_a_gpu_report_device_error(lib):
     assert lib.coda_gemm_rowscale(A, B, None, C, 256, 512, 512, None) == DEVICE
     assert lib.coda_rms_reduce(A, 16, 1, 64, 1e-6, B, None) == DEVICE
+    assert lib.coda_fp8_quantize(A, 16, 16, 1, B, C, D, None) == DEVICE
+    assert lib.coda_gemm_rowscale_partial_fp8(A, B, C, D, A, 1, 64, 1e-6, None, B, 16, 64, 64, None) == DEVICE
 
 
 def test_binding_refuses_cpu_tensors(lib):
