@@ -168,7 +168,8 @@ constexpr int64_t kCEBwdChunk = 4096;
 // of A and B) as fit next to the epilogue's shared memory, at most 8.
 template <class Epi>
 constexpr int pair_stages() {
-  constexpr int budget = 232448 - 1024 - 256 - kEpiWarps * Epi::kSmemPerWarp;
+  constexpr int budget = 232448 - 1024 - 256 - GemmSmem<256, 1, true, Epi>::kEpiBytes -
+                         GemmSmem<256, 1, true, Epi>::kXchgBytes;
   constexpr int st = budget / (2 * kBM * kBK * 2);
   return st > 8 ? 8 : st;
 }
@@ -198,6 +199,7 @@ coda_status_t run_gemm(int dev, DevInfo* info, GemmParams<Epi>& p, int M, int N,
   auto kern = coda_gemm_kernel<BN, STAGES, A_MN, B_MN, PAIR, Epi>;
   constexpr int smem = GemmSmem<BN, STAGES, PAIR, Epi>::kBytes;
   constexpr int kTileM = PAIR ? 2 * kBM : kBM;
+  constexpr int kThr = 64 + 32 * epi_warps<Epi>::value;  // producer + MMA warps, epilogue warps
   KernelCache& kc = g_kcache[dev][kind];
   {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -212,7 +214,7 @@ coda_status_t run_gemm(int dev, DevInfo* info, GemmParams<Epi>& p, int M, int N,
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
         cfg.gridDim = dim3(2 * (info->sms / 2), 1, 1);
-        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.blockDim = dim3(kThr, 1, 1);
         cfg.dynamicSmemBytes = smem;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
@@ -236,7 +238,7 @@ coda_status_t run_gemm(int dev, DevInfo* info, GemmParams<Epi>& p, int M, int N,
   p.wait_ns = static_cast<uint64_t>(g_wait_ns);
   if (!PAIR) {
     const int grid = p.sched.ntiles < info->sms ? p.sched.ntiles : info->sms;
-    kern<<<grid, kThreads, smem, stream>>>(p);
+    kern<<<grid, kThr, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
   }
   const int clusters = p.sched.ntiles < kc.max_clusters ? p.sched.ntiles : kc.max_clusters;
@@ -247,7 +249,7 @@ coda_status_t run_gemm(int dev, DevInfo* info, GemmParams<Epi>& p, int M, int N,
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(kThr, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;

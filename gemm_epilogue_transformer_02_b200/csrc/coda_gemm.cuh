@@ -66,6 +66,18 @@ struct epi_fp8<E, decltype(void(E::kFp8))> {
   static constexpr bool value = E::kFp8;
 };
 
+// Epilogue warps: 4 (one per TMEM lane quarter) unless the epilogue declares
+// kWarps = 8 (two per lane quarter, each taking half of the tile's columns,
+// for epilogues whose work outlasts the mainloop of a tile).
+template <class E, class = void>
+struct epi_warps {
+  static constexpr int value = kEpiWarps;
+};
+template <class E>
+struct epi_warps<E, decltype(void(E::kWarps))> {
+  static constexpr int value = E::kWarps;
+};
+
 template <class Epi>
 struct GemmParams {
   CUtensorMap tmA;
@@ -88,16 +100,30 @@ struct TileCtx {
   uint64_t* wbars;   // this warp's epilogue mbarriers
   bool has_next;     // this CTA has another tile after this one
   int nrow0, ncol0;  // first row of this warp / first column of that next tile
+  // Column range of the tile this warp handles: all of it, or (with eight
+  // epilogue warps) one half, the two halves of a lane quarter meeting in
+  // `xchg` (two parity slots of 32 floats) behind the mbarrier `xbar`.
+  int cbeg = 0, cend = 256;
+  bool split = false;
+  int half = 0;
+  int par = 0;       // tile parity: the xchg slot and the xbar phase of this tile
+  float* xchg = nullptr;
+  uint64_t* xbar = nullptr;
 };
 
 template <int BN, int STAGES, bool PAIR, class Epi>
 struct GemmSmem {
+  static constexpr int kEW = epi_warps<Epi>::value;
   static constexpr int kABytes = kBM * kBK * 2;                     // this CTA's 128 rows of A
   static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * kBK * 2;    // this CTA's columns of B
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kEpiBytes = kEpiWarps * Epi::kSmemPerWarp;
-  static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1 + kEpiWarps * Epi::kBarsPerWarp;
-  static constexpr int kBytes = 1024 /*align slack*/ + STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 16;
+  static constexpr int kEpiBytes = kEW * Epi::kSmemPerWarp;
+  static constexpr int kXchgBytes = kEW == 8 ? 4 * 2 * 32 * 4 : 0;  // per lane quarter: two slots of 32 floats
+  static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1 + kEW * Epi::kBarsPerWarp;
+  static constexpr int kBytes =
+      1024 /*align slack*/ + STAGES * kStageBytes + kEpiBytes + kXchgBytes + kNumBars * 8 + 16;
+  static_assert(kEW == 4 || kEW == 8, "four or eight epilogue warps");
+  static_assert(kEW == 4 || Epi::kBarsPerWarp >= 1, "eight epilogue warps pair up through an mbarrier");
   static_assert(Epi::kSmemPerWarp % 1024 == 0, "per-warp epilogue buffers keep the 128-byte swizzle alignment");
 };
 
@@ -116,8 +142,10 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
 // waits for both CTAs' copies on its full barriers (the copies of rank 1
 // complete there), and its commits arrive on the barriers of both CTAs.
 template <int BN, int STAGES, bool A_MN, bool B_MN, bool PAIR, class Epi>
-__global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_constant__ GemmParams<Epi> p) {
+__global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
+    coda_gemm_kernel(const __grid_constant__ GemmParams<Epi> p) {
   using S = GemmSmem<BN, STAGES, PAIR, Epi>;
+  constexpr int kEW = S::kEW;
   static_assert(BN % 64 == 0 && BN <= 256, "BN must be a multiple of 64, at most 256");
   static_assert(2 * BN == 512 || 2 * BN == 256 || 2 * BN == 128, "TMEM columns must be a power of two");
   static_assert(!PAIR || BN == 256, "pair tiles are 256 x 256");
@@ -131,14 +159,15 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * S::kABytes;
   uint8_t* sEpi = smem + STAGES * S::kStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + S::kEpiBytes);
+  float* sXchg = reinterpret_cast<float*>(sEpi + S::kEpiBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + S::kEpiBytes + S::kXchgBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* ebars = drain + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ebars + kEpiWarps * Epi::kBarsPerWarp);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ebars + kEW * Epi::kBarsPerWarp);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -154,10 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], PAIR ? 2 * kEpiWarps : kEpiWarps);
+      mbar_init(&tempty[a], PAIR ? 2 * kEW : kEW);
     }
     mbar_init(drain, 1);
-    for (int i = 0; i < kEpiWarps * Epi::kBarsPerWarp; ++i) mbar_init(&ebars[i], 1);
+    for (int i = 0; i < kEW * Epi::kBarsPerWarp; ++i) mbar_init(&ebars[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -334,6 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
     // --------------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int ew = warp - 2;
+    const int half = kEW == 8 ? ew >> 2 : 0;  // warps 2-5: first half of the columns, 6-9: second
     uint8_t* wsmem = sEpi + ew * Epi::kSmemPerWarp;
     uint64_t* wbars = ebars + ew * Epi::kBarsPerWarp;
     // accumulator release goes to rank 0's barriers (where the MMA waits)
@@ -367,6 +397,15 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_kernel(const __grid_con
         p.sched.map(t + tile_step, nmb, nnb);
         c.nrow0 = nmb * kTileM + static_cast<int>(rank) * kBM + q * 32;
         c.ncol0 = nnb * BN;
+      }
+      c.split = kEW == 8;
+      c.half = half;
+      c.cbeg = kEW == 8 ? half * (BN / 2) : 0;
+      c.cend = kEW == 8 ? (half + 1) * (BN / 2) : BN;
+      c.par = it & 1;
+      if (kEW == 8) {
+        c.xchg = sXchg + q * 64;                                        // the lane quarter's two slots
+        c.xbar = ebars + (half == 0 ? ew : ew - 4) * Epi::kBarsPerWarp;  // the first-half warp's barrier
       }
       const bool ok = Epi::template tile<BN>(p.ep, c, st, w);
       tc_fence_before();
@@ -420,10 +459,10 @@ __device__ __forceinline__ float acc_at(const uint32_t (&v0)[32], const uint32_t
 //     h = acc * sa * sb + res;  out1 = bf16(h);  partial += h^2;
 //     out2 = hg8 = e4m3(gamma * h / s_out) (round to nearest even, saturating);
 //     amax = max |gamma * h| (the next call's scale, by atomic max on its bits)
-// The input tile is read straight into registers (each thread its own row,
-// 128 bytes per 64-column chunk) one chunk ahead, and the first chunk of the
-// next tile is requested before this tile's last chunk is processed, so its
-// latency hides behind the epilogue math.  Outputs are staged in shared
+// The input tile is read straight into registers (each thread its own row)
+// 32 columns ahead, and the first columns of the next tile are requested
+// before this tile's last ones are processed, so their latency hides behind
+// the epilogue math.  Outputs are staged in shared
 // memory (128-byte swizzle) and written by TMA stores from one staging buffer
 // per warp (a second buffer would cost the mainloop its sixth pipeline stage,
 // which is worth more: 63.5 against 65.5 us on the 1B block's first GEMM).
@@ -437,7 +476,13 @@ struct EpiLoadStore2 {
   static constexpr int kOut2Bytes = MODE == 1 ? 8192 : 4096;
   static constexpr int kBufBytes = 4096 + kOut2Bytes;
   static constexpr int kSmemPerWarp = kNBuf * kBufBytes;
-  static constexpr int kBarsPerWarp = 0;
+  // Behind the e4m3 mainloop (twice the bf16 rate) the FP8 epilogue outlasts
+  // a tile's MMAs: eight warps, two per lane quarter, each taking half of the
+  // tile's columns (54 against 67 us on the 1B block's first GEMM).  The bf16
+  // modes keep four warps and with them a sixth pipeline stage (63.5 against
+  // 66.6 us with eight warps and five stages).
+  static constexpr int kWarps = MODE == 2 ? 8 : 4;
+  static constexpr int kBarsPerWarp = MODE == 2 ? 1 : 0;  // the halves' hand-over of the row sums
   static constexpr bool kPairedB = false;
 
   struct Params {
@@ -456,7 +501,7 @@ struct EpiLoadStore2 {
 
   struct State {
     uint32_t cnt;   // chunks processed by this warp (selects the staging buffer)
-    uint4 pre[8];   // prefetched input chunk (64 bf16 of this thread's row)
+    uint4 pre[4];   // prefetched input: 32 bf16 of this thread's row
     int pre_row, pre_col;  // which chunk `pre` holds (pre_col < 0: none)
   };
 
@@ -467,9 +512,9 @@ struct EpiLoadStore2 {
   }
 
   __device__ static __forceinline__ void load_chunk(const Params& ep, int M, int N, int row, int col,
-                                                    uint4 (&v)[8]) {
+                                                    uint4 (&v)[4]) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 4; ++j) {
       v[j] = make_uint4(0, 0, 0, 0);
       if (ep.in != nullptr && row < M && col + j * 8 < N)
         v[j] = __ldg(reinterpret_cast<const uint4*>(ep.in + static_cast<size_t>(row) * N + col + j * 8));
@@ -477,11 +522,12 @@ struct EpiLoadStore2 {
   }
 
   template <int BN>
-  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
-    const int col0 = c.nb * BN;
+  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx& w) {
+    const int col0 = c.nb * BN + c.cbeg;  // first column of this warp's share of the tile
     const int row = c.row0 + c.lane;
     int nch = (c.N - col0 + 63) / 64;
-    if (nch > BN / 64) nch = BN / 64;
+    if (nch > (c.cend - c.cbeg) / 64) nch = (c.cend - c.cbeg) / 64;
+    if (nch < 0) nch = 0;
     const bool rows_live = c.row0 < c.M;
     float rs = 1.f;
     if (MODE == 1) rs = (row < c.M) ? __ldg(ep.r + row) : 0.f;
@@ -492,25 +538,13 @@ struct EpiLoadStore2 {
     }
 
     if (st.pre_col != col0 || st.pre_row != row) load_chunk(ep, c.M, c.N, row, col0, st.pre);
-    float ss = 0.f;
+    // Row sums: each 64-column chunk from zero, the chunks of the tile's first
+    // and second halves added in order, then the halves: the same rounding
+    // whether one warp or two cover the tile.
+    float ss_lo = 0.f, ss_hi = 0.f;
     for (int ch = 0; ch < nch; ++ch) {
       const int cc = col0 + ch * 64;
-      uint4 cur[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) cur[j] = st.pre[j];
-      // request the next chunk (of this tile, or the first of the next tile)
-      if (ch + 1 < nch) {
-        load_chunk(ep, c.M, c.N, row, cc + 64, st.pre);
-        st.pre_row = row;
-        st.pre_col = cc + 64;
-      } else if (c.has_next) {
-        const int nrow = c.nrow0 + c.lane;
-        load_chunk(ep, c.M, c.N, nrow, c.ncol0, st.pre);
-        st.pre_row = nrow;
-        st.pre_col = c.ncol0;
-      } else {
-        st.pre_col = -1;
-      }
+      float ss = 0.f;
       const int b = kNBuf == 2 ? static_cast<int>(st.cnt & 1) : 0;
       uint8_t* R = c.wsmem + b * kBufBytes;
       uint8_t* G = R + 4096;
@@ -521,13 +555,35 @@ struct EpiLoadStore2 {
           bulk_wait_read<0>();
       }
       __syncwarp();
-      uint32_t v0[32], v1[32];
-      tmem_ld64(c.taddr + ch * 64, v0, v1);
       uint32_t q8lo = 0, q8hi = 0;  // MODE 2: codes of the even j, stored with the odd j
+      // the chunk's accumulator in two 32-column loads (fewer live registers)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int hh = 0; hh < 2; ++hh) {
+      uint4 cur[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) cur[u] = st.pre[u];
+      // request the next 32 input columns (of this tile, or the first of the next tile)
+      if (hh == 0 || ch + 1 < nch) {
+        const int nc = cc + (hh + 1) * 32;
+        load_chunk(ep, c.M, c.N, row, nc, st.pre);
+        st.pre_row = row;
+        st.pre_col = nc;
+      } else if (c.has_next) {
+        const int nrow = c.nrow0 + c.lane;
+        load_chunk(ep, c.M, c.N, nrow, c.ncol0 + c.cbeg, st.pre);
+        st.pre_row = nrow;
+        st.pre_col = c.ncol0 + c.cbeg;
+      } else {
+        st.pre_col = -1;
+      }
+      uint32_t v[32];
+      tmem_ld32(c.taddr + c.cbeg + ch * 64 + hh * 32, v);
+      tmem_ld_wait(v);
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int j = hh * 4 + jj;
         const uint32_t off = sw128_off(c.lane, j);
-        const uint32_t inw[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
+        const uint32_t inw[4] = {cur[jj].x, cur[jj].y, cur[jj].z, cur[jj].w};
         uint32_t o1[4];
         if (MODE == 2) {
           const uint4 g4 = cc + j * 8 < c.N ? __ldg(reinterpret_cast<const uint4*>(ep.gamma + cc + j * 8))
@@ -536,8 +592,8 @@ struct EpiLoadStore2 {
           uint32_t q[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float h0 = fmaf(acc_at(v0, v1, j * 8 + 2 * e), asc, bf16lo(inw[e]));
-            const float h1 = fmaf(acc_at(v0, v1, j * 8 + 2 * e + 1), asc, bf16hi(inw[e]));
+            const float h0 = fmaf(__uint_as_float(v[jj * 8 + 2 * e]), asc, bf16lo(inw[e]));
+            const float h1 = fmaf(__uint_as_float(v[jj * 8 + 2 * e + 1]), asc, bf16hi(inw[e]));
             ss = fmaf(h0, h0, ss);
             ss = fmaf(h1, h1, ss);
             o1[e] = pack_bf16x2(h0, h1);
@@ -562,8 +618,8 @@ struct EpiLoadStore2 {
           const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float h0 = acc_at(v0, v1, j * 8 + 2 * e) + bf16lo(inw[e]);
-            const float h1 = acc_at(v0, v1, j * 8 + 2 * e + 1) + bf16hi(inw[e]);
+            const float h0 = __uint_as_float(v[jj * 8 + 2 * e]) + bf16lo(inw[e]);
+            const float h1 = __uint_as_float(v[jj * 8 + 2 * e + 1]) + bf16hi(inw[e]);
             ss = fmaf(h0, h0, ss);
             ss = fmaf(h1, h1, ss);
             o1[e] = pack_bf16x2(h0, h1);
@@ -574,8 +630,8 @@ struct EpiLoadStore2 {
           float dg[8];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float p0 = acc_at(v0, v1, j * 8 + 2 * e);
-            const float p1 = acc_at(v0, v1, j * 8 + 2 * e + 1);
+            const float p0 = __uint_as_float(v[jj * 8 + 2 * e]);
+            const float p1 = __uint_as_float(v[jj * 8 + 2 * e + 1]);
             const float g0 = bf16lo(inw[e]);
             const float g1 = bf16hi(inw[e]);
             ss = fmaf(g0, p0, ss);
@@ -595,6 +651,7 @@ struct EpiLoadStore2 {
         }
         st_shared_v4(R + off, make_uint4(o1[0], o1[1], o1[2], o1[3]));
       }
+      }
       fence_async_smem();
       __syncwarp();
       if (c.lane == 0 && rows_live) {
@@ -611,8 +668,25 @@ struct EpiLoadStore2 {
       }
       if (c.lane == 0) bulk_commit();
       ++st.cnt;
+      if ((c.cbeg >> 6) + ch < (BN >> 7))
+        ss_lo += ss;
+      else
+        ss_hi += ss;
     }
-    if (ep.partial != nullptr && row < c.M) ep.partial[static_cast<size_t>(c.nb) * c.M + row] = ss;
+    float ssum = ss_lo + ss_hi;
+    if (c.split) {
+      // the second half hands its sum to the first half of the same lane quarter
+      if (c.half == 1) {
+        c.xchg[c.par * 32 + c.lane] = ss_hi;
+        __syncwarp();
+        if (c.lane == 0) mbar_arrive(c.xbar);
+      } else {
+        if (!__all_sync(0xffffffffu, mbar_wait(c.xbar, static_cast<uint32_t>(c.par), w))) return false;
+        ssum = ss_lo + c.xchg[c.par * 32 + c.lane];
+      }
+    }
+    if (ep.partial != nullptr && row < c.M && c.half == 0)
+      ep.partial[static_cast<size_t>(c.nb) * c.M + row] = ssum;
     if (MODE == 2) {
       const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(amx));  // |hg| >= 0: bits order as values
       if (c.lane == 0 && m != 0u) atomicMax(ep.amax, m);
