@@ -117,3 +117,20 @@ def rmsnorm_block_fp8(x8, sx, W1t8, sw1, res, gamma, s_hg, W2t8, sw2, eps: float
     out = r[:, None] * acc2 * (np.float64(s_hg) * np.float64(sw2))
     return {"h": h, "partial": partial, "r": r, "hg": hg, "hg8": hg8,
             "amax": float(np.abs(hg).max()) if hg.size else 0.0, "out": out}
+
+
+def rmsnorm_block_fp8_unfused(x8, sx, W1t8, sw1, res, gamma, s_y, W2t8, sw2, eps: float) -> dict:
+    """The FP8 block as separate operators, the comparison chain for the fused
+    FP8 block: t = (decode(x8) decode(W1t8)^T) sx sw1; h = t + res;
+    r = 1 / sqrt(mean(h^2) + eps); y = gamma * h * r; y8 = encode(y / s_y);
+    amax = max |y|; out = (decode(y8) decode(W2t8)^T) s_y sw2.  Here the
+    normalised y is quantised (its scale s_y the caller's, as for hg8)."""
+    t = e4m3_decode(x8) @ e4m3_decode(W1t8).T * (np.float64(sx) * np.float64(sw1))
+    h = t + np.asarray(res, dtype=np.float64)
+    N = h.shape[1]
+    r = 1.0 / np.sqrt((h * h).sum(axis=1) / N + eps)
+    y = np.asarray(gamma, dtype=np.float64)[None, :] * h * r[:, None]
+    y8 = e4m3_encode(y / np.float64(s_y))
+    out = e4m3_decode(y8) @ e4m3_decode(W2t8).T * (np.float64(s_y) * np.float64(sw2))
+    return {"t": t, "h": h, "r": r, "y": y, "y8": y8,
+            "amax": float(np.abs(y).max()) if y.size else 0.0, "out": out}

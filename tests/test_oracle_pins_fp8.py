@@ -128,3 +128,29 @@ def test_fp8_block_within_e4m3_bound_of_exact_block():
     bound = exact["r"][:, None] * (step @ np.abs(W2))
     assert np.all(np.abs(f["out"] - exact["out"]) <= bound * (1 + 1e-9))
     assert np.abs(f["out"] - exact["out"]).max() > 0  # the quantisation is really there
+
+
+def test_fp8_unfused_chain_brute_force_and_error_bound():
+    """The unfused FP8 chain: pure-Python brute force on a tiny ragged shape,
+    and with s_y = amax(y)/448 within e4m3's rounding of y of the exact block
+    evaluated on the dequantised GEMM operands."""
+    x8, sx, W1t8, sw1, res, gamma, W2t8, sw2 = _tiny_fp8_inputs(3, 5, 7, 4, 13)
+    s_y = 0.002
+    f = F8.rmsnorm_block_fp8_unfused(x8, sx, W1t8, sw1, res, gamma, s_y, W2t8, sw2, 1e-6)
+    d = F8.e4m3_table()
+    M, K, N, N2 = 3, 5, 7, 4
+    for i in range(M):
+        h = [sum(d[x8[i, k]] * d[W1t8[j, k]] for k in range(K)) * sx * sw1 + res[i, j] for j in range(N)]
+        r = 1.0 / math.sqrt(sum(v * v for v in h) / N + 1e-6)
+        y8 = [int(F8.e4m3_encode(np.array([gamma[j] * h[j] * r / s_y]))[0]) for j in range(N)]
+        assert list(f["y8"][i]) == y8
+        for j in range(N2):
+            want = sum(d[y8[k]] * d[W2t8[j, k]] for k in range(N)) * s_y * sw2
+            assert f["out"][i, j] == pytest.approx(want, rel=1e-12, abs=1e-12)
+    x8, sx, W1t8, sw1, res, gamma, W2t8, sw2 = _tiny_fp8_inputs(16, 32, 48, 24, 14)
+    W2 = F8.dequantize(W2t8, sw2).T
+    exact = O.rmsnorm_block_unfused(F8.dequantize(x8, sx), res, F8.dequantize(W1t8, sw1).T, W2, gamma, 1e-6)
+    s_y = float(F8.quant_scale(np.abs(exact["y"]).max()))
+    f = F8.rmsnorm_block_fp8_unfused(x8, sx, W1t8, sw1, res, gamma, s_y, W2t8, sw2, 1e-6)
+    step = np.maximum(np.abs(exact["y"]) * 2.0 ** -4, 2.0 ** -10 * s_y)
+    assert np.all(np.abs(f["out"] - exact["out"]) <= (step @ np.abs(W2)) * (1 + 1e-9))
