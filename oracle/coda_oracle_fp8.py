@@ -119,14 +119,22 @@ def rmsnorm_block_fp8(x8, sx, W1t8, sw1, res, gamma, s_hg, W2t8, sw2, eps: float
             "amax": float(np.abs(hg).max()) if hg.size else 0.0, "out": out}
 
 
+def round_bf16(v) -> np.ndarray:
+    """Round to the nearest bf16 value (8 significant bits), ties to even."""
+    v = np.asarray(v, dtype=np.float64)
+    m, e = np.frexp(v)               # v = m 2^e, 0.5 <= |m| < 1
+    return np.ldexp(np.round(m * 256.0), e - 8)  # numpy rounds halves to even
+
+
 def rmsnorm_block_fp8_unfused(x8, sx, W1t8, sw1, res, gamma, s_y, W2t8, sw2, eps: float) -> dict:
     """The FP8 block as separate operators, the comparison chain for the fused
-    FP8 block: t = (decode(x8) decode(W1t8)^T) sx sw1; h = t + res;
+    FP8 block, each intermediate stored in bf16 as the chain stores it:
+    t = bf16((decode(x8) decode(W1t8)^T) sx sw1); h = bf16(t + res);
     r = 1 / sqrt(mean(h^2) + eps); y = gamma * h * r; y8 = encode(y / s_y);
     amax = max |y|; out = (decode(y8) decode(W2t8)^T) s_y sw2.  Here the
     normalised y is quantised (its scale s_y the caller's, as for hg8)."""
-    t = e4m3_decode(x8) @ e4m3_decode(W1t8).T * (np.float64(sx) * np.float64(sw1))
-    h = t + np.asarray(res, dtype=np.float64)
+    t = round_bf16(e4m3_decode(x8) @ e4m3_decode(W1t8).T * (np.float64(sx) * np.float64(sw1)))
+    h = round_bf16(t + np.asarray(res, dtype=np.float64))
     N = h.shape[1]
     r = 1.0 / np.sqrt((h * h).sum(axis=1) / N + eps)
     y = np.asarray(gamma, dtype=np.float64)[None, :] * h * r[:, None]

@@ -130,6 +130,17 @@ def test_fp8_block_within_e4m3_bound_of_exact_block():
     assert np.abs(f["out"] - exact["out"]).max() > 0  # the quantisation is really there
 
 
+def test_round_bf16_matches_torch_and_ties():
+    g = torch.Generator().manual_seed(6)
+    v = torch.randn(50000, generator=g, dtype=torch.float32) * 37.0
+    want = v.to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(F8.round_bf16(v.double().numpy()), want)
+    # halfway cases: 1 + 2^-8 lies between 1 and 1 + 2^-7 (odd last bit): even -> 1;
+    # 1 + 3 * 2^-8 between 1 + 2^-7 (odd) and 1 + 2^-6 (even) -> 1 + 2^-6
+    np.testing.assert_array_equal(F8.round_bf16([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8)]),
+                                  [1.0, 1 + 2.0 ** -6, -1.0])
+
+
 def test_fp8_unfused_chain_brute_force_and_error_bound():
     """The unfused FP8 chain: pure-Python brute force on a tiny ragged shape,
     and with s_y = amax(y)/448 within e4m3's rounding of y of the exact block
@@ -139,8 +150,18 @@ def test_fp8_unfused_chain_brute_force_and_error_bound():
     f = F8.rmsnorm_block_fp8_unfused(x8, sx, W1t8, sw1, res, gamma, s_y, W2t8, sw2, 1e-6)
     d = F8.e4m3_table()
     M, K, N, N2 = 3, 5, 7, 4
+    def bf16(v):  # round to 8 significant bits, ties to even, written out for one value
+        if v == 0:
+            return 0.0
+        e = math.floor(math.log2(abs(v))) - 7
+        q = v / 2.0 ** e
+        fl = math.floor(q)
+        rq = fl + 1 if (q - fl > 0.5 or (q - fl == 0.5 and fl % 2 == 1)) else fl
+        return rq * 2.0 ** e
+
     for i in range(M):
-        h = [sum(d[x8[i, k]] * d[W1t8[j, k]] for k in range(K)) * sx * sw1 + res[i, j] for j in range(N)]
+        t = [bf16(sum(d[x8[i, k]] * d[W1t8[j, k]] for k in range(K)) * sx * sw1) for j in range(N)]
+        h = [bf16(t[j] + res[i, j]) for j in range(N)]
         r = 1.0 / math.sqrt(sum(v * v for v in h) / N + 1e-6)
         y8 = [int(F8.e4m3_encode(np.array([gamma[j] * h[j] * r / s_y]))[0]) for j in range(N)]
         assert list(f["y8"][i]) == y8
@@ -152,5 +173,10 @@ def test_fp8_unfused_chain_brute_force_and_error_bound():
     exact = O.rmsnorm_block_unfused(F8.dequantize(x8, sx), res, F8.dequantize(W1t8, sw1).T, W2, gamma, 1e-6)
     s_y = float(F8.quant_scale(np.abs(exact["y"]).max()))
     f = F8.rmsnorm_block_fp8_unfused(x8, sx, W1t8, sw1, res, gamma, s_y, W2t8, sw2, 1e-6)
-    step = np.maximum(np.abs(exact["y"]) * 2.0 ** -4, 2.0 ** -10 * s_y)
+    # e4m3's half step of y, and what the bf16 rounding of t and h (2^-8 each,
+    # relative) carries into y (r moves by far less and is covered by 1.1)
+    t_exact = F8.dequantize(x8, sx) @ F8.dequantize(W1t8, sw1).T
+    carried = 1.1 * np.abs(gamma)[None, :] * exact["r"][:, None] * 2.0 ** -8 * (
+        np.abs(t_exact) + np.abs(exact["h"]))
+    step = 2.0 ** -4 * (np.abs(exact["y"]) + carried) + 2.0 ** -10 * s_y + carried
     assert np.all(np.abs(f["out"] - exact["out"]) <= (step @ np.abs(W2)) * (1 + 1e-9))
