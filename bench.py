@@ -568,6 +568,13 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
            "partial": torch.empty(C.partial_cols(D), M_TOK, dtype=torch.float32, device=dev),
            "r": torch.empty(M_TOK, dtype=torch.float32, device=dev)}
 
+    s_y = torch.ones(1, dtype=torch.float32, device=dev)
+    bu8 = {"t": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
+           "h": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
+           "y8": torch.empty(M_TOK, D, dtype=torch.uint8, device=dev),
+           "amax": torch.empty(1, dtype=torch.float32, device=dev),
+           "r": torch.empty(M_TOK, dtype=torch.float32, device=dev)}
+
     def f8(evs=None):
         C.gemm_rmsnorm_gemm(x, res_d, W1, W2, gamma, EPS, out=out16, bufs=b16)
         if evs:
@@ -580,11 +587,17 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
             evs[2].record(stream)
         C.gemm_rowscale_partial_fp8(b8["hg8"], s_hg, W2t8, sw2, b8["partial"], D, EPS, out=out8, r_out=b8["r"])
         C.fp8_scale_from_amax(b8["amax"], scale_out=s_hg)
+        if evs:
+            evs[3].record(stream)
+            flush.zero_()
+            evs[4].record(stream)
+        C.unfused_block_fp8(x8, sx, W1t8, sw1, res_d, gamma, s_y, W2t8, sw2, EPS, out=out8, bufs=bu8)
+        C.fp8_scale_from_amax(bu8["amax"], scale_out=s_y)
 
     for _ in range(3):
         f8(None)
-    _, parts = timed(f8, steps, 0, inner_events=3)
-    k = [sum(p[i] for p in parts) / len(parts) for i in range(4)]
+    _, parts = timed(f8, steps, 0, inner_events=5)
+    k = [sum(p[i] for p in parts) / len(parts) for i in range(6)]
     f_blk = 2.0 * M_TOK * D * (D + N2)
     ms8 = k[2] + k[3]
     res["fp8_block"] = {"ms": round(ms8, 4), "tflops": round(f_blk / ms8 / 1e9, 1),
@@ -592,9 +605,10 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
                         "gemm_res_partialrms_fp8_ms": round(k[2], 4),
                         "gemm_rowscale_partial_fp8_ms": round(k[3], 4),
                         "gemm_rowscale_partial_fp8_tflops": round(2.0 * M_TOK * D * N2 / k[3] / 1e9, 1),
+                        "unfused_fp8_chain_ms": round(k[5], 4), "speedup_vs_unfused_fp8": round(k[5] / ms8, 4),
                         "bf16_block_ms_same_steps": round(k[0], 4), "speedup_vs_bf16_block": round(k[0] / ms8, 4),
-                        "scaling": "per-tensor e4m3; hg8 scale from the previous step's amax"}
-    del res_d, x8, W1t8, W2t8, b8, out8, out16, b16
+                        "scaling": "per-tensor e4m3; hg8 (y8) scale from the previous step's amax"}
+    del res_d, x8, W1t8, W2t8, b8, out8, out16, b16, bu8
 
     # QKV projection with RoPE in its epilogue (1B attention input: 32 q + 8 k + 8 v heads of 64)
     n_qkv, rope_cols = 48 * 64, 40 * 64

@@ -71,6 +71,8 @@ _SIGS = {
     "coda_fp8_scale_from_amax": (_ST, [_P, _P, _P]),
     "coda_gemm_res_partialrms_fp8": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "coda_gemm_rowscale_partial_fp8": (_ST, [_P, _P, _P, _P, _P, _I64, _I64, _F, _P, _P, _I64, _I64, _I64, _P]),
+    "coda_gemm_fp8": (_ST, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "coda_unfused_rmsnorm_fp8": (_ST, [_P, _P, _F, _P, _P, _P, _P, _I64, _I64, _P]),
 }
 
 _lib = None
@@ -551,6 +553,46 @@ def gemm_rmsnorm_gemm_fp8(x8, sx, W1t8, sw1, res, gamma, s_hg, W2t8, sw2, eps: f
                                                     partial_out=b.get("partial"))
     out, r = gemm_rowscale_partial_fp8(hg8, s_hg, W2t8, sw2, partial, N, eps, out=out, r_out=b.get("r"))
     return {"out": out, "h": h, "hg8": hg8, "amax": amax, "partial": partial, "r": r}
+
+
+def gemm_fp8(A8, sa, Wt8, sw, out=None):
+    """out = bf16(sa * sw * (A8 Wt8^T)) with e4m3 A8 [M, K] and Wt8 [N, K]."""
+    M, K = A8.shape
+    N = Wt8.shape[0]
+    _need(A8, U8, "A8")
+    _need(Wt8, U8, "Wt8", (N, K))
+    _need(sa, F32, "sa", (1,))
+    _need(sw, F32, "sw", (1,))
+    out = _empty((M, N), BF16, A8) if out is None else out
+    _call("coda_gemm_fp8", _ptr(A8), _ptr(sa), _ptr(Wt8), _ptr(sw), _ptr(out), M, N, K, _stream())
+    return out
+
+
+def unfused_rmsnorm_fp8(h, gamma, eps: float, s_y, y8_out=None, amax_out=None, r_out=None):
+    """y8 = e4m3(gamma * h * r / s_y), amax = max |y|; returns (y8, amax, r)."""
+    M, N = h.shape
+    _need(h, BF16, "h")
+    _need(gamma, BF16, "gamma", (N,))
+    _need(s_y, F32, "s_y", (1,))
+    y8_out = _empty((M, N), U8, h) if y8_out is None else y8_out
+    amax_out = _empty((1,), F32, h) if amax_out is None else amax_out
+    r_out = _empty((M,), F32, h) if r_out is None else r_out
+    _call("coda_unfused_rmsnorm_fp8", _ptr(h), _ptr(gamma), float(eps), _ptr(s_y), _ptr(y8_out), _ptr(amax_out),
+          _ptr(r_out), M, N, _stream())
+    return y8_out, amax_out, r_out
+
+
+def unfused_block_fp8(x8, sx, W1t8, sw1, res, gamma, s_y, W2t8, sw2, eps: float, out=None, bufs=None):
+    """The unfused FP8 chain: FP8 GEMM -> residual add -> RMSNorm with an e4m3
+    output -> FP8 GEMM, every intermediate in HBM.  Returns dict(out, t, h,
+    y8, amax, r)."""
+    b = bufs or {}
+    t = gemm_fp8(x8, sx, W1t8, sw1, out=b.get("t"))
+    h = unfused_add(t, res, out=b.get("h"))
+    y8, amax, r = unfused_rmsnorm_fp8(h, gamma, eps, s_y, y8_out=b.get("y8"), amax_out=b.get("amax"),
+                                      r_out=b.get("r"))
+    out = gemm_fp8(y8, s_y, W2t8, sw2, out=out)
+    return {"out": out, "t": t, "h": h, "y8": y8, "amax": amax, "r": r}
 
 
 def unfused_block(x, res, W1, W2, gamma, eps: float, out=None, bufs=None):

@@ -1070,6 +1070,51 @@ coda_status_t coda_gemm_rowscale_partial_fp8(const uint8_t* A8, const float* sa,
                                                                     static_cast<cudaStream_t>(stream));
 }
 
+coda_status_t coda_gemm_fp8(const uint8_t* A8, const float* sa, const uint8_t* Wt8, const float* sw, uint16_t* out,
+                            int64_t M, int64_t N, int64_t K, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(N) && fp8_dim_ok(K), CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(A8 && sa && Wt8 && sw && out, CODA_ERR_NULL);
+  CODA_CHECK(al16(A8) && al16(Wt8) && al16(out), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  using Epi = EpiRowScaleF8;
+  GemmParams<Epi> p{};
+  if (!(tmap2d_u8(&p.tmA, A8, K, M, K, 128, kBM) && tmap2d_u8(&p.tmB, Wt8, K, N, K, 128, 128) &&
+        map_out_bf16(&p.ep.tmOut, out, M, N, N)))
+    return CODA_ERR_INTERNAL;
+  p.ep.sa = sa;
+  p.ep.sb = sw;
+  const int n_nt = static_cast<int>((N + 255) / 256);
+  return run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M),
+                                                                    static_cast<int>(N), static_cast<int>(K), n_nt,
+                                                                    raster_group(M, N, K), kKindRowScaleF8,
+                                                                    static_cast<cudaStream_t>(stream));
+}
+
+coda_status_t coda_unfused_rmsnorm_fp8(const uint16_t* h, const uint16_t* gamma, float eps, const float* s_y,
+                                       uint8_t* y8_out, float* amax_out, float* r_out, int64_t M, int64_t N,
+                                       void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && fp8_dim_ok(N) && eps >= 0.f, CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(h && gamma && s_y && y8_out && amax_out, CODA_ERR_NULL);
+  CODA_CHECK(al16(h) && al16(gamma) && al16(y8_out) && al16(amax_out) && al16(r_out), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  coda_status_t st = current_device(&dev, &info);
+  if (st != CODA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(amax_out, 0, sizeof(float), s) != cudaSuccess) return CODA_ERR_LAUNCH;
+  rmsnorm_e4m3_kernel<<<static_cast<int>(M), kNormThreads, 0, s>>>(
+      reinterpret_cast<const __nv_bfloat16*>(h), reinterpret_cast<const __nv_bfloat16*>(gamma), eps, s_y, y8_out,
+      r_out, reinterpret_cast<unsigned*>(amax_out), static_cast<int>(N));
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}
+
 }  // extern "C"
 
 // =========================================================================

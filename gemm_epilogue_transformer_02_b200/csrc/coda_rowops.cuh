@@ -427,6 +427,59 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const __nv_bfloat
   }
 }
 
+// The same with an e4m3 output for the unfused FP8 chain: y8 = e4m3(y / s_y)
+// (s_y a device float), amax = max |y| (fp32 bits by atomic max; zeroed by
+// the caller).  N % 8 == 0.
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_e4m3_kernel(
+    const __nv_bfloat16* __restrict__ h, const __nv_bfloat16* __restrict__ gamma, float eps,
+    const float* __restrict__ s_y, uint8_t* __restrict__ y8, float* __restrict__ r_out, unsigned* amax, int N) {
+  __shared__ float red[kNormThreads / 32];
+  __shared__ unsigned mx[kNormThreads / 32];
+  const size_t rowoff = static_cast<size_t>(blockIdx.x) * N;
+  float s = 0.f;
+  for (int c = threadIdx.x * 8; c < N; c += kNormThreads * 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(h + rowoff + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float a = bf16lo(w[e]), b = bf16hi(w[e]);
+      s = fmaf(a, a, fmaf(b, b, s));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int k = 0; k < kNormThreads / 32; ++k) tot += red[k];
+  const float rr = rsqrtf(tot / static_cast<float>(N) + eps);
+  if (threadIdx.x == 0 && r_out != nullptr) r_out[blockIdx.x] = rr;
+  const float inv = 1.0f / __ldg(s_y);
+  float m = 0.f;
+  for (int c = threadIdx.x * 8; c < N; c += kNormThreads * 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(h + rowoff + c);
+    const uint4 g = *reinterpret_cast<const uint4*>(gamma + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w}, gw[4] = {g.x, g.y, g.z, g.w};
+    uint32_t q[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float y0 = bf16lo(gw[e]) * bf16lo(w[e]) * rr;
+      const float y1 = bf16hi(gw[e]) * bf16hi(w[e]) * rr;
+      m = fmaxf(m, fmaxf(fabsf(y0), fabsf(y1)));
+      q[e] = pack_e4m3x2(y0 * inv, y1 * inv);
+    }
+    *reinterpret_cast<uint2*>(y8 + rowoff + c) = make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
+  }
+  const unsigned u = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+  if ((threadIdx.x & 31) == 0) mx[threadIdx.x >> 5] = u;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const unsigned t = __reduce_max_sync(0xffffffffu, threadIdx.x < kNormThreads / 32 ? mx[threadIdx.x] : 0u);
+    if (threadIdx.x == 0 && t != 0u) atomicMax(amax, t);
+  }
+}
+
 // ------------------------------------------------------------ bounded-wait self test
 
 // Waits on an mbarrier that nothing ever arrives on, with the given limit.

@@ -343,6 +343,19 @@ coda_status_t coda_gemm_rowscale_partial_fp8(const uint8_t* A8, const float* sa,
                                              float* r_out, uint16_t* out, int64_t M, int64_t N, int64_t K,
                                              void* stream);
 
+/* The unfused FP8 chain the fused FP8 block is measured against:
+ * coda_gemm_fp8 gives t = bf16(sa * sw * (A8 Wt8^T)) (A8 [M, K], Wt8 [N, K]
+ * e4m3; K a multiple of 16); after coda_unfused_add (h = t + res),
+ * coda_unfused_rmsnorm_fp8 writes y8 = e4m3(gamma * h * r / s_y) [M, N]
+ * (r = 1/sqrt(mean(h^2) + eps), r_out [M] or NULL), amax_out = max |y|
+ * (zeroed by the call), N a multiple of 16; then coda_gemm_fp8(y8, s_y, W2t8,
+ * ...) gives out. */
+coda_status_t coda_gemm_fp8(const uint8_t* A8, const float* sa, const uint8_t* Wt8, const float* sw, uint16_t* out,
+                            int64_t M, int64_t N, int64_t K, void* stream);
+coda_status_t coda_unfused_rmsnorm_fp8(const uint16_t* h, const uint16_t* gamma, float eps, const float* s_y,
+                                       uint8_t* y8_out, float* amax_out, float* r_out, int64_t M, int64_t N,
+                                       void* stream);
+
 /* ---------------------------------------------------------------- testing */
 
 /* Launches one block that waits on a barrier nothing ever signals, with time
