@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libcoda.so")
 
 SOURCES = ["coda.cu"]
-DEPS = ["coda.cu", "coda_device.cuh", "coda_gemm.cuh", "coda_rowops.cuh", "coda_block.cuh"]
+DEPS = ["coda.cu", "coda_device.cuh", "coda_gemm.cuh", "coda_rowops.cuh", "coda_block.cuh", "coda_grouped.cuh"]
 
 
 def nvcc_path() -> str:

@@ -218,7 +218,7 @@ size_t coda_lmhead_ce_bwd_workspace_size(int64_t M, int64_t V);
  * The vocabulary is processed in chunks of 4096 columns: a GEMM recomputes the
  * chunk's logits and its epilogue writes G_chunk (bf16, in the workspace;
  * the logits are never stored), then dH += G_chunk W_chunk^T and
- * dW_chunk = H^T G_chunk.  The label entry d_i (p - 1) dominates its dW
+ * dW_chunk = H^T G_chunk run as one grouped launch.  The label entry d_i (p - 1) dominates its dW
  * column, so the part of it that bf16 drops is kept in fp32 and added back in
  * the epilogues of the dH and dW GEMMs (rows bucketed by label beforehand;
  * each dW column sums its rows in increasing row order, so the result is
@@ -278,7 +278,9 @@ coda_status_t coda_rms_reduce_bwd_noalloc(const float* pdr, const float* r, cons
 
 /* Backward of h = x W1 + res: dx_out = bf16(dh W1^T) [M, K], dW1_out = x^T dh
  * (fp32) [K, N]; dres equals dh.  dh [M, N] bf16, x [M, K] bf16, W1 [K, N] bf16.
- * Either output may be NULL (not computed). */
+ * Either output may be NULL (not computed).  With both requested and M >= N
+ * the two GEMMs share one persistent launch (the dW1 tiles first, the dx
+ * tiles filling each CTA pair up to a common makespan); otherwise two. */
 coda_status_t coda_gemm_res_partialrms_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* W1,
                                            uint16_t* dx_out, float* dW1_out, int64_t M, int64_t N, int64_t K,
                                            void* stream);
