@@ -4,6 +4,8 @@
 // no device allocations of its own.
 #include <mutex>
 
+#include <cmath>
+
 #include "coda.h"
 #include "coda_device.cuh"
 #include "coda_block.cuh"
@@ -671,7 +673,8 @@ coda_status_t coda_gemm_qkv_rope(const uint16_t* x, const uint16_t* W_qkv, const
   p.ep.positions = positions;
   p.ep.head_dim = static_cast<int>(head_dim);
   p.ep.rope_cols = static_cast<int>(rope_cols);
-  p.ep.log2_theta = log2f(theta);
+  for (int i = 0; i < head_dim / 2; ++i)
+    p.ep.turn[i] = std::pow(static_cast<double>(theta), -2.0 * i / static_cast<double>(head_dim)) / (2.0 * M_PI);
   return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(
       dev, info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>((N + 255) / 256),
       raster_group(M, N, K), kKindRope, static_cast<cudaStream_t>(stream));

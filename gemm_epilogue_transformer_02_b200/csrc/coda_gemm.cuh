@@ -1212,16 +1212,17 @@ struct EpiCE {
 // i + head_dim/2 form a pair rotated by the angle pos * theta^(-2 i / head_dim):
 //   (a, b) -> (a cos - b sin, b cos + a sin);
 // heads at or beyond rope_cols (v) are stored unrotated.  One thread owns one
-// row, so both columns of every pair are in its registers, and the sines and
-// cosines of its row are computed once per 32 frequencies and reused for every
-// head of the tile.  The angle is taken in turns, pos * theta^(-2i/d) / (2 pi),
-// in fp64; only its fractional part goes to sincospif, so large positions
-// keep their accuracy without a range reduction.
+// row, so both columns of every pair are in its registers.  The angle is taken
+// in turns, pos * theta^(-2i/d) / (2 pi), in fp64 (the per-frequency factors
+// come precomputed in the kernel parameters); only its fractional part goes
+// to sincospif, so large positions keep their accuracy without a range
+// reduction.  With head_dim 64 the sines and cosines of the row's 32
+// frequencies are computed once per tile and reused for every head.  Each
+// head is staged on its own (one or two 64-column boxes) and stored at once,
+// so the staging takes 8 KB per warp and the mainloop keeps six stages.
 // ---------------------------------------------------------------------------
 struct EpiRope {
-  // one 256-column x 32-row bf16 staging tile (four 64-column boxes) + 1 KB of
-  // per-frequency turns; a multiple of 1024 keeps the 128-byte swizzle alignment
-  static constexpr int kSmemPerWarp = 16384 + 1024;
+  static constexpr int kSmemPerWarp = 8192;  // two 64-column x 32-row bf16 boxes
   static constexpr int kBarsPerWarp = 0;
   static constexpr bool kPairedB = false;
 
@@ -1230,49 +1231,44 @@ struct EpiRope {
     const int* positions;   // [M]
     int head_dim;           // 64 or 128
     int rope_cols;          // columns [0, rope_cols) are rotated; a multiple of head_dim
-    float log2_theta;
+    double turn[64];        // theta^(-2i/head_dim) / (2 pi), i < head_dim / 2
   };
   struct State {
-    bool freq_ready;
+    uint32_t cnt;  // heads staged so far (alternates the two boxes when head_dim is 64)
   };
-  __device__ static void init_state(State& s) { s.freq_ready = false; }
+  __device__ static void init_state(State& s) { s.cnt = 0; }
 
   template <int BN>
   __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
-    constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
     const int col0 = c.nb * BN;
     const int row = c.row0 + c.lane;
     const int dh = ep.head_dim;
     const int half = dh >> 1;
-    double* turn = reinterpret_cast<double*>(c.wsmem + 16384);
-    if (!st.freq_ready) {
-      for (int i = c.lane; i < half; i += 32)
-        turn[i] = exp2(-(2.0 * i / dh) * static_cast<double>(ep.log2_theta)) * kInvTwoPi;
-      __syncwarp();
-      st.freq_ready = true;
-    }
     const double pos = (row < c.M) ? static_cast<double>(ep.positions[row]) : 0.0;
     int ncols = c.N - col0;
     if (ncols > BN) ncols = BN;
     const int nheads = ncols / dh;
-    const bool any_rot = col0 < ep.rope_cols;
-    uint8_t* S = c.wsmem;
-    if (c.lane == 0) bulk_wait_read<0>();  // the previous tile's stores have read the staging
-    __syncwarp();
-    for (int s = 0; s < half / 32; ++s) {
-      float cs[32], sn[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        cs[e] = 1.f;
-        sn[e] = 0.f;
-        if (any_rot) {
-          const double t = pos * turn[s * 32 + e];
-          sincospif(static_cast<float>(2.0 * (t - rint(t))), &sn[e], &cs[e]);
-        }
+    float cs[32], sn[32];
+    for (int hd = 0; hd < nheads; ++hd) {
+      const int hc0 = hd * dh;  // head's first column within the tile
+      const bool rot = col0 + hc0 < ep.rope_cols;
+      // head_dim 64: one box per head, two in turn; 128: both boxes per head
+      uint8_t* S = c.wsmem + (dh == 64 ? (st.cnt & 1) * 4096 : 0);
+      if (c.lane == 0) {
+        if (dh == 64)
+          bulk_wait_read<1>();  // this box was last stored two heads ago
+        else
+          bulk_wait_read<0>();
       }
-      for (int hd = 0; hd < nheads; ++hd) {
-        const int hc0 = hd * dh;  // head's first column within the tile
-        const bool rot = col0 + hc0 < ep.rope_cols;
+      __syncwarp();
+      for (int s = 0; s < half / 32; ++s) {
+        if (rot && (dh != 64 || hd == 0 || col0 + (hd - 1) * dh >= ep.rope_cols)) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const double t = pos * ep.turn[s * 32 + e];
+            sincospif(static_cast<float>(2.0 * (t - rint(t))), &sn[e], &cs[e]);
+          }
+        }
         uint32_t va[32], vb[32];
         tmem_ld32(c.taddr + hc0 + s * 32, va);
         tmem_ld32(c.taddr + hc0 + half + s * 32, vb);
@@ -1295,21 +1291,22 @@ struct EpiRope {
             pa[e2] = pack_bf16x2(oa[0], oa[1]);
             pb[e2] = pack_bf16x2(ob[0], ob[1]);
           }
-          const int ca = hc0 + s * 32 + q * 8;
-          const int cb = hc0 + half + s * 32 + q * 8;
+          const int ca = s * 32 + q * 8;  // columns within the head
+          const int cb = half + s * 32 + q * 8;
           st_shared_v4(S + (ca >> 6) * 4096 + sw128_off(c.lane, (ca & 63) >> 3),
                        make_uint4(pa[0], pa[1], pa[2], pa[3]));
           st_shared_v4(S + (cb >> 6) * 4096 + sw128_off(c.lane, (cb & 63) >> 3),
                        make_uint4(pb[0], pb[1], pb[2], pb[3]));
         }
       }
-    }
-    fence_async_smem();
-    __syncwarp();
-    if (c.lane == 0) {
-      if (c.row0 < c.M)
-        for (int bx = 0; bx < (ncols + 63) / 64; ++bx) tma_store_2d(&ep.tmOut, S + bx * 4096, col0 + bx * 64, c.row0);
-      bulk_commit();
+      fence_async_smem();
+      __syncwarp();
+      if (c.lane == 0) {
+        if (c.row0 < c.M)
+          for (int bx = 0; bx < dh / 64; ++bx) tma_store_2d(&ep.tmOut, S + bx * 4096, col0 + hc0 + bx * 64, c.row0);
+        bulk_commit();
+      }
+      ++st.cnt;
     }
     return true;
   }
