@@ -72,6 +72,8 @@ _SIGS = {
     "coda_gemm_res_partialrms_fp8": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "coda_gemm_rowscale_partial_fp8": (_ST, [_P, _P, _P, _P, _P, _I64, _I64, _F, _P, _P, _I64, _I64, _I64, _P]),
     "coda_gemm_fp8": (_ST, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "coda_rmsnorm_block_host_workspace_size": (_SZ, [_I64, _I64, _I64, _I64]),
+    "coda_rmsnorm_block_host": (_ST, [_P, _P, _P, _P, _P, _F, _P, _P, _SZ, _I64, _I64, _I64, _I64, _I64, _P]),
     "coda_unfused_rmsnorm_fp8": (_ST, [_P, _P, _F, _P, _P, _P, _P, _I64, _I64, _P]),
 }
 
@@ -593,6 +595,45 @@ def unfused_block_fp8(x8, sx, W1t8, sw1, res, gamma, s_y, W2t8, sw2, eps: float,
                                       r_out=b.get("r"))
     out = gemm_fp8(y8, s_y, W2t8, sw2, out=out)
     return {"out": out, "t": t, "h": h, "y8": y8, "amax": amax, "r": r}
+
+
+def _need_host(t, dtype, name, shape=None):
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+def rmsnorm_block_host(x_host, res_host, W1, W2, gamma, eps: float, out_host=None, chunk_rows: int = 512,
+                       ws=None):
+    """The block with host-resident x, res and out (pin them for overlap);
+    weights on the device.  Rows stream through in chunks whose copies in
+    and out overlap the compute.  Returns out_host (complete once the
+    current stream is synchronised)."""
+    M, K = x_host.shape
+    N = W1.shape[1]
+    N2 = W2.shape[1]
+    _need_host(x_host, BF16, "x_host")
+    if res_host is not None:
+        _need_host(res_host, BF16, "res_host", (M, N))
+    _need(W1, BF16, "W1", (K, N))
+    _need(W2, BF16, "W2", (N, N2))
+    _need(gamma, BF16, "gamma", (N,))
+    if out_host is None:
+        out_host = torch.empty((M, N2), dtype=BF16, pin_memory=True)
+    _need_host(out_host, BF16, "out_host", (M, N2))
+    nb = int(load_library().coda_rmsnorm_block_host_workspace_size(K, N, N2, chunk_rows))
+    if ws is None:
+        ws = _empty((max(nb, 16),), torch.uint8, W1)
+    _call("coda_rmsnorm_block_host", x_host.data_ptr(), None if res_host is None else res_host.data_ptr(), _ptr(W1),
+          _ptr(W2), _ptr(gamma), float(eps), out_host.data_ptr(), _ptr(ws), ws.numel(), M, K, N, N2, chunk_rows,
+          _stream())
+    return out_host
 
 
 def unfused_block(x, res, W1, W2, gamma, eps: float, out=None, bufs=None):

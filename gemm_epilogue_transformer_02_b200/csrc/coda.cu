@@ -1225,6 +1225,153 @@ coda_status_t coda_unfused_rmsnorm_fp8(const uint16_t* h, const uint16_t* gamma,
   return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
 }
 
+// ------------------------------------------------- host-buffer block pipeline
+
+}  // extern "C"
+
+namespace {
+
+// Streams and events of the host-buffer pipeline, created once per device.
+struct HostPipe {
+  bool init = false;
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t start = nullptr;
+  cudaEvent_t in_done[2] = {}, comp_done[2] = {}, out_done[2] = {};
+};
+HostPipe g_pipe[64];
+
+coda_status_t host_pipe(int dev, HostPipe** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.init) {
+    bool ok = cudaStreamCreateWithFlags(&hp.s_in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.s_out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; ok && i < 2; ++i)
+      ok = cudaEventCreateWithFlags(&hp.in_done[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.comp_done[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.out_done[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      return CODA_ERR_LAUNCH;
+    }
+    hp.init = true;
+  }
+  *out = &hp;
+  return CODA_OK;
+}
+
+// Per-slot buffers of one chunk of chunk_rows rows.
+struct HostSlot {
+  uint16_t *x, *res, *h, *hg, *out;
+  float *partial, *r;
+};
+
+size_t host_slot_bytes(int64_t C, int64_t K, int64_t N, int64_t N2) {
+  const size_t T = static_cast<size_t>((N + 255) / 256);
+  return align256(static_cast<size_t>(C * K) * 2) + 3 * align256(static_cast<size_t>(C * N) * 2) +
+         align256(static_cast<size_t>(C * N2) * 2) + align256(T * static_cast<size_t>(C) * 4) +
+         align256(static_cast<size_t>(C) * 4);
+}
+
+HostSlot host_slot(void* base, int64_t C, int64_t K, int64_t N, int64_t N2) {
+  const size_t T = static_cast<size_t>((N + 255) / 256);
+  uint8_t* p = static_cast<uint8_t*>(base);
+  HostSlot sl;
+  sl.x = reinterpret_cast<uint16_t*>(p);
+  p += align256(static_cast<size_t>(C * K) * 2);
+  sl.res = reinterpret_cast<uint16_t*>(p);
+  p += align256(static_cast<size_t>(C * N) * 2);
+  sl.h = reinterpret_cast<uint16_t*>(p);
+  p += align256(static_cast<size_t>(C * N) * 2);
+  sl.hg = reinterpret_cast<uint16_t*>(p);
+  p += align256(static_cast<size_t>(C * N) * 2);
+  sl.out = reinterpret_cast<uint16_t*>(p);
+  p += align256(static_cast<size_t>(C * N2) * 2);
+  sl.partial = reinterpret_cast<float*>(p);
+  p += align256(T * static_cast<size_t>(C) * 4);
+  sl.r = reinterpret_cast<float*>(p);
+  return sl;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t coda_rmsnorm_block_host_workspace_size(int64_t K, int64_t N, int64_t N2, int64_t chunk_rows) {
+  if (chunk_rows <= 0 || K <= 0 || N <= 0 || N2 <= 0) return 0;
+  return 2 * host_slot_bytes(chunk_rows, K, N, N2);
+}
+
+coda_status_t coda_rmsnorm_block_host(const uint16_t* x_host, const uint16_t* res_host, const uint16_t* W1,
+                                      const uint16_t* W2, const uint16_t* gamma, float eps, uint16_t* out_host,
+                                      void* ws, size_t ws_bytes, int64_t M, int64_t K, int64_t N, int64_t N2,
+                                      int64_t chunk_rows, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && dim_ok(K) && dim_ok(N) && dim_ok(N2) && eps >= 0.f &&
+                 chunk_rows > 0 && chunk_rows % 256 == 0,
+             CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(x_host && W1 && W2 && gamma && out_host && ws, CODA_ERR_NULL);
+  CODA_CHECK(al16(W1) && al16(W2) && al16(gamma) && al16(ws), CODA_ERR_ALIGN);
+  CODA_CHECK(ws_bytes >= coda_rmsnorm_block_host_workspace_size(K, N, N2, chunk_rows), CODA_ERR_WORKSPACE);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  HostPipe* hp = nullptr;
+  {
+    const coda_status_t ps = host_pipe(dev, &hp);
+    if (ps != CODA_OK) return ps;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t slot_bytes = host_slot_bytes(chunk_rows, K, N, N2);
+  const HostSlot slot[2] = {host_slot(ws, chunk_rows, K, N, N2),
+                            host_slot(static_cast<uint8_t*>(ws) + slot_bytes, chunk_rows, K, N, N2)};
+  // nothing of this call runs before the caller's earlier work on `stream`
+  bool ok = cudaEventRecord(hp->start, s) == cudaSuccess && cudaStreamWaitEvent(hp->s_in, hp->start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(hp->s_out, hp->start, 0) == cudaSuccess;
+  const int64_t nchunks = (M + chunk_rows - 1) / chunk_rows;
+  for (int64_t i = 0; ok && i < nchunks; ++i) {
+    const int b = static_cast<int>(i & 1);
+    const HostSlot& sl = slot[b];
+    const int64_t r0 = i * chunk_rows;
+    const int64_t rows = M - r0 < chunk_rows ? M - r0 : chunk_rows;
+    // inputs of chunk i into slot b, once chunk i - 2 has finished computing from it
+    if (i >= 2) ok = ok && cudaStreamWaitEvent(hp->s_in, hp->comp_done[b], 0) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(sl.x, x_host + r0 * K, static_cast<size_t>(rows * K) * 2, cudaMemcpyHostToDevice,
+                               hp->s_in) == cudaSuccess;
+    if (res_host)
+      ok = ok && cudaMemcpyAsync(sl.res, res_host + r0 * N, static_cast<size_t>(rows * N) * 2,
+                                 cudaMemcpyHostToDevice, hp->s_in) == cudaSuccess;
+    ok = ok && cudaEventRecord(hp->in_done[b], hp->s_in) == cudaSuccess;
+    // the block on the caller's stream, once the inputs are in and the output
+    // slot has been copied out (chunk i - 2)
+    ok = ok && cudaStreamWaitEvent(s, hp->in_done[b], 0) == cudaSuccess;
+    if (i >= 2) ok = ok && cudaStreamWaitEvent(s, hp->out_done[b], 0) == cudaSuccess;
+    if (!ok) break;
+    coda_status_t st = coda_gemm_res_partialrms(sl.x, W1, res_host ? sl.res : nullptr, gamma, sl.h, sl.hg, sl.partial,
+                                                rows, N, K, s);
+    if (st != CODA_OK) return st;
+    st = coda_gemm_rowscale_partial(sl.hg, W2, sl.partial, (N + 255) / 256, N, eps, sl.r, sl.out, rows, N2, N, s);
+    if (st != CODA_OK) return st;
+    ok = cudaEventRecord(hp->comp_done[b], s) == cudaSuccess &&
+         cudaStreamWaitEvent(hp->s_out, hp->comp_done[b], 0) == cudaSuccess &&
+         cudaMemcpyAsync(out_host + r0 * N2, sl.out, static_cast<size_t>(rows * N2) * 2, cudaMemcpyDeviceToHost,
+                         hp->s_out) == cudaSuccess &&
+         cudaEventRecord(hp->out_done[b], hp->s_out) == cudaSuccess;
+  }
+  // the caller's stream waits for the last copies out (and so for everything)
+  ok = ok && cudaStreamWaitEvent(s, hp->out_done[(nchunks - 1) & 1], 0) == cudaSuccess;
+  if (nchunks >= 2) ok = ok && cudaStreamWaitEvent(s, hp->out_done[nchunks & 1], 0) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    return CODA_ERR_LAUNCH;
+  }
+  return CODA_OK;
+}
+
 }  // extern "C"
 
 // =========================================================================

@@ -296,6 +296,24 @@ coda_status_t coda_unfused_add(const uint16_t* a, const uint16_t* b, uint16_t* o
 coda_status_t coda_unfused_rmsnorm(const uint16_t* h, const uint16_t* gamma, float eps, uint16_t* y_out,
                                    float* r_out, int64_t M, int64_t N, void* stream);
 
+/* The block with host-resident activations: x [M, K] and res [M, N] (or
+ * NULL) are read from host memory and out [M, N2] written to host memory;
+ * W1, W2 and gamma are device pointers (resident weights).  The rows go
+ * through in chunks of chunk_rows (a multiple of 256): while chunk i runs the
+ * two GEMMs on `stream`, chunk i + 1 is copied in and chunk i - 1 copied out
+ * on two streams of the library's own, so the copies overlap each other and
+ * the compute.  Host buffers should be pinned (page-locked) for the copies
+ * to overlap.  h, hg, partial and r stay in the workspace (two chunk slots,
+ * coda_rmsnorm_block_host_workspace_size bytes).  On return the work is
+ * queued; out_host is complete once `stream` is synchronised.  Results are
+ * bitwise those of coda_gemm_res_partialrms + coda_gemm_rowscale_partial on
+ * the whole batch. */
+size_t coda_rmsnorm_block_host_workspace_size(int64_t K, int64_t N, int64_t N2, int64_t chunk_rows);
+coda_status_t coda_rmsnorm_block_host(const uint16_t* x_host, const uint16_t* res_host, const uint16_t* W1,
+                                      const uint16_t* W2, const uint16_t* gamma, float eps, uint16_t* out_host,
+                                      void* ws, size_t ws_bytes, int64_t M, int64_t K, int64_t N, int64_t N2,
+                                      int64_t chunk_rows, void* stream);
+
 /* ------------------------------------------------------------ FP8 (e4m3)
  *
  * The block with FP8 GEMM operands.  The KuCoin news flash "CODA: new research

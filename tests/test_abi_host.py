@@ -112,6 +112,10 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert p8(A, B, C, D, None, None, B, None, C, D, A, 16, 64, 64, None) == NULL  # gamma
     assert p8(A, B, C, D, None, A, B, None, MIS, D, A, 16, 64, 64, None) == ALIGN
     assert p8(A, B, C, D, None, A, B, None, C, D, A, 0, 64, 64, None) == OK       # empty batch
+    hb = lib.coda_rmsnorm_block_host
+    assert hb(A, None, B, C, D, 1e-6, A, B, 1 << 30, 256, 64, 64, 64, 100, None) == SHAPE   # chunk not 256-aligned
+    assert hb(None, None, B, C, D, 1e-6, A, B, 1 << 30, 256, 64, 64, 64, 256, None) == NULL
+    assert hb(A, None, B, C, D, 1e-6, A, B, 16, 256, 64, 64, 64, 256, None) == WS
     r8 = lib.coda_gemm_rowscale_partial_fp8
     assert r8(A, B, C, D, A, 1, 64, 1e-6, None, B, 16, 64, 40, None) == SHAPE     # K
     assert r8(A, B, C, D, A, 0, 64, 1e-6, None, B, 16, 64, 64, None) == SHAPE     # T
