@@ -393,7 +393,7 @@ def run_ours(args):
         e2e_val = DD.weak_scaling_value(FLOPS_BLOCK, e_steps, DD.max_over_ranks(sum(tot_e), dev) / 1e3, ws) / 1e12
     h2d = 2 * (x_h.numel() + res_h.numel())
     d2h = 2 * out_h.numel()
-    del x_h, res_h, out_h, x_d, res_d
+    del x_h, res_h, out_h, ws_host
 
     # ---- the other hot-path rows (same inputs where the path continues)
     path = {}
