@@ -87,6 +87,12 @@ struct GemmParams {
   int M, N, K;       // GEMM sizes; N counts accumulator columns of the output space
   TileSched sched;
   uint64_t wait_ns;
+  // Programmatic dependent launch: pdl_trigger lets the next kernel on the
+  // stream (launched with programmatic serialisation) start its prologue on
+  // SMs this grid has left; pdl_wait makes this grid wait, after its own
+  // prologue, until the previous grid has completed and its writes are
+  // visible (a hardware dependency, like stream order).
+  int pdl_trigger, pdl_wait;
 };
 
 // Per-warp context handed to the epilogue for one tile.
@@ -210,6 +216,8 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const WaitCtx w{abort_flag, p.wait_ns};
+  if (p.pdl_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (p.pdl_wait) asm volatile("griddepcontrol.wait;" ::: "memory");
   const int nkb = (p.K + kKb - 1) / kKb;
   const int ntiles = p.sched.ntiles;
 

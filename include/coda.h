@@ -121,7 +121,12 @@ coda_status_t coda_gemm_rowscale(const uint16_t* A, const uint16_t* W, const flo
  * coda_rms_reduce, so the same r), then out = bf16(r_i * (A W)_ij).  r_out
  * [M] fp32 (may be NULL) receives r for the backward.  One launch instead of
  * two for the block's second half.  partial [T, M] fp32, A [M, K], W [K, N],
- * out [M, N] bf16; N_norm is the hidden size the partials were taken over. */
+ * out [M, N] bf16; N_norm is the hidden size the partials were taken over.
+ * Launched with programmatic stream serialisation: its CTAs may run their
+ * prologue while the preceding kernel on the stream (coda_gemm_res_partialrms
+ * lets them) still finishes, but read nothing before that kernel has
+ * completed, so the stream order holds as for any launch.  The same holds
+ * for coda_gemm_rowscale_partial_fp8 after coda_gemm_res_partialrms_fp8. */
 coda_status_t coda_gemm_rowscale_partial(const uint16_t* A, const uint16_t* W, const float* partial, int64_t T,
                                          int64_t N_norm, float eps, float* r_out, uint16_t* out, int64_t M,
                                          int64_t N, int64_t K, void* stream);
