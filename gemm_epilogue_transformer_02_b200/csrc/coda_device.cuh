@@ -123,6 +123,16 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* s
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
+// 2^x with the PTX instruction ex2.approx.ftz.f32 (one special-function-unit
+// operation; relative error about 2^-22; results below 2^-126 flush to zero).
+// Used by the cross-entropy epilogues, whose exponentials are probabilities
+// and sums of them, where neither matters.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Wait until at most N committed bulk groups still read shared memory.
 template <int N>
 __device__ __forceinline__ void bulk_wait_read() {

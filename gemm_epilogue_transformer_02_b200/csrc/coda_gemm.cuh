@@ -1184,22 +1184,22 @@ struct EpiCE {
       tmem_ld_wait(v);
       float z[32];
       float cm = -INFINITY;
-      const long long d = lab - cc;  // label position inside this chunk, if any
+      const long long d = lab - cc;                                    // label position inside this chunk,
+      const int dl = (d >= 0 && d < 32) ? static_cast<int>(d) : -1;   // if any
+      const bool whole = cc + 32 <= V;                                 // no ragged columns in this chunk
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        z[e] = (cc + e < V) ? rs * __uint_as_float(v[e]) : -INFINITY;
+        z[e] = (whole || cc + e < V) ? rs * __uint_as_float(v[e]) : -INFINITY;
         cm = fmaxf(cm, z[e]);
-        if (d == e) {
-          zl = z[e];
-          got = true;
-        }
+        zl = (e == dl) ? z[e] : zl;
       }
+      got = got || dl >= 0;
       const float mn = fmaxf(m, cm);
       const float base = mn * kL2E;
       float sum = 0.f;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) sum += exp2f(fmaf(z[e], kL2E, -base));
-      s = s * exp2f((m - mn) * kL2E) + sum;
+      for (int e = 0; e < 32; ++e) sum += ex2_approx(fmaf(z[e], kL2E, -base));
+      s = s * ex2_approx((m - mn) * kL2E) + sum;
       m = mn;
     }
     if (valid) {
@@ -1368,6 +1368,9 @@ struct EpiCEGrad {
     const long long lab = live ? ep.labels[row] - ep.col_offset : -1;
     for (int ch = 0; ch < nch; ++ch) {
       const int cc = col0 + ch * 64;
+      const long long dd = lab - cc;                                    // label column inside this chunk,
+      const int ll = (dd >= 0 && dd < 64) ? static_cast<int>(dd) : -1;  // if any
+      float glab = 0.f;
       uint8_t* O = c.wsmem + (st.cnt & 1) * 4096;
       if (c.lane == 0) bulk_wait_read<1>();
       __syncwarp();
@@ -1383,18 +1386,20 @@ struct EpiCEGrad {
           for (int h = 0; h < 2; ++h) {
             const int jj = j * 8 + 2 * e + h;
             const float z = rs * acc_at(v0, v1, jj);
-            const float p = exp2f(fmaf(z, kL2E, -lse2));
-            const bool hit = lab == static_cast<long long>(cc + jj);
-            gg[h] = d * (p - (hit ? 1.0f : 0.0f));
-            if (hit && ep.resid != nullptr) {
-              // the label entry dominates its dW column: keep what bf16 rounding drops
-              ep.resid[row] = gg[h] - __bfloat162float(__float2bfloat16_rn(gg[h]));
+            const float p = ex2_approx(fmaf(z, kL2E, -lse2));
+            float g = d * p;
+            if (jj == ll) {
+              g = d * (p - 1.0f);
+              glab = g;
             }
+            gg[h] = g;
           }
           o[e] = pack_bf16x2(gg[0], gg[1]);
         }
         st_shared_v4(O + sw128_off(c.lane, j), make_uint4(o[0], o[1], o[2], o[3]));
       }
+      // the label entry dominates its dW column: keep what bf16 rounding drops
+      if (ll >= 0 && ep.resid != nullptr) ep.resid[row] = glab - __bfloat162float(__float2bfloat16_rn(glab));
       fence_async_smem();
       __syncwarp();
       if (c.lane == 0) {
