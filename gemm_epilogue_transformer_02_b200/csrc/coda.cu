@@ -202,7 +202,7 @@ static_assert(kKindCount <= 32, "kernel kinds fit the cache");
 
 template <int BN, int STAGES, bool A_MN, bool B_MN, bool PAIR, class Epi>
 coda_status_t run_gemm(int dev, DevInfo* info, GemmParams<Epi>& p, int M, int N, int K, int n_nt, int group_m,
-                       KernelKind kind, cudaStream_t stream, bool pdl_secondary = false) {
+                       KernelKind kind, cudaStream_t stream) {
   auto kern = coda_gemm_kernel<BN, STAGES, A_MN, B_MN, PAIR, Epi>;
   constexpr int smem = GemmSmem<BN, STAGES, PAIR, Epi>::kBytes;
   constexpr int kTileM = PAIR ? 2 * kBM : kBM;
@@ -261,16 +261,17 @@ coda_status_t run_gemm(int dev, DevInfo* info, GemmParams<Epi>& p, int M, int N,
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // Programmatic dependent launch: this grid may start (prologue only) while
+  // the previous kernel on the stream finishes, and waits for it in
+  // griddepcontrol.wait; it lets the next one start likewise.
   cudaLaunchAttribute attr2[2];
-  if (pdl_secondary) {
-    // may start while the previous kernel on the stream still runs; waits for it in griddepcontrol.wait
-    attr2[0] = attr[0];
-    attr2[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr2[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr2;
-    cfg.numAttrs = 2;
-    p.pdl_wait = 1;
-  }
+  attr2[0] = attr[0];
+  attr2[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr2[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr2;
+  cfg.numAttrs = 2;
+  p.pdl_wait = 1;
+  p.pdl_trigger = 1;
   if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return CODA_ERR_LAUNCH;
   return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
 }
@@ -363,8 +364,12 @@ coda_status_t run_grouped(int dev, DevInfo* info, GroupedParams<E0, E1>& p, cons
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cudaLaunchAttribute attr2[2];  // programmatic dependent launch, as in run_gemm
+  attr2[0] = attr[0];
+  attr2[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr2[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr2;
+  cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return CODA_ERR_LAUNCH;
   return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
 }
@@ -453,7 +458,6 @@ coda_status_t coda_gemm_res_partialrms(const uint16_t* x, const uint16_t* W, con
   p.ep.partial = partial;
   p.ep.has_out1 = h_out != nullptr;
   p.ep.has_out2 = hg_out != nullptr;
-  p.pdl_trigger = 1;  // the second GEMM of the block may start its prologue on SMs this grid has left
   const int n_nt = static_cast<int>((N + 255) / 256);
   return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), n_nt,
       raster_group(M, N, K), kKindResPartial, static_cast<cudaStream_t>(stream));
@@ -630,7 +634,7 @@ coda_status_t coda_gemm_rowscale_partial(const uint16_t* A, const uint16_t* W, c
   p.ep.r_out = r_out;
   const int n_nt = static_cast<int>((N + 255) / 256);
   return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), n_nt,
-      raster_group(M, N, K), kKindRowScale, static_cast<cudaStream_t>(stream), /*pdl_secondary=*/true);
+      raster_group(M, N, K), kKindRowScale, static_cast<cudaStream_t>(stream));
 }
 
 coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const float* r, uint16_t* act_out,
@@ -1150,7 +1154,6 @@ coda_status_t coda_gemm_res_partialrms_fp8(const uint8_t* x8, const float* sx, c
   p.ep.sb = sw;
   p.ep.s_out = s_hg;
   p.ep.amax = reinterpret_cast<unsigned*>(amax_out);
-  p.pdl_trigger = 1;  // the block's second GEMM may start its prologue on SMs this grid has left
   const int n_nt = static_cast<int>((N + 255) / 256);
   return run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M),
                                                                     static_cast<int>(N), static_cast<int>(K), n_nt,
@@ -1189,8 +1192,7 @@ coda_status_t coda_gemm_rowscale_partial_fp8(const uint8_t* A8, const float* sa,
   return run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M),
                                                                     static_cast<int>(N), static_cast<int>(K), n_nt,
                                                                     raster_group(M, N, K), kKindRowScaleF8,
-                                                                    static_cast<cudaStream_t>(stream),
-                                                                    /*pdl_secondary=*/true);
+                                                                    static_cast<cudaStream_t>(stream));
 }
 
 coda_status_t coda_gemm_fp8(const uint8_t* A8, const float* sa, const uint8_t* Wt8, const float* sw, uint16_t* out,

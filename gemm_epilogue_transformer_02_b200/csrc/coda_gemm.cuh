@@ -87,10 +87,11 @@ struct GemmParams {
   int M, N, K;       // GEMM sizes; N counts accumulator columns of the output space
   TileSched sched;
   uint64_t wait_ns;
-  // Programmatic dependent launch: pdl_trigger lets the next kernel on the
-  // stream (launched with programmatic serialisation) start its prologue on
-  // SMs this grid has left; pdl_wait makes this grid wait, after its own
-  // prologue, until the previous grid has completed and its writes are
+  // Programmatic dependent launch (set for every CTA-pair launch):
+  // pdl_trigger lets the next kernel on the stream, if launched with
+  // programmatic serialisation, start its prologue on SMs this grid has left;
+  // pdl_wait makes this grid wait, after its own prologue and before any
+  // global read, until the previous grid has completed and its writes are
   // visible (a hardware dependency, like stream order).
   int pdl_trigger, pdl_wait;
 };

@@ -178,6 +178,10 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_grouped_kernel(const __
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const WaitCtx w{abort_flag, p.wait_ns};
+  // launched with programmatic serialisation: let the next kernel start its
+  // prologue, and wait for the previous one before reading anything
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
