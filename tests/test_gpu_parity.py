@@ -331,3 +331,21 @@ def test_swiglu_mlp_backward_chain():
     check("d_y", bw["d_y"], ref["d_y"])
     check("dW_gu", bw["dW_gu"], ref["dW_gu"])
     check("dW_down", bw["dW_down"], ref["dW_down"])
+
+
+def test_stream_order_holds_with_programmatic_launch():
+    """Every pair GEMM is launched with programmatic stream serialisation and
+    lets the next one start early; work placed between two GEMMs on the
+    stream must still be seen.  Scaling the partials by 4 between the two
+    GEMMs of the block halves r (eps = 0), so out must halve exactly."""
+    inp = synth.tiny_block()
+    x, res, W1, W2, g = (dev(t) for t in (inp.x, inp.res, inp.W1, inp.W2, inp.gamma))
+    h, hg, part = C.gemm_res_partialrms(x, W1, res, g)
+    out_ref, _ = C.gemm_rowscale_partial(hg, W2, part, 512, 0.0)
+    for _ in range(3):  # the same sequence with an ordinary stream op in between
+        h, hg, part = C.gemm_res_partialrms(x, W1, res, g)
+        part.mul_(4.0)
+        out, r = C.gemm_rowscale_partial(hg, W2, part, 512, 0.0)
+        torch.cuda.synchronize()
+        C.poll_status()
+        assert torch.equal(out.float() * 2, out_ref.float())
