@@ -18,23 +18,32 @@
  *     (running max and sum-exp of online normalisation).
  *
  * Conventions (all calls):
- *   - Every tensor pointer is a DEVICE pointer owned by the caller; the library
- *     never allocates, frees or keeps a pointer after the call returns.
- *     Scratch space is passed in by the caller, sized by the *_workspace_size
- *     queries.
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller (the one
+ *     exception, coda_rmsnorm_block_host, says which of its pointers are host
+ *     memory); the library never allocates device memory for a call, frees
+ *     or keeps a pointer after the call returns.  Scratch space is passed in
+ *     by the caller, sized by the *_workspace_size queries.  What the library
+ *     keeps for the life of the process: per device, the kernel attributes it
+ *     has set, the device status word, the static scratch array of
+ *     coda_rms_reduce_bwd_noalloc, and the two streams and six events of
+ *     coda_rmsnorm_block_host (created on its first call).
  *   - Tensors are dense row-major.  Weights are stored [in, out]; activations
  *     [tokens, features].  bf16 tensors are passed as uint16_t bit patterns
  *     (IEEE bfloat16); float tensors are fp32; labels are int64.
  *   - Every tensor base pointer must be 16-byte aligned.  M (tokens) may be any
  *     value >= 0 (M == 0 is a no-op); feature sizes N, K, F, V must be > 0 and
- *     multiples of 8 (the tensor-memory-access copies need 16-byte rows).
+ *     multiples of 8 (the tensor-memory-access copies need 16-byte rows), of
+ *     16 where an e4m3 (1-byte) tensor has that row length.
  *   - Outputs must not alias inputs unless a call says otherwise.
  *   - Each call enqueues its kernels on `stream` (a cudaStream_t; NULL = the
  *     legacy default stream) and returns without synchronising.  Calls are
- *     reentrant and keep no state between calls, except the device status
- *     word read by coda_poll_status().
- *   - Arithmetic: bf16 inputs, fp32 accumulation in tensor memory, fp32
- *     epilogue math, bf16 outputs rounded to nearest-even.
+ *     reentrant and keep no state between calls beyond what is listed above.
+ *     The GEMM kernels use programmatic dependent launch: one may start its
+ *     prologue while the previous GEMM on the stream finishes, but reads
+ *     nothing before that kernel has completed, so stream order holds as
+ *     for any launch.
+ *   - Arithmetic: bf16 inputs (e4m3 for the FP8 calls), fp32 accumulation in
+ *     tensor memory, fp32 epilogue math, bf16 outputs rounded to nearest-even.
  *   - Return value: CODA_OK, or an error.  Argument errors (NULL, SHAPE,
  *     ALIGN, WORKSPACE) are detected on the host before any CUDA call and
  *     nothing is launched.  CODA_ERR_DEVICE: the current device is not
