@@ -349,3 +349,39 @@ def test_stream_order_holds_with_programmatic_launch():
         torch.cuda.synchronize()
         C.poll_status()
         assert torch.equal(out.float() * 2, out_ref.float())
+
+
+def test_degenerate_rows_zero_hidden_state():
+    """Rows whose h is exactly zero (x and res zero) have no RMS: their partials
+    are 0, r = 1/sqrt(eps), and since hg is 0 their output row is exactly 0;
+    the other rows are unaffected.  With eps = 0 the same rows give r = inf
+    and a NaN output (0 * inf), as the definition does."""
+    inp = synth.tiny_block()
+    x, res = inp.x.clone(), inp.res.clone()
+    zero_rows = [0, 5, 255]
+    x[zero_rows] = 0
+    res[zero_rows] = 0
+    d = [dev(t) for t in (x, res, inp.W1, inp.W2, inp.gamma)]
+    f = C.gemm_rmsnorm_gemm(*d, inp.eps)
+    C.poll_status()
+    ref = O.rmsnorm_block_unfused(b(x), b(res), b(inp.W1), b(inp.W2), b(inp.gamma), inp.eps)
+    check("out", f["out"], ref["out"])
+    zr = torch.as_tensor(zero_rows, device="cuda")
+    assert torch.all(f["out"][zr] == 0)
+    assert torch.all(f["partial"][:, zr] == 0)
+    assert torch.allclose(f["r"][zr], torch.full((3,), 1.0 / math.sqrt(inp.eps), device="cuda"), rtol=1e-6)
+    g0 = C.gemm_rmsnorm_gemm(*d, 0.0)
+    C.poll_status()
+    assert torch.isinf(g0["r"][zr]).all() and torch.isnan(g0["out"][zr].float()).all()
+    keep = torch.as_tensor([i for i in range(256) if i not in zero_rows], device="cuda")
+    assert torch.isfinite(g0["out"][keep].float()).all()
+
+
+def test_fp8_quantize_all_zero_tensor():
+    """An all-zero tensor has amax 0, scale 1 and all-zero codes."""
+    t = torch.zeros(64, 32, dtype=torch.bfloat16, device="cuda")
+    for tr in (False, True):
+        codes, amax, scale = C.fp8_quantize(t, transpose=tr)
+        torch.cuda.synchronize()
+        assert float(amax.item()) == 0.0 and float(scale.item()) == 1.0
+        assert int(codes.count_nonzero().item()) == 0
