@@ -108,8 +108,10 @@ struct TileCtx {
   bool has_next;     // this CTA has another tile after this one
   int nrow0, ncol0;  // first row of this warp / first column of that next tile
   // Column range of the tile this warp handles: all of it, or (with eight
-  // epilogue warps) one half, the two halves of a lane quarter meeting in
-  // `xchg` (two parity slots of 32 floats) behind the mbarrier `xbar`.
+  // epilogue warps) one half.  Epilogues that sum over a row's columns
+  // (kBarsPerWarp >= 1) combine the two halves of a lane quarter in `xchg`
+  // (two parity slots of 32 floats) behind the mbarrier `xbar`; for the
+  // others both stay null.
   int cbeg = 0, cend = 256;
   bool split = false;
   int half = 0;
@@ -125,12 +127,12 @@ struct GemmSmem {
   static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * kBK * 2;    // this CTA's columns of B
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kEpiBytes = kEW * Epi::kSmemPerWarp;
-  static constexpr int kXchgBytes = kEW == 8 ? 4 * 2 * 32 * 4 : 0;  // per lane quarter: two slots of 32 floats
+  static constexpr bool kHandOver = kEW == 8 && Epi::kBarsPerWarp >= 1;  // halves combine a row sum
+  static constexpr int kXchgBytes = kHandOver ? 4 * 2 * 32 * 4 : 0;     // per lane quarter: two slots of 32 floats
   static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1 + kEW * Epi::kBarsPerWarp;
   static constexpr int kBytes =
       1024 /*align slack*/ + STAGES * kStageBytes + kEpiBytes + kXchgBytes + kNumBars * 8 + 16;
   static_assert(kEW == 4 || kEW == 8, "four or eight epilogue warps");
-  static_assert(kEW == 4 || Epi::kBarsPerWarp >= 1, "eight epilogue warps pair up through an mbarrier");
   static_assert(Epi::kSmemPerWarp % 1024 == 0, "per-warp epilogue buffers keep the 128-byte swizzle alignment");
 };
 
@@ -412,7 +414,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
       c.cbeg = kEW == 8 ? half * (BN / 2) : 0;
       c.cend = kEW == 8 ? (half + 1) * (BN / 2) : BN;
       c.par = it & 1;
-      if (kEW == 8) {
+      if (S::kHandOver) {
         c.xchg = sXchg + q * 64;                                        // the lane quarter's two slots
         c.xbar = ebars + (half == 0 ? ew : ew - 4) * Epi::kBarsPerWarp;  // the first-half warp's barrier
       }
@@ -1231,6 +1233,11 @@ struct EpiCE {
 // so the staging takes 8 KB per warp and the mainloop keeps six stages.
 // ---------------------------------------------------------------------------
 struct EpiRope {
+  // Eight warps, two per lane quarter, each taking half of the tile's columns
+  // (whole heads: 128 columns are two heads of 64 or one of 128).  With
+  // 128-wide heads this is 6 % faster than four warps; with 64-wide heads the
+  // two take the same time.
+  static constexpr int kWarps = 8;
   static constexpr int kSmemPerWarp = 8192;  // two 64-column x 32-row bf16 boxes
   static constexpr int kBarsPerWarp = 0;
   static constexpr bool kPairedB = false;
@@ -1249,17 +1256,17 @@ struct EpiRope {
 
   template <int BN>
   __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
-    const int col0 = c.nb * BN;
+    const int col0 = c.nb * BN + c.cbeg;  // first column of this warp's half of the tile
     const int row = c.row0 + c.lane;
     const int dh = ep.head_dim;
     const int half = dh >> 1;
     const double pos = (row < c.M) ? static_cast<double>(ep.positions[row]) : 0.0;
     int ncols = c.N - col0;
-    if (ncols > BN) ncols = BN;
+    if (ncols > c.cend - c.cbeg) ncols = c.cend - c.cbeg;
     const int nheads = ncols / dh;
     float cs[32], sn[32];
     for (int hd = 0; hd < nheads; ++hd) {
-      const int hc0 = hd * dh;  // head's first column within the tile
+      const int hc0 = hd * dh;  // head's first column within this warp's half
       const bool rot = col0 + hc0 < ep.rope_cols;
       // head_dim 64: one box per head, two in turn; 128: both boxes per head
       uint8_t* S = c.wsmem + (dh == 64 ? (st.cnt & 1) * 4096 : 0);
@@ -1279,8 +1286,8 @@ struct EpiRope {
           }
         }
         uint32_t va[32], vb[32];
-        tmem_ld32(c.taddr + hc0 + s * 32, va);
-        tmem_ld32(c.taddr + hc0 + half + s * 32, vb);
+        tmem_ld32(c.taddr + c.cbeg + hc0 + s * 32, va);
+        tmem_ld32(c.taddr + c.cbeg + hc0 + half + s * 32, vb);
         tmem_ld_wait(va);
         reg_pin(vb);
 #pragma unroll
