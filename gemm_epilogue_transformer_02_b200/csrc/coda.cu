@@ -711,10 +711,10 @@ coda_status_t coda_gemm_swiglu_bwd(const uint16_t* d_out, const uint16_t* W_down
   GemmParams<Epi> p{};
   // d_act = d_out W_down^T: W_down [F, N] read as [F rows of length N] (K-major), GEMM K = N.
   if (!(map_a(&p.tmA, d_out, false, M, N) && map_b(&p.tmB, W_down, false, F, N, N, 128) &&
+        map_out_bf16(&p.ep.tmG, gateup, M, F, 2 * F) && map_out_bf16(&p.ep.tmU, gateup + F, M, F, 2 * F) &&
         map_out_bf16(&p.ep.tmDG, d_gateup_out, M, F, 2 * F) &&
         map_out_bf16(&p.ep.tmDU, d_gateup_out + F, M, F, 2 * F)))
     return CODA_ERR_INTERNAL;
-  p.ep.gu = reinterpret_cast<const __nv_bfloat16*>(gateup);
   const int n_nt = static_cast<int>((F + 255) / 256);
   return run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(
       dev, info, p, static_cast<int>(M), static_cast<int>(F), static_cast<int>(N), n_nt, raster_group(M, F, N),

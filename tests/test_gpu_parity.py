@@ -300,7 +300,10 @@ def test_bounded_wait_gives_up_and_reports_timeout():
 
 # ------------------------------------------------------------ SwiGLU backward
 
-@pytest.mark.parametrize("M,N,F", [(300, 136, 200), (256, 512, 384)])
+# (2600, 72, 2000): 88 tiles on 74 CTA pairs, so some pairs run two and load
+# the second tile's first gate/up chunk during the first; ragged rows, a
+# ragged last 64-column chunk and a K shorter than one k-block pair
+@pytest.mark.parametrize("M,N,F", [(300, 136, 200), (256, 512, 384), (2600, 72, 2000)])
 def test_gemm_swiglu_bwd(M, N, F):
     g = gen(500 + F)
     d_out = synth.normal_bf16(g, (M, N))
