@@ -1247,7 +1247,11 @@ coda_status_t coda_unfused_rmsnorm_fp8(const uint16_t* h, const uint16_t* gamma,
 namespace {
 
 // Streams and events of the host-buffer pipeline, created once per device.
+// `mu` is held while a call enqueues its work: the events are re-recorded by
+// every call, and a wait must see the record of its own call, not one made
+// at the same time by another host thread on another stream.
 struct HostPipe {
+  std::mutex mu;
   bool init = false;
   cudaStream_t s_in = nullptr, s_out = nullptr;
   cudaEvent_t start = nullptr;
@@ -1340,6 +1344,7 @@ coda_status_t coda_rmsnorm_block_host(const uint16_t* x_host, const uint16_t* re
     const coda_status_t ps = host_pipe(dev, &hp);
     if (ps != CODA_OK) return ps;
   }
+  std::lock_guard<std::mutex> call_lock(hp->mu);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t slot_bytes = host_slot_bytes(chunk_rows, K, N, N2);
   const HostSlot slot[2] = {host_slot(ws, chunk_rows, K, N, N2),
@@ -1348,6 +1353,13 @@ coda_status_t coda_rmsnorm_block_host(const uint16_t* x_host, const uint16_t* re
   bool ok = cudaEventRecord(hp->start, s) == cudaSuccess && cudaStreamWaitEvent(hp->s_in, hp->start, 0) == cudaSuccess &&
             cudaStreamWaitEvent(hp->s_out, hp->start, 0) == cudaSuccess;
   const int64_t nchunks = (M + chunk_rows - 1) / chunk_rows;
+  coda_status_t st = CODA_OK;
+  // On an error part-way: the copies already queued on the library's streams
+  // still end before anything the caller queues on `stream` after this call.
+  auto drain = [&]() {
+    if (cudaEventRecord(hp->in_done[0], hp->s_in) == cudaSuccess) cudaStreamWaitEvent(s, hp->in_done[0], 0);
+    if (cudaEventRecord(hp->out_done[0], hp->s_out) == cudaSuccess) cudaStreamWaitEvent(s, hp->out_done[0], 0);
+  };
   for (int64_t i = 0; ok && i < nchunks; ++i) {
     const int b = static_cast<int>(i & 1);
     const HostSlot& sl = slot[b];
@@ -1366,11 +1378,14 @@ coda_status_t coda_rmsnorm_block_host(const uint16_t* x_host, const uint16_t* re
     ok = ok && cudaStreamWaitEvent(s, hp->in_done[b], 0) == cudaSuccess;
     if (i >= 2) ok = ok && cudaStreamWaitEvent(s, hp->out_done[b], 0) == cudaSuccess;
     if (!ok) break;
-    coda_status_t st = coda_gemm_res_partialrms(sl.x, W1, res_host ? sl.res : nullptr, gamma, sl.h, sl.hg, sl.partial,
-                                                rows, N, K, s);
-    if (st != CODA_OK) return st;
-    st = coda_gemm_rowscale_partial(sl.hg, W2, sl.partial, (N + 255) / 256, N, eps, sl.r, sl.out, rows, N2, N, s);
-    if (st != CODA_OK) return st;
+    st = coda_gemm_res_partialrms(sl.x, W1, res_host ? sl.res : nullptr, gamma, sl.h, sl.hg, sl.partial, rows, N, K,
+                                  s);
+    if (st == CODA_OK)
+      st = coda_gemm_rowscale_partial(sl.hg, W2, sl.partial, (N + 255) / 256, N, eps, sl.r, sl.out, rows, N2, N, s);
+    if (st != CODA_OK) {
+      drain();
+      return st;
+    }
     ok = cudaEventRecord(hp->comp_done[b], s) == cudaSuccess &&
          cudaStreamWaitEvent(hp->s_out, hp->comp_done[b], 0) == cudaSuccess &&
          cudaMemcpyAsync(out_host + r0 * N2, sl.out, static_cast<size_t>(rows * N2) * 2, cudaMemcpyDeviceToHost,
@@ -1382,6 +1397,7 @@ coda_status_t coda_rmsnorm_block_host(const uint16_t* x_host, const uint16_t* re
   if (nchunks >= 2) ok = ok && cudaStreamWaitEvent(s, hp->out_done[nchunks & 1], 0) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
+    drain();
     return CODA_ERR_LAUNCH;
   }
   return CODA_OK;

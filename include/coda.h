@@ -321,7 +321,10 @@ coda_status_t coda_unfused_rmsnorm(const uint16_t* h, const uint16_t* gamma, flo
  * coda_rmsnorm_block_host_workspace_size bytes).  On return the work is
  * queued; out_host is complete once `stream` is synchronised.  Results are
  * bitwise those of coda_gemm_res_partialrms + coda_gemm_rowscale_partial on
- * the whole batch. */
+ * the whole batch.  Calls made at the same time from several host threads
+ * on one device take turns while they enqueue (they share the library's two
+ * copy streams and their events); their GPU work still overlaps.  On an error
+ * part-way, `stream` still waits for the copies already queued. */
 size_t coda_rmsnorm_block_host_workspace_size(int64_t K, int64_t N, int64_t N2, int64_t chunk_rows);
 coda_status_t coda_rmsnorm_block_host(const uint16_t* x_host, const uint16_t* res_host, const uint16_t* W1,
                                       const uint16_t* W2, const uint16_t* gamma, float eps, uint16_t* out_host,

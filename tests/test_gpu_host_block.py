@@ -50,3 +50,43 @@ def test_host_block_rejects_device_tensors_and_bad_chunks():
         C.rmsnorm_block_host(inp.x.cuda(), None, W1, W2, gamma, inp.eps)
     with pytest.raises(C.CodaError):
         C.rmsnorm_block_host(inp.x.pin_memory(), None, W1, W2, gamma, inp.eps, chunk_rows=100)
+
+
+def test_host_block_concurrent_callers():
+    """Two host threads, each on its own stream and workspace, call the
+    host-buffer block at the same time: the library's shared copy streams
+    and events must keep every call's copies ordered after its own compute."""
+    import threading
+
+    shape = (1000, 264, 776, 392)
+    M, K, N, N2 = shape
+    ins = [synth.block_inputs(M, K, N, N2, seed=70 + t, w_std=0.04) for t in range(2)]
+    W1, W2, gamma = (t.cuda() for t in (ins[0].W1, ins[0].W2, ins[0].gamma))
+    refs = [C.gemm_rmsnorm_gemm(i.x.cuda(), i.res.cuda(), W1, W2, gamma, i.eps)["out"].cpu() for i in ins]
+    nb = int(C.load_library().coda_rmsnorm_block_host_workspace_size(K, N, N2, 256))
+    outs = [[], []]
+    errors = []
+
+    def worker(t):
+        try:
+            s = torch.cuda.Stream()
+            ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+            x_h, res_h = ins[t].x.pin_memory(), ins[t].res.pin_memory()
+            with torch.cuda.stream(s):
+                for _ in range(24):
+                    outs[t].append(C.rmsnorm_block_host(x_h, res_h, W1, W2, gamma, ins[t].eps, chunk_rows=256, ws=ws))
+            s.synchronize()
+        except Exception as e:  # reported on the main thread
+            errors.append(e)
+
+    th = [threading.Thread(target=worker, args=(t,)) for t in range(2)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join()
+    assert not errors, errors
+    C.poll_status()
+    for t in range(2):
+        assert len(outs[t]) == 24
+        for o in outs[t]:
+            assert torch.equal(o, refs[t])
