@@ -176,6 +176,22 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------- workload description
+
+DATA = "synthetic (seeded N(0,1) activations, N(0,0.02) weights, gamma = 1+0.1N(0,1))"
+
+
+def arm_config(l2, ws):
+    """The workload `config` of the JSON line; both arms report the same one."""
+    return {"workload": WORKLOAD, "tokens": M_TOK, "hidden": D, "n2": N2, "eps": EPS,
+            "l2": ("flushed (256 MB write) before every timed step; inputs also exceed L2"
+                   if l2 == "flush" else
+                   "no flush: the step's working set (x, res 64 MB, W1, W2 72 MB, h, hg 64 MB, out "
+                   "256 MB) is 3.6x the 126 MB L2, and each step's 256 MB output write evicts the "
+                   "next step's inputs"),
+            "parallelism": f"dp{ws} (independent batches, no collective on the data path)"}
+
+
 # --------------------------------------------------------------------- reference arm
 
 def cpu_threads():
@@ -243,8 +259,8 @@ def run_reference(args):
     line = {
         "impl": "reference", "metric": METRIC, "value": round(val, 5), "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample_rows_per_step": rows},
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
+        "config": arm_config(args.l2, ws),
         "cpu_baseline": {"value": round(val, 5), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                          "sample": f"{rows} token rows of the block per step (fp64 numpy oracle, unfused)"},
         "e2e": {"value": round(val, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -426,14 +442,8 @@ def run_ours(args):
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(total_s * 1e3 / args.steps, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, gamma = 1+0.1N(0,1))",
-            "config": {"workload": WORKLOAD, "tokens": M_TOK, "hidden": D, "n2": N2, "eps": EPS,
-                       "l2": ("flushed (256 MB write) before every timed step; inputs also exceed L2"
-                              if args.l2 == "flush" else
-                              "no flush: the step's working set (x, res 64 MB, W1, W2 72 MB, h, hg 64 MB, out "
-                              "256 MB) is 3.6x the 126 MB L2, and each step's 256 MB output write evicts the "
-                              "next step's inputs"),
-                       "parallelism": f"dp{ws} (independent batches, no collective on the data path)"},
+            "data": DATA,
+            "config": arm_config(args.l2, ws),
             "roofline": {"bound": "tensor", "kernel": "coda_gemm_rowscale_partial (GEMM2, 8192x2048x16384)",
                          "achieved": round(ach_g2, 1), "peak": burst, "unit": "TFLOP/s",
                          "frac": round(ach_g2 / burst, 4),
