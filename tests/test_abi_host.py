@@ -67,6 +67,12 @@ D = ctypes.c_void_p(0x40000)
 MIS = ctypes.c_void_p(0x30008)  # 8-byte aligned only
 
 
+# The pointers below are fake: these tests run only where no kernel can launch,
+# so that a validation that ever stopped rejecting them could not reach a GPU.
+no_gpu_only = pytest.mark.skipif(torch.cuda.is_available(), reason="fake pointers: CPU-only check")
+
+
+@no_gpu_only
 def test_argument_errors_are_reported_before_any_launch(lib):
     f = lib.coda_gemm_rowscale
     assert f(None, B, None, C, 256, 512, 512, None) == NULL
@@ -120,6 +126,59 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert r8(A, B, C, D, A, 1, 64, 1e-6, None, B, 16, 64, 40, None) == SHAPE     # K
     assert r8(A, B, C, D, A, 0, 64, 1e-6, None, B, 16, 64, 64, None) == SHAPE     # T
     assert r8(A, B, C, D, A, 1, 64, 1e-6, None, None, 16, 64, 64, None) == NULL   # out
+
+
+@no_gpu_only
+def test_argument_errors_of_the_remaining_calls(lib):
+    rp = lib.coda_gemm_rowscale_partial  # (A, W, partial, T, N_norm, eps, r_out, out, M, N, K, stream)
+    assert rp(A, B, C, 0, 64, 1e-6, None, D, 16, 64, 64, None) == SHAPE        # T
+    assert rp(A, B, C, 1, 0, 1e-6, None, D, 16, 64, 64, None) == SHAPE         # N_norm
+    assert rp(A, B, None, 1, 64, 1e-6, None, D, 16, 64, 64, None) == NULL      # partial
+    assert rp(A, B, C, 1, 64, 1e-6, MIS, D, 16, 64, 64, None) == ALIGN         # r_out
+    assert rp(A, B, C, 1, 64, 1e-6, None, D, 0, 64, 64, None) == OK            # empty batch
+
+    blk = lib.coda_rmsnorm_block  # (x, res, W1, W2, gamma, eps, h, hg, partial, r, out, ws, bytes, M, K, N, N2, s)
+    assert blk(A, None, B, C, D, -1.0, A, B, C, D, A, B, 1 << 20, 16, 64, 64, 64, None) == SHAPE
+    assert blk(A, None, B, C, D, 1e-6, None, B, C, D, A, B, 1 << 20, 16, 64, 64, 64, None) == NULL
+    assert blk(A, MIS, B, C, D, 1e-6, A, B, C, D, A, B, 1 << 20, 16, 64, 64, 64, None) == ALIGN
+    assert blk(A, None, B, C, D, 1e-6, A, B, C, D, A, B, 0, 16, 64, 64, 64, None) == WS
+
+    rope = lib.coda_gemm_qkv_rope  # (x, W, positions, out, M, N, K, head_dim, rope_cols, theta, stream)
+    assert rope(A, B, C, D, 16, 384, 64, 96, 192, 5e5, None) == SHAPE     # head_dim 64 or 128 only
+    assert rope(A, B, C, D, 16, 328, 64, 64, 192, 5e5, None) == SHAPE     # N not whole heads
+    assert rope(A, B, C, D, 16, 384, 64, 64, 100, 5e5, None) == SHAPE     # rope_cols not whole heads
+    assert rope(A, B, C, D, 16, 384, 64, 64, 448, 5e5, None) == SHAPE     # rope_cols > N
+    assert rope(A, B, C, D, 16, 384, 64, 64, 192, 1.0, None) == SHAPE     # theta
+    assert rope(A, B, None, D, 16, 384, 64, 64, 192, 5e5, None) == NULL   # positions
+    assert rope(A, B, C, MIS, 16, 384, 64, 64, 192, 5e5, None) == ALIGN
+    assert rope(A, B, C, D, 0, 384, 64, 64, 192, 5e5, None) == OK
+
+    sb = lib.coda_gemm_swiglu_bwd  # (d_out, W_down, gateup, d_gateup, M, F, N, stream)
+    assert sb(A, B, C, D, 16, 60, 64, None) == SHAPE                     # F not a multiple of 8
+    assert sb(A, B, None, D, 16, 64, 64, None) == NULL
+    assert sb(A, B, MIS, D, 16, 64, 64, None) == ALIGN
+    assert sb(A, B, C, D, 0, 64, 64, None) == OK
+
+    cb = lib.coda_lmhead_ce_bwd  # (H, W, labels, lse, d_loss, r, dH, dW, ws, bytes, M, V, K, stream)
+    assert cb(A, B, C, D, None, None, A, B, C, 1 << 30, 16, 60, 64, None) == SHAPE   # V
+    assert cb(A, B, C, None, None, None, A, B, C, 1 << 30, 16, 64, 64, None) == NULL  # lse
+    assert cb(A, B, C, D, MIS, None, A, B, C, 1 << 30, 16, 64, 64, None) == ALIGN     # d_loss
+    assert cb(A, B, C, D, None, None, A, B, C, 0, 16, 64, 64, None) == WS
+    assert lib.coda_lmhead_ce_bwd_workspace_size(8192, 128256) > 0
+
+    na = lib.coda_rms_reduce_bwd_noalloc  # (pdr, r, d_hg, h, gamma, dh, dgamma, M, T, N, stream)
+    assert na(A, B, C, D, A, B, C, 16, 0, 64, None) == SHAPE
+    assert na(A, B, C, D, None, B, C, 16, 1, 64, None) == NULL
+    assert na(A, B, C, D, A, B, C, 32768, 8, 2048, None) == WS   # ceil(M / 32) * N above the static 2^20 floats
+
+    g8 = lib.coda_gemm_fp8  # (A8, sa, Wt8, sw, out, M, N, K, stream)
+    assert g8(A, B, C, D, A, 16, 64, 24, None) == SHAPE   # K not a multiple of 16
+    assert g8(A, None, C, D, A, 16, 64, 64, None) == NULL  # sa
+    assert g8(A, B, C, D, MIS, 16, 64, 64, None) == ALIGN
+    u8 = lib.coda_unfused_rmsnorm_fp8  # (h, gamma, eps, s_y, y8, amax, r, M, N, stream)
+    assert u8(A, B, 1e-6, C, D, A, None, 16, 24, None) == SHAPE   # N not a multiple of 16
+    assert u8(A, B, 1e-6, None, D, A, None, 16, 64, None) == NULL  # s_y
+    assert u8(A, B, 1e-6, C, D, A, MIS, 16, 64, None) == ALIGN     # r_out
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
