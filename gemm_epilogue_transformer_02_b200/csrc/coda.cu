@@ -688,8 +688,12 @@ coda_status_t coda_gemm_qkv_rope(const uint16_t* x, const uint16_t* W_qkv, const
   p.ep.positions = positions;
   p.ep.head_dim = static_cast<int>(head_dim);
   p.ep.rope_cols = static_cast<int>(rope_cols);
+  // The angle of frequency i in turns, theta^(-2i/head_dim) / (2 pi) < 1, as a
+  // 64-bit fraction (ldexp by 64 stays below 2^64; the conversion drops less
+  // than 2^-64 turn, which a position below 2^31 grows to under 2^-33 turn).
   for (int i = 0; i < head_dim / 2; ++i)
-    p.ep.turn[i] = std::pow(static_cast<double>(theta), -2.0 * i / static_cast<double>(head_dim)) / (2.0 * M_PI);
+    p.ep.turn_fx[i] = static_cast<uint64_t>(
+        std::ldexp(std::pow(static_cast<double>(theta), -2.0 * i / static_cast<double>(head_dim)) / (2.0 * M_PI), 64));
   return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(
       dev, info, p, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>((N + 255) / 256),
       raster_group(M, N, K), kKindRope, static_cast<cudaStream_t>(stream));

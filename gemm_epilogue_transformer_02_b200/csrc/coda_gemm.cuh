@@ -1263,7 +1263,7 @@ struct EpiRope {
     const int* positions;   // [M]
     int head_dim;           // 64 or 128
     int rope_cols;          // columns [0, rope_cols) are rotated; a multiple of head_dim
-    double turn[64];        // theta^(-2i/head_dim) / (2 pi), i < head_dim / 2
+    uint64_t turn_fx[64];   // theta^(-2i/head_dim) / (2 pi), i < head_dim / 2, in units of 2^-64 turn
   };
   struct State {
     uint32_t cnt;  // heads staged so far (alternates the two boxes when head_dim is 64)
@@ -1276,7 +1276,9 @@ struct EpiRope {
     const int row = c.row0 + c.lane;
     const int dh = ep.head_dim;
     const int half = dh >> 1;
-    const double pos = (row < c.M) ? static_cast<double>(ep.positions[row]) : 0.0;
+    // the position as a 64-bit integer: pos x turn_fx mod 2^64 is the angle's
+    // fraction of a turn, exact (two's complement keeps negative positions right)
+    const uint64_t pos = (row < c.M) ? static_cast<uint64_t>(static_cast<int64_t>(ep.positions[row])) : 0u;
     int ncols = c.N - col0;
     if (ncols > c.cend - c.cbeg) ncols = c.cend - c.cbeg;
     const int nheads = ncols / dh;
@@ -1297,8 +1299,11 @@ struct EpiRope {
         if (rot && (dh != 64 || hd == 0 || col0 + (hd - 1) * dh >= ep.rope_cols)) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const double t = pos * ep.turn[s * 32 + e];
-            sincospif(static_cast<float>(2.0 * (t - rint(t))), &sn[e], &cs[e]);
+            // top 32 bits: the signed fraction of a turn in [-1/2, 1/2) x 2^32;
+            // times 2^-31 it is the angle over pi, in [-1, 1)
+            const uint64_t t = pos * ep.turn_fx[s * 32 + e];
+            const float a = static_cast<float>(static_cast<int32_t>(static_cast<uint32_t>(t >> 32))) * 0x1p-31f;
+            sincospif(a, &sn[e], &cs[e]);
           }
         }
         uint32_t va[32], vb[32];
