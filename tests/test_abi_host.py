@@ -198,3 +198,27 @@ def test_binding_refuses_cpu_tensors(lib):
 def test_build_flags_target_sm100a():
     src = open(os.path.join(os.path.dirname(binding.LIB_PATH), "build.py")).read()
     assert "arch=compute_100a,code=sm_100a" in src
+
+
+def test_product_never_touches_the_oracle():
+    """The library package neither imports nor reads anything under oracle/:
+    the oracle is test infrastructure, and there is no CPU fallback."""
+    pkg = os.path.dirname(binding.LIB_PATH)
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                # (the seeded input generator, shared with the tests, may name it in prose)
+                assert not re.search(r"(from|import)\s+oracle\b|[\'\"]oracle[/\'\"]|coda_oracle", text), \
+                    os.path.join(dirpath, f)
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """A missing libcoda.so is an error, never a silent fallback."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("binding_missing", binding.__file__)
+    m = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(m)
+    m.LIB_PATH = str(tmp_path / "libcoda.so")
+    with pytest.raises(RuntimeError, match="not found"):
+        m.load_library()
