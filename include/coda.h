@@ -182,8 +182,11 @@ coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const fl
  *   (a, b) -> (a cos - b sin, b cos + a sin);
  * columns from rope_cols on (v) are stored unrotated; out = bf16.
  * x [M, K] bf16, W_qkv [K, N] bf16 (q heads, then k heads, then v heads),
- * positions [M] int32, out [M, N] bf16; head_dim 64 or 128, N and rope_cols
- * multiples of head_dim, theta > 1 (LLaMA-3: 500000). */
+ * positions [M] int32 (any value, negative included), out [M, N] bf16;
+ * head_dim 64 or 128, N and rope_cols multiples of head_dim, theta > 1
+ * (LLaMA-3: 500000).  Each angle is reduced to a fraction of a turn exactly
+ * (the position times the frequency in 2^-64 turn, in 64-bit integers) before
+ * the fp32 sine and cosine, so long positions lose no accuracy. */
 coda_status_t coda_gemm_qkv_rope(const uint16_t* x, const uint16_t* W_qkv, const int32_t* positions, uint16_t* out,
                                  int64_t M, int64_t N, int64_t K, int64_t head_dim, int64_t rope_cols, float theta,
                                  void* stream);
