@@ -10,9 +10,10 @@ roofline, and its time against this library's own unfused
 GEMM -> add -> RMSNorm -> GEMM chain.  A step is one pass of the block
 (partial-RMS GEMM, light reduction, row-scaled GEMM) over one batch with the
 inputs resident in HBM; L2 is flushed (256 MB write) before every timed step.
-The other hot-path rows (SwiGLU + down projection, fused LM-head
-cross-entropy, the block backward) are timed in the same run and reported
-under "path".
+The other hot-path rows (SwiGLU + down projection and its backward, the FP8
+block beside the bf16 one, QKV + RoPE, the fused LM-head cross-entropy and its
+backward, the block backward) are timed in the same run and reported under
+"path"; ``--sweep`` adds the block at larger hidden sizes.
 
 Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no
 collective on the data path); time = max over ranks of the device time.
