@@ -28,8 +28,9 @@ def pytest_sessionfinish(session, exitstatus):
     if not _util.RESULTS:
         return
     import json
-    out = os.path.join(ROOT, "gpurun_out")
-    if os.path.isdir(out):
+    # opt-in: the directory named by CODA_PARITY_REPORT_DIR receives parity_errors.json
+    out = os.environ.get("CODA_PARITY_REPORT_DIR", "")
+    if out and os.path.isdir(out):
         path = os.path.join(out, "parity_errors.json")
         prev = {}
         if os.path.exists(path):
