@@ -63,3 +63,16 @@ def test_qkv_rope_leaves_v_columns():
     qkv = x @ W
     np.testing.assert_allclose(out[:, 16:], qkv[:, 16:], rtol=1e-14)
     np.testing.assert_allclose(out[:, :16], O.rope_rotate(qkv[:, :16], [0, 1, 2, 3], 8, 10000.0), rtol=1e-14)
+
+
+def test_rotations_compose_and_negative_positions_invert():
+    """Rotations by positions add: rotating by p1 then p2 equals rotating by
+    p1 + p2, and a negative position undoes the positive one (the kernel takes
+    any int32 position)."""
+    r = np.random.default_rng(35)
+    t = r.normal(size=(3, 256))
+    p1, p2 = [7, 2047, 123456], [5, -2047, 1_000_000]
+    both = O.rope_rotate(O.rope_rotate(t, p1, 128, 500000.0), p2, 128, 500000.0)
+    np.testing.assert_allclose(both, O.rope_rotate(t, np.add(p1, p2), 128, 500000.0), rtol=0, atol=1e-9)
+    back = O.rope_rotate(O.rope_rotate(t, p1, 64, 500000.0), np.negative(p1), 64, 500000.0)
+    np.testing.assert_allclose(back, t, rtol=0, atol=1e-9)
