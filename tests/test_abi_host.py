@@ -222,3 +222,18 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
     m.LIB_PATH = str(tmp_path / "libcoda.so")
     with pytest.raises(RuntimeError, match="not found"):
         m.load_library()
+
+
+@no_gpu_only
+def test_abi_from_plain_c(tmp_path):
+    """The header compiles as C99 and the library links and answers from C."""
+    src = os.path.join(os.path.dirname(__file__), "c", "abi_from_c.c")
+    inc = os.path.dirname(binding.HEADER_PATH)
+    libdir = os.path.dirname(binding.LIB_PATH)
+    exe = str(tmp_path / "abi_from_c")
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", inc, src, "-o", exe,
+                         "-L", libdir, "-l:libcoda.so", "-Wl,-rpath," + libdir], capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, run.stdout + run.stderr
+    assert "abi_from_c ok" in run.stdout
