@@ -76,4 +76,11 @@ def test_reference_arm_line_on_rank0():
     assert p.returncode == 0
     line = json.loads(p.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
-    assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["e2e"]["value"] == line["value"] == line["cpu_baseline"]["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    # the same metric and workload config as the GPU arm's line
+    sys.path.insert(0, ROOT)
+    import bench
+    assert line["metric"] == bench.METRIC and line["higher_is_better"] is True
+    assert line["config"] == bench.arm_config("flush", 1)
