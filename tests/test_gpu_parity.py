@@ -116,8 +116,8 @@ def test_tiny_block_matches_unfused_definition(fold):
     f = C.gemm_rmsnorm_gemm(dev(inp.x), dev(inp.res), dev(inp.W1), dev(inp.W2), dev(inp.gamma), inp.eps,
                             fold_reduce=fold)
     ref = O.rmsnorm_block_unfused(b(inp.x), b(inp.res), b(inp.W1), b(inp.W2), b(inp.gamma), inp.eps)
-    check("out", f["out"], ref["out"])
-    check("h", f["h"], ref["h"])
+    check("out", f["out"], ref["out"], strict=True)
+    check("h", f["h"], ref["h"], strict=True)
     check_rel("r", f["r"], ref["r"], 1e-3)
     # the unfused comparison chain rounds t, h and y to bf16 as well: a looser bar
     u = C.unfused_block(dev(inp.x), dev(inp.res), dev(inp.W1), dev(inp.W2), dev(inp.gamma), inp.eps)
