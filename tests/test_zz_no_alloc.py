@@ -4,9 +4,11 @@ coda_rms_reduce_bwd_noalloc serves callers that cannot allocate device memory
 at call time (a fixed device-memory budget after start-up, or a framework that
 owns all device memory and cannot hand out a workspace).  It keeps its scratch
 in a static device array inside the library instead of a caller workspace.
-These tests call both entry points through the C ABI on the same inputs, twice
-in a row with different sizes, and compare the outputs.  The file is named so
-that pytest collects it last; it also passes when run alone in a fresh process.
+These tests call both entry points through the C ABI on the same inputs, several
+times in a row with sizes that shrink and grow, and require identical outputs.
+(Sizes beyond the array are rejected before any launch; that is tested on the
+host, without a device.)  The file is named so that pytest collects it last;
+it also passes when run alone in a fresh process.
 """
 import ctypes
 
@@ -15,11 +17,8 @@ import torch
 
 from gemm_epilogue_transformer_02_b200 import binding as C
 from gemm_epilogue_transformer_02_b200 import synth
-from tests._util import check
 
 pytestmark = pytest.mark.gpu
-
-WORKSPACE_ERR = 4
 
 
 def _inputs(M, N, seed):
@@ -56,21 +55,16 @@ def _gpu():
     C.load_library()
 
 
-def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
-    for M, N, seed in ((300, 520, 1), (8192, 2048, 2)):
+def test_noalloc_matches_workspace_entry_point_on_calls_in_a_row():
+    """Large, small, large, small: each call leaves its partials in the shared
+    array, and a later call over a smaller or differently shaped problem must
+    not read any of them.  Both entry points run the same kernels on the same
+    inputs, so their outputs must be identical bit for bit."""
+    for M, N, seed in ((8192, 2048, 2), (300, 520, 1), (8192, 2048, 3), (1000, 776, 4)):
         args = _inputs(M, N, seed)
         dh_ref, dgamma_ref = C.rms_reduce_bwd(*args)      # caller-allocated workspace
         dh, dgamma = _noalloc(*args)                      # library's static scratch
         torch.cuda.synchronize()
-        check("noalloc dh", dh, dh_ref.double().cpu().numpy())
-        check("noalloc dgamma", dgamma, dgamma_ref.double().cpu().numpy())
+        assert torch.equal(dh, dh_ref), (M, N)
+        assert torch.equal(dgamma, dgamma_ref), (M, N)
     C.poll_status()
-
-
-def test_noalloc_rejects_sizes_beyond_its_scratch():
-    lib = C.load_library()
-    x = torch.zeros(16, dtype=torch.float32, device="cuda")
-    # ceil(32768 / 32) * 2048 = 2^21 floats > 2^20
-    st = lib.coda_rms_reduce_bwd_noalloc(_p(x), _p(x), _p(x), _p(x), _p(x), _p(x), _p(x), 32768, 8, 2048,
-                                         ctypes.c_void_p(0))
-    assert st == WORKSPACE_ERR
