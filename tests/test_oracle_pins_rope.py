@@ -7,13 +7,54 @@ section "Five kinds of building blocks" (RoPE as an elementwise transform).
 The rotate-half form with angle pos * theta^(-2i/d) is the plain reading.
 Pins: position 0 is the identity; every rotated pair keeps its norm; the
 q.k product of two rotated vectors depends only on the position difference;
-brute force with Python's math on a tiny case.
+brute force with Python's math on a tiny case.  Those hold for any choice of
+frequencies, so the frequencies themselves are pinned against values fixed by
+the published source of RoPE, RoFormer (Su et al., 2021, section 3.2.2: pair i
+of a d-wide head turns by pos * base^(-2(i-1)/d), i = 1..d/2), evaluated in
+40-digit decimal arithmetic in tests/golden/closed_forms.txt.
 """
 import math
+import os
 
 import numpy as np
+import pytest
 
 from oracle import coda_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "closed_forms.txt")
+
+
+def _golden():
+    out = {}
+    with open(GOLDEN) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            name, val = line.split()[:2]
+            out[name] = float(val)
+    return out
+
+
+# (base, head width d, 0-based pair index, position, golden key suffix)
+@pytest.mark.parametrize("base,d,i,pos,key", [(10000.0, 64, 16, 100, "b10000_d64_i16_p100"),
+                                              (500000.0, 128, 32, 707, "b500000_d128_i32_p707")])
+def test_frequencies_match_roformer(base, d, i, pos, key):
+    """A unit vector on the first column of pair i, and one on its partner,
+    turned by one position: the outputs are the cosine and sine of the
+    angle RoFormer's frequency gives.  A frequency exponent of -i/d instead of
+    -2i/d, a pair of (i, i+1) instead of (i, i + d/2), or a swapped sign of
+    the rotation fails here."""
+    g = _golden()
+    c, s = g["rope_cos_" + key], g["rope_sin_" + key]
+    t = np.zeros((2, 2 * d))
+    t[0, d + i] = 1.0          # second head, first column of pair i
+    t[1, d + i + d // 2] = 1.0  # second head, partner column
+    out = O.rope_rotate(t, [pos, pos], d, base)
+    np.testing.assert_allclose([out[0, d + i], out[0, d + i + d // 2]], [c, s], rtol=0, atol=1e-13)
+    np.testing.assert_allclose([out[1, d + i], out[1, d + i + d // 2]], [-s, c], rtol=0, atol=1e-13)
+    rest = np.ones(2 * d, dtype=bool)
+    rest[[d + i, d + i + d // 2]] = False
+    assert not np.any(out[:, rest])
 
 
 def test_position_zero_is_identity_and_pairs_keep_norm():
