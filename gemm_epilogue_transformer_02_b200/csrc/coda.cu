@@ -17,8 +17,8 @@ namespace {
 
 using namespace coda;
 
-constexpr int64_t kPartialTile = 256;  // BN of the tiles that emit partial sums
-constexpr int kVersion = 1;
+constexpr int64_t kPartialTile = 128;  // columns per partial sum: one half of a 256-column tile
+constexpr int kVersion = 2;  // 2: partial sums per 128-column slot
 
 int64_t g_wait_ns = 1000000000LL;
 
@@ -174,8 +174,7 @@ constexpr int64_t kCEBwdChunk = 4096;
 // of A and B) as fit next to the epilogue's shared memory, at most 8.
 template <class Epi>
 constexpr int pair_stages() {
-  constexpr int budget = 232448 - 1024 - 256 - GemmSmem<256, 1, true, Epi>::kEpiBytes -
-                         GemmSmem<256, 1, true, Epi>::kXchgBytes;
+  constexpr int budget = 232448 - 1024 - 256 - GemmSmem<256, 1, true, Epi>::kEpiBytes;
   constexpr int st = budget / (2 * kBM * kBK * 2);
   return st > 8 ? 8 : st;
 }
@@ -248,7 +247,18 @@ coda_status_t run_gemm(int dev, DevInfo* info, GemmParams<Epi>& p, int M, int N,
     kern<<<grid, kThr, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
   }
-  const int clusters = p.sched.ntiles < kc.max_clusters ? p.sched.ntiles : kc.max_clusters;
+  // A last partial wave of whole tiles that fills at most half of the CTA
+  // pairs runs as a wave of half tiles (128 columns) on twice as many pairs:
+  // e.g. 256 tiles on 74 pairs end in 34 tiles, 3.46 waves taking four
+  // tile-times; the 68 halves take about half of one.  (A grid of fewer
+  // tiles than pairs is one such wave: all of its tiles are halved.)
+  p.sched.nsplit = 0;
+  if (epi_split<Epi>::value && (B_MN || p.has_bh)) {
+    const int last = p.sched.ntiles % kc.max_clusters;
+    if (last > 0 && 2 * last <= kc.max_clusters) p.sched.nsplit = last;
+  }
+  const int units = p.sched.ntiles + p.sched.nsplit;
+  const int clusters = units < kc.max_clusters ? units : kc.max_clusters;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -570,7 +580,7 @@ coda_status_t coda_rmsnorm_block(const uint16_t* x, const uint16_t* res, const u
   p.ep1.has_out2 = 1;
   p.ep2.r = nullptr;
   p.ep2.partial = partial_out;
-  p.ep2.T = static_cast<int>((N + 255) / 256);
+  p.ep2.T = static_cast<int>(coda_partial_cols(N));
   p.ep2.inv_n = 1.0f / static_cast<float>(N);
   p.ep2.eps = eps;
   p.ep2.r_out = r_out;
@@ -588,7 +598,14 @@ coda_status_t coda_rmsnorm_block(const uint16_t* x, const uint16_t* res, const u
   p.wait_ns = static_cast<uint64_t>(g_wait_ns);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(ws, 0, static_cast<size_t>(p.n_mt) * 4, s) != cudaSuccess) return CODA_ERR_LAUNCH;
-  const int total = p.n1 + p.n2;
+  // as in run_gemm: a last partial wave on at most half of the pairs runs as
+  // half tiles (of the second GEMM, whose tiles come last)
+  p.nsplit = 0;
+  {
+    const int last = (p.n1 + p.n2) % kc.max_clusters;
+    if (last > 0 && 2 * last <= kc.max_clusters) p.nsplit = last < p.n2 ? last : p.n2;
+  }
+  const int total = p.n1 + p.n2 + p.nsplit;
   const int clusters = total < kc.max_clusters ? total : kc.max_clusters;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -881,6 +898,39 @@ coda_status_t coda_lmhead_ce_bwd(const uint16_t* H, const uint16_t* W, const int
   return CODA_OK;
 }
 
+coda_status_t coda_loss_stats(const float* loss, int64_t M, float* stats_out, void* stream) {
+  CODA_CHECK(M > 0 && M < (int64_t(1) << 24), CODA_ERR_SHAPE);  // the count is exact in fp32
+  CODA_CHECK(loss && stats_out, CODA_ERR_NULL);
+  CODA_CHECK(al16(loss) && al16(stats_out), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  loss_stats_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(loss, static_cast<int>(M), stats_out);
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}
+
+coda_status_t coda_ce_global_finish(const float* stats, int64_t M, float* mean_out, float* d_loss_out,
+                                    void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31), CODA_ERR_SHAPE);
+  CODA_CHECK(stats && (mean_out || d_loss_out), CODA_ERR_NULL);
+  CODA_CHECK(al16(stats) && al16(mean_out) && al16(d_loss_out), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  const int grid = d_loss_out != nullptr && M > 256 ? static_cast<int>((M + 255) / 256 < info->sms ? (M + 255) / 256
+                                                                                                    : info->sms)
+                                                      : 1;
+  ce_global_finish_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(stats, static_cast<int>(M), mean_out,
+                                                                               d_loss_out);
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}
+
 size_t coda_gemm_rowscale_bwd_workspace_size(int64_t M, int64_t N) {
   if (M < 0 || N <= 0) return 0;
   return align256(static_cast<size_t>(M) * N * 2);
@@ -909,9 +959,10 @@ coda_status_t coda_gemm_rowscale_bwd(const uint16_t* dOut, const uint16_t* hg, c
     using Epi = EpiLoadStore2<1>;
     GemmParams<Epi> p{};
     if (!(map_a(&p.tmA, dOut, false, M, N2) && map_b(&p.tmB, W2, false, N, N2, N2, 128) &&
-          map_out_bf16(&p.ep.tmOut1, y, M, N, N) &&
+          map_b(&p.tmBh, W2, false, N, N2, N2, 64) && map_out_bf16(&p.ep.tmOut1, y, M, N, N) &&
           map_out_f32(&p.ep.tmOut2, d_hg_out, M, N)))
       return CODA_ERR_INTERNAL;
+    p.has_bh = 1;
     p.ep.in = reinterpret_cast<const __nv_bfloat16*>(hg);
     p.ep.gamma = nullptr;
     p.ep.r = r;
@@ -962,7 +1013,7 @@ coda_status_t coda_rms_reduce_bwd(const float* pdr, const float* r, const float*
       reinterpret_cast<const __nv_bfloat16*>(gamma), reinterpret_cast<__nv_bfloat16*>(dh_out), part,
       static_cast<int>(M), static_cast<int>(T), static_cast<int>(N));
   if (cudaGetLastError() != cudaSuccess) return CODA_ERR_LAUNCH;
-  dgamma_final_kernel<<<static_cast<int>((N + 255) / 256), 256, 0, s>>>(part, nblk, static_cast<int>(N), dgamma_out);
+  dgamma_final_kernel<<<static_cast<int>((N + kDgCols - 1) / kDgCols), kDgCols * kDgGroups, 0, s>>>(part, nblk, static_cast<int>(N), dgamma_out);
   return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
 }
 
@@ -1002,8 +1053,9 @@ coda_status_t coda_gemm_res_partialrms_bwd(const uint16_t* dh, const uint16_t* x
     using Epi = EpiRowScale;
     GemmParams<Epi> p{};
     if (!(map_a(&p.tmA, dh, false, M, N) && map_b(&p.tmB, W1, false, K, N, N, 128) &&
-          map_out_bf16(&p.ep.tmOut, dx_out, M, K, K)))
+          map_b(&p.tmBh, W1, false, K, N, N, 64) && map_out_bf16(&p.ep.tmOut, dx_out, M, K, K)))
       return CODA_ERR_INTERNAL;
+    p.has_bh = 1;
     p.ep.r = nullptr;
     coda_status_t st = run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(K),
                                                            static_cast<int>(N), static_cast<int>((K + 255) / 256),
@@ -1291,14 +1343,14 @@ struct HostSlot {
 };
 
 size_t host_slot_bytes(int64_t C, int64_t K, int64_t N, int64_t N2) {
-  const size_t T = static_cast<size_t>((N + 255) / 256);
+  const size_t T = static_cast<size_t>(coda_partial_cols(N));
   return align256(static_cast<size_t>(C * K) * 2) + 3 * align256(static_cast<size_t>(C * N) * 2) +
          align256(static_cast<size_t>(C * N2) * 2) + align256(T * static_cast<size_t>(C) * 4) +
          align256(static_cast<size_t>(C) * 4);
 }
 
 HostSlot host_slot(void* base, int64_t C, int64_t K, int64_t N, int64_t N2) {
-  const size_t T = static_cast<size_t>((N + 255) / 256);
+  const size_t T = static_cast<size_t>(coda_partial_cols(N));
   uint8_t* p = static_cast<uint8_t*>(base);
   HostSlot sl;
   sl.x = reinterpret_cast<uint16_t*>(p);
@@ -1385,7 +1437,7 @@ coda_status_t coda_rmsnorm_block_host(const uint16_t* x_host, const uint16_t* re
     st = coda_gemm_res_partialrms(sl.x, W1, res_host ? sl.res : nullptr, gamma, sl.h, sl.hg, sl.partial, rows, N, K,
                                   s);
     if (st == CODA_OK)
-      st = coda_gemm_rowscale_partial(sl.hg, W2, sl.partial, (N + 255) / 256, N, eps, sl.r, sl.out, rows, N2, N, s);
+      st = coda_gemm_rowscale_partial(sl.hg, W2, sl.partial, coda_partial_cols(N), N, eps, sl.r, sl.out, rows, N2, N, s);
     if (st != CODA_OK) {
       drain();
       return st;
@@ -1484,7 +1536,7 @@ extern "C" coda_status_t coda_rms_reduce_bwd_noalloc(const float* pdr, const flo
       pdr, r, d_hg, reinterpret_cast<const __nv_bfloat16*>(h), reinterpret_cast<const __nv_bfloat16*>(gamma),
       reinterpret_cast<__nv_bfloat16*>(dh_out), part, static_cast<int>(M), static_cast<int>(T), static_cast<int>(N));
   if (cudaGetLastError() != cudaSuccess) return CODA_ERR_LAUNCH;
-  dgamma_final_kernel<<<static_cast<int>((N + 255) / 256), 256, 0, s>>>(part, static_cast<int>(nblk),
+  dgamma_final_kernel<<<static_cast<int>((N + kDgCols - 1) / kDgCols), kDgCols * kDgGroups, 0, s>>>(part, static_cast<int>(nblk),
                                                                         static_cast<int>(N), dgamma_out);
   return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
 }

@@ -38,22 +38,32 @@ struct BlockParams {
   int* ready;        // [n_mt] completion counters (zero at launch)
   int M, K1, N1, N2;
   int n_mt, n_nt1, n_nt2, n1, n2;
+  // the last nsplit second-GEMM tiles run as two 128-column halves each (a
+  // last partial wave on at most half of the pairs becomes a wave of halves)
+  int nsplit;
   int ready_target;  // counter value of a finished row block: n_nt1 tiles x 2 CTAs x 4 warps
   uint64_t wait_ns;
 };
 
 struct BlockTile {
   int phase, mb, nb;
+  int half;  // -1: a whole tile; 0 or 1: that 128-column half of a second-GEMM tile
 };
 
 __device__ __forceinline__ BlockTile block_tile(const BlockParams& p, int t) {
   BlockTile b;
+  b.half = -1;
   if (t < p.n1) {
     b.phase = 0;
     b.mb = t / p.n_nt1;
     b.nb = t - b.mb * p.n_nt1;
   } else {
-    const int u = t - p.n1;
+    int u = t - p.n1;
+    const int s0 = p.n2 - p.nsplit;
+    if (u >= s0) {
+      b.half = (u - s0) & 1;
+      u = s0 + ((u - s0) >> 1);
+    }
     b.phase = 1;
     b.nb = u / p.n_mt;
     b.mb = u - b.nb * p.n_mt;
@@ -100,7 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1) coda_block_kernel(const __grid_co
   const uint32_t rank = cluster_ctarank();
   const int tile_step = static_cast<int>(gridDim.x >> 1);
   const int tile_first = static_cast<int>(blockIdx.x >> 1);
-  const int ntiles = p.n1 + p.n2;
+  const int ntiles = p.n1 + p.n2 + p.nsplit;  // schedule units
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -153,7 +163,10 @@ __global__ void __launch_bounds__(kThreads, 1) coda_block_kernel(const __grid_co
           fence_proxy_async_global();
         }
         const int arow = bt.mb * kTileM + static_cast<int>(rank) * kBM;
-        const int bcol = bt.nb * BN + static_cast<int>(rank) * kBCols;
+        // a half tile: 64 B columns per CTA, starting at its half
+        const int bcol = bt.half < 0 ? bt.nb * BN + static_cast<int>(rank) * kBCols
+                                     : bt.nb * BN + bt.half * (BN / 2) + static_cast<int>(rank) * (kBCols / 2);
+        const int nbox = bt.half < 0 ? kBCols / 64 : kBCols / 128;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, w)) {
             ok = false;
@@ -161,11 +174,11 @@ __global__ void __launch_bounds__(kThreads, 1) coda_block_kernel(const __grid_co
           }
           uint8_t* a = sA + stage * S::kABytes;
           uint8_t* b = sB + stage * S::kBBytes;
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * S::kStageBytes);
+          if (rank == 0)
+            mbar_arrive_expect_tx(&full[stage], bt.half < 0 ? 2 * S::kStageBytes : 2 * (S::kABytes + S::kBBytes / 2));
           const uint32_t fb = full0 + stage * 8;
           tma_load_2d_pair(a, mA, fb, kb * kBK, arow);
-#pragma unroll
-          for (int j = 0; j < kBCols / 64; ++j)
+          for (int j = 0; j < nbox; ++j)
             tma_load_2d_pair(b + j * (64 * kBK * 2), mB, fb, bcol + j * 64, kb * kBK);
           ++issued;
           if (++stage == STAGES) {
@@ -189,17 +202,20 @@ __global__ void __launch_bounds__(kThreads, 1) coda_block_kernel(const __grid_co
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0 && rank == 0) {
       constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, BN, false, true);
+      constexpr uint32_t kIdescH = idesc_bf16_f32(kTileM, BN / 2, false, true);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
       for (int t = tile_first; ok && t < ntiles; t += tile_step, ++it) {
-        const int nkb = t < p.n1 ? nkb1 : nkb2;
+        const BlockTile bt = block_tile(p, t);
+        const int nkb = bt.phase == 0 ? nkb1 : nkb2;
+        const uint32_t idesc = bt.half < 0 ? kIdesc : kIdescH;
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         if (!mbar_wait(&tempty[acc], aph ^ 1u, w)) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + acc * BN;
+        const uint32_t d = tmem_base + acc * BN + (bt.half > 0 ? BN / 2 : 0);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, w)) {
             ok = false;
@@ -212,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1) coda_block_kernel(const __grid_co
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(b0 + kk * 16 * 128, 64 * kBK * 2, 1024);
-            tc_mma_bf16_pair(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            tc_mma_bf16_pair(d, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           tc_commit_pair_mc(&empty[stage], 0x3);
           if (++stage == STAGES) {
@@ -269,6 +285,10 @@ __global__ void __launch_bounds__(kThreads, 1) coda_block_kernel(const __grid_co
       } else {
         c.N = p.N2;
         c.has_next = false;
+        if (bt.half >= 0) {
+          c.cbeg = bt.half * (BN / 2);
+          c.cend = c.cbeg + BN / 2;
+        }
         if (!in_phase2) {
           // the staging buffers change owners: the first GEMM's stores must have read them
           if (lane == 0) bulk_wait_read<0>();

@@ -42,6 +42,25 @@ struct TileSched {
   int n_nt;     // N tiles
   int group_m;  // M tiles per raster group
   int ntiles;
+  // The last `nsplit` tiles in raster order are handed out as two units each,
+  // their two 128-column halves, so that a last partial wave of whole tiles
+  // on under half of the CTA pairs becomes a wave of half tiles on all of
+  // them (0: every unit is a whole tile).
+  int nsplit;
+
+  __device__ __forceinline__ int nunits() const { return ntiles + nsplit; }
+
+  // Unit u -> tile (mb, nb) and half (-1 for a whole tile, else 0 or 1).
+  __device__ __forceinline__ void map_unit(int u, int& mb, int& nb, int& half) const {
+    const int s0 = ntiles - nsplit;
+    int t = u;
+    half = -1;
+    if (u >= s0) {
+      t = s0 + ((u - s0) >> 1);
+      half = (u - s0) & 1;
+    }
+    map(t, mb, nb);
+  }
 
   __device__ __forceinline__ void map(int t, int& mb, int& nb) const {
     const int per_group = group_m * n_nt;
@@ -78,11 +97,25 @@ struct epi_warps<E, decltype(void(E::kWarps))> {
   static constexpr int value = E::kWarps;
 };
 
+// Epilogues that declare kSplitN = true take a column range of 128 (a half
+// tile, c.cbeg = 0 or 128) as well as whole tiles; the host may then split
+// the last partial wave (TileSched::nsplit).
+template <class E, class = void>
+struct epi_split {
+  static constexpr bool value = false;
+};
+template <class E>
+struct epi_split<E, decltype(void(E::kSplitN))> {
+  static constexpr bool value = E::kSplitN;
+};
+
 template <class Epi>
 struct GemmParams {
   CUtensorMap tmA;
   CUtensorMap tmB;
   CUtensorMap tmB2;  // second half of a paired B operand (SwiGLU up columns)
+  CUtensorMap tmBh;  // K-major B with a 64-row box: this CTA's columns of a half tile
+  int has_bh;        // tmBh is encoded (a K-major B may then be split into half tiles)
   typename Epi::Params ep;
   int M, N, K;       // GEMM sizes; N counts accumulator columns of the output space
   TileSched sched;
@@ -107,17 +140,12 @@ struct TileCtx {
   uint64_t* wbars;   // this warp's epilogue mbarriers
   bool has_next;     // this CTA has another tile after this one
   int nrow0, ncol0;  // first row of this warp / first column of that next tile
-  // Column range of the tile this warp handles: all of it, or (with eight
-  // epilogue warps) one half.  Epilogues that sum over a row's columns
-  // (kBarsPerWarp >= 1) combine the two halves of a lane quarter in `xchg`
-  // (two parity slots of 32 floats) behind the mbarrier `xbar`; for the
-  // others both stay null.
+  // Column range of the tile this warp handles, in accumulator columns: all
+  // of it; with eight epilogue warps one half (`split`, `half`); or, for a
+  // half-tile unit of the split last wave, the 128 columns it computed.
   int cbeg = 0, cend = 256;
   bool split = false;
   int half = 0;
-  int par = 0;       // tile parity: the xchg slot and the xbar phase of this tile
-  float* xchg = nullptr;
-  uint64_t* xbar = nullptr;
 };
 
 template <int BN, int STAGES, bool PAIR, class Epi>
@@ -127,11 +155,9 @@ struct GemmSmem {
   static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * kBK * 2;    // this CTA's columns of B
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kEpiBytes = kEW * Epi::kSmemPerWarp;
-  static constexpr bool kHandOver = kEW == 8 && Epi::kBarsPerWarp >= 1;  // halves combine a row sum
-  static constexpr int kXchgBytes = kHandOver ? 4 * 2 * 32 * 4 : 0;     // per lane quarter: two slots of 32 floats
   static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1 + kEW * Epi::kBarsPerWarp;
   static constexpr int kBytes =
-      1024 /*align slack*/ + STAGES * kStageBytes + kEpiBytes + kXchgBytes + kNumBars * 8 + 16;
+      1024 /*align slack*/ + STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 16;
   static_assert(kEW == 4 || kEW == 8, "four or eight epilogue warps");
   static_assert(Epi::kSmemPerWarp % 1024 == 0, "per-warp epilogue buffers keep the 128-byte swizzle alignment");
 };
@@ -163,13 +189,14 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
   constexpr bool kF8 = epi_fp8<Epi>::value;
   constexpr int kKb = kF8 ? 2 * kBK : kBK;       // K elements per k-block (128 bytes per row)
   static_assert(!kF8 || (!A_MN && !B_MN && PAIR), "e4m3 operands: K-major A and B, CTA pairs");
+  constexpr bool kSplit = epi_split<Epi>::value;
+  static_assert(!kSplit || (PAIR && kEW == 4 && !kF8 && !Epi::kPairedB), "half tiles: bf16 CTA pairs, 4 epilogue warps");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * S::kABytes;
   uint8_t* sEpi = smem + STAGES * S::kStageBytes;
-  float* sXchg = reinterpret_cast<float*>(sEpi + S::kEpiBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + S::kEpiBytes + S::kXchgBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + S::kEpiBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
@@ -222,7 +249,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
   if (p.pdl_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (p.pdl_wait) asm volatile("griddepcontrol.wait;" ::: "memory");
   const int nkb = (p.K + kKb - 1) / kKb;
-  const int ntiles = p.sched.ntiles;
+  const int ntiles = p.sched.nunits();  // schedule units: whole tiles, then (with nsplit) half tiles
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -233,10 +260,12 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
       bool ok = true;
       const uint32_t full0 = PAIR ? mapa_shared(smem_u32(full), 0) : 0u;  // rank 0's full[0]
       for (int t = tile_first; ok && t < ntiles; t += tile_step) {
-        int mb, nb;
-        p.sched.map(t, mb, nb);
+        int mb, nb, half;
+        p.sched.map_unit(t, mb, nb, half);
         const int arow = mb * kTileM + static_cast<int>(rank) * kBM;  // first A row of this CTA
-        const int bcol = nb * BN + static_cast<int>(rank) * kBCols;   // first B column of this CTA
+        // first B column of this CTA: a half tile covers BN/2 columns, kBCols/2 per CTA
+        const int bcol = half < 0 ? nb * BN + static_cast<int>(rank) * kBCols
+                                  : nb * BN + half * (BN / 2) + static_cast<int>(rank) * (kBCols / 2);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, w)) {
             ok = false;
@@ -245,7 +274,9 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
           uint8_t* a = sA + stage * S::kABytes;
           uint8_t* b = sB + stage * S::kBBytes;
           if (PAIR) {
-            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * S::kStageBytes);
+            if (rank == 0)
+              mbar_arrive_expect_tx(&full[stage], half < 0 ? 2 * S::kStageBytes
+                                                           : 2 * (S::kABytes + S::kBBytes / 2));
             const uint32_t fb = full0 + stage * 8;
             if (!A_MN) {
               tma_load_2d_pair(a, &p.tmA, fb, kb * kKb, arow);
@@ -254,7 +285,13 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
               for (int j = 0; j < kBM / 64; ++j)
                 tma_load_2d_pair(a + j * (64 * kBK * 2), &p.tmA, fb, arow + j * 64, kb * kBK);
             }
-            if (!B_MN) {
+            if (kSplit && half >= 0) {
+              // this CTA's 64 columns of the half tile
+              if (!B_MN)
+                tma_load_2d_pair(b, &p.tmBh, fb, kb * kKb, bcol);
+              else
+                tma_load_2d_pair(b, &p.tmB, fb, bcol, kb * kBK);
+            } else if (!B_MN) {
               tma_load_2d_pair(b, &p.tmB, fb, kb * kKb, bcol);
             } else if (Epi::kPairedB) {
               // rank 0 holds the gate half, rank 1 the up half of the accumulator columns
@@ -317,6 +354,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0 && rank == 0) {
       constexpr uint32_t kIdesc = kF8 ? idesc_e4m3_f32(kTileM, BN) : idesc_bf16_f32(kTileM, BN, A_MN, B_MN);
+      constexpr uint32_t kIdescH = idesc_bf16_f32(kTileM, BN / 2, A_MN, B_MN);  // a half tile: N = BN / 2
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -324,9 +362,16 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
       for (int t = tile_first; ok && t < ntiles; t += tile_step, ++it) {
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
+        int half = -1;
+        if (kSplit) {
+          int mb_, nb_;
+          p.sched.map_unit(t, mb_, nb_, half);
+        }
+        const uint32_t idesc = (kSplit && half >= 0) ? kIdescH : kIdesc;
         if (!mbar_wait(&tempty[acc], aph ^ 1u, w)) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + acc * BN;
+        // a half tile accumulates into the accumulator columns it covers
+        const uint32_t d = tmem_base + acc * BN + (half > 0 ? BN / 2 : 0);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, w)) {
             ok = false;
@@ -344,7 +389,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
             if (kF8)
               tc_mma_f8_pair(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
             else if (PAIR)
-              tc_mma_bf16_pair(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+              tc_mma_bf16_pair(d, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
             else
               tc_mma_bf16(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
           }
@@ -383,8 +428,8 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
     Epi::init_state(st);
     int it = 0;
     for (int t = tile_first; t < ntiles; t += tile_step, ++it) {
-      int mb, nb;
-      p.sched.map(t, mb, nb);
+      int mb, nb, half_t;
+      p.sched.map_unit(t, mb, nb, half_t);
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       // Warp-uniform outcome: tcgen05.ld below is a warp-collective instruction.
@@ -404,19 +449,19 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
       c.nrow0 = 0;
       c.ncol0 = 0;
       if (c.has_next) {
-        int nmb, nnb;
-        p.sched.map(t + tile_step, nmb, nnb);
+        int nmb, nnb, nhalf;
+        p.sched.map_unit(t + tile_step, nmb, nnb, nhalf);
         c.nrow0 = nmb * kTileM + static_cast<int>(rank) * kBM + q * 32;
-        c.ncol0 = nnb * BN;
+        c.ncol0 = nnb * BN + (nhalf > 0 ? BN / 2 : 0);
       }
       c.split = kEW == 8;
       c.half = half;
       c.cbeg = kEW == 8 ? half * (BN / 2) : 0;
       c.cend = kEW == 8 ? (half + 1) * (BN / 2) : BN;
-      c.par = it & 1;
-      if (S::kHandOver) {
-        c.xchg = sXchg + q * 64;                                        // the lane quarter's two slots
-        c.xbar = ebars + (half == 0 ? ew : ew - 4) * Epi::kBarsPerWarp;  // the first-half warp's barrier
+      if (kSplit && half_t >= 0) {
+        // a half tile: its 128 columns, in the accumulator columns of the same range
+        c.cbeg = half_t * (BN / 2);
+        c.cend = c.cbeg + BN / 2;
       }
       const bool ok = Epi::template tile<BN>(p.ep, c, st, w);
       tc_fence_before();
@@ -477,7 +522,7 @@ __device__ __forceinline__ float acc_at(const uint32_t (&v0)[32], const uint32_t
 // memory (128-byte swizzle) and written by TMA stores from one staging buffer
 // per warp (a second buffer would cost the mainloop its sixth pipeline stage,
 // which is worth more: 63.5 against 65.5 us on the 1B block's first GEMM).
-// partial is laid out [column tile][row] (fp32).
+// partial is laid out [128-column slot][row] (fp32).
 // ---------------------------------------------------------------------------
 template <int MODE>
 struct EpiLoadStore2 {
@@ -493,8 +538,11 @@ struct EpiLoadStore2 {
   // modes keep four warps and with them a sixth pipeline stage (63.5 against
   // 66.6 us with eight warps and five stages).
   static constexpr int kWarps = MODE == 2 ? 8 : 4;
-  static constexpr int kBarsPerWarp = MODE == 2 ? 1 : 0;  // the halves' hand-over of the row sums
+  static constexpr int kBarsPerWarp = 0;
   static constexpr bool kPairedB = false;
+  // bf16 modes take half tiles (the split last wave); the e4m3 mode keeps
+  // whole tiles (its eight warps already halve each tile's columns)
+  static constexpr bool kSplitN = MODE != 2;
 
   struct Params {
     CUtensorMap tmOut1;          // [M, N] bf16, box 64 x 32
@@ -533,7 +581,8 @@ struct EpiLoadStore2 {
   }
 
   template <int BN>
-  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx& w) {
+  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
+    static_assert(BN == 256, "partials are kept per 128-column half of a 256-column tile");
     const int col0 = c.nb * BN + c.cbeg;  // first column of this warp's share of the tile
     const int row = c.row0 + c.lane;
     int nch = (c.N - col0 + 63) / 64;
@@ -580,6 +629,8 @@ struct EpiLoadStore2 {
         st.pre_row = row;
         st.pre_col = nc;
       } else if (c.has_next) {
+        // (with eight warps the next tile has the same split of columns; a
+        // half-tile unit is the last unit of its CTA pair)
         const int nrow = c.nrow0 + c.lane;
         load_chunk(ep, c.M, c.N, nrow, c.ncol0 + c.cbeg, st.pre);
         st.pre_row = nrow;
@@ -684,20 +735,15 @@ struct EpiLoadStore2 {
       else
         ss_hi += ss;
     }
-    float ssum = ss_lo + ss_hi;
-    if (c.split) {
-      // the second half hands its sum to the first half of the same lane quarter
-      if (c.half == 1) {
-        c.xchg[c.par * 32 + c.lane] = ss_hi;
-        __syncwarp();
-        if (c.lane == 0) mbar_arrive(c.xbar);
-      } else {
-        if (!__all_sync(0xffffffffu, mbar_wait(c.xbar, static_cast<uint32_t>(c.par), w))) return false;
-        ssum = ss_lo + c.xchg[c.par * 32 + c.lane];
-      }
+    // One partial per 128-column slot: slot 2 nb holds the tile's first half,
+    // slot 2 nb + 1 its second half (when it starts inside N).  Whichever warp,
+    // or half-tile unit, covers a half writes its slot, so halves computed by
+    // different warps or CTA pairs need no hand-over.
+    if (ep.partial != nullptr && row < c.M) {
+      const int s0 = 2 * c.nb;
+      if (c.cbeg < BN / 2) ep.partial[static_cast<size_t>(s0) * c.M + row] = ss_lo;
+      if (c.cend > BN / 2 && (s0 + 1) * (BN / 2) < c.N) ep.partial[static_cast<size_t>(s0 + 1) * c.M + row] = ss_hi;
     }
-    if (ep.partial != nullptr && row < c.M && c.half == 0)
-      ep.partial[static_cast<size_t>(c.nb) * c.M + row] = ssum;
     if (MODE == 2) {
       const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(amx));  // |hg| >= 0: bits order as values
       if (c.lane == 0 && m != 0u) atomicMax(ep.amax, m);
@@ -723,6 +769,7 @@ struct EpiRowScale {
   static constexpr int kSmemPerWarp = 2 * 4096;
   static constexpr int kBarsPerWarp = 0;
   static constexpr bool kPairedB = false;
+  static constexpr bool kSplitN = true;
 
   struct Params {
     CUtensorMap tmOut;     // [M, N] bf16, box 64 x 32
@@ -741,10 +788,10 @@ struct EpiRowScale {
 
   template <int BN>
   __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
-    const int col0 = c.nb * BN;
+    const int col0 = c.nb * BN + c.cbeg;  // first column of this unit (a half tile starts at 128)
     const int row = c.row0 + c.lane;
     int nch = (c.N - col0 + 63) / 64;
-    if (nch > BN / 64) nch = BN / 64;
+    if (nch > (c.cend - c.cbeg) / 64) nch = (c.cend - c.cbeg) / 64;
     float rs = 1.f;
     if (ep.partial != nullptr) {
       rs = 0.f;
@@ -754,7 +801,7 @@ struct EpiRowScale {
         // by other CTAs of the same kernel
         for (int t = 0; t < ep.T; ++t) sum += __ldcg(ep.partial + static_cast<size_t>(t) * c.M + row);
         rs = rsqrtf(sum * ep.inv_n + ep.eps);
-        if (ep.r_out != nullptr && c.nb == 0) ep.r_out[row] = rs;
+        if (ep.r_out != nullptr && c.nb == 0 && c.cbeg == 0) ep.r_out[row] = rs;
       }
     } else if (ep.r != nullptr) {
       rs = (row < c.M) ? __ldg(ep.r + row) : 0.f;
@@ -765,7 +812,7 @@ struct EpiRowScale {
       if (c.lane == 0) bulk_wait_read<1>();
       __syncwarp();
       uint32_t v0[32], v1[32];
-      tmem_ld64(c.taddr + ch * 64, v0, v1);
+      tmem_ld64(c.taddr + c.cbeg + ch * 64, v0, v1);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         uint32_t o[4];
@@ -796,6 +843,7 @@ struct EpiRowScale {
 // the bf16 block.
 struct EpiRowScaleF8 : EpiRowScale {
   static constexpr bool kFp8 = true;
+  static constexpr bool kSplitN = false;
 };
 
 // ---------------------------------------------------------------------------
@@ -812,6 +860,7 @@ struct EpiStoreF32 {
   static constexpr int kSmemPerWarp = 2 * 4096;
   static constexpr int kBarsPerWarp = 0;
   static constexpr bool kPairedB = false;
+  static constexpr bool kSplitN = true;
 
   struct Params {
     CUtensorMap tmOut;   // [M, N] fp32, box 32 x 32
@@ -832,13 +881,13 @@ struct EpiStoreF32 {
   template <int BN>
   __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
     static_assert(BN <= 256 && 256 % BN == 0, "a tile lies within one 256-column label bucket");
-    const int col0 = c.nb * BN;
+    const int col0 = c.nb * BN + c.cbeg;  // first column of this unit (a half tile starts at 128)
     const int row = c.row0 + c.lane;
     int nch = (c.N - col0 + 31) / 32;
-    if (nch > BN / 32) nch = BN / 32;
+    if (nch > (c.cend - c.cbeg) / 32) nch = (c.cend - c.cbeg) / 32;
     // this tile's run of (label, row) entries
     int e0 = 0, e1 = 0;
-    if (ep.fix_start != nullptr) {
+    if (ep.fix_start != nullptr && nch > 0) {
       const int bkt = ep.fix_tile0 + col0 / 256;
       e0 = ep.fix_start[bkt];
       e1 = ep.fix_start[bkt + 1];
@@ -880,7 +929,7 @@ struct EpiStoreF32 {
       if (c.lane == 0) bulk_wait_read<1>();
       __syncwarp();
       uint32_t v[32];
-      tmem_ld32(c.taddr + ch * 32, v);
+      tmem_ld32(c.taddr + c.cbeg + ch * 32, v);
       tmem_ld_wait(v);
       if (ep.accum != nullptr) {
 #pragma unroll

@@ -28,9 +28,12 @@ __global__ void rms_reduce_kernel(const float* __restrict__ partial, int M, int 
 //   dh = gamma * d_hg + coef * h  (d_hg fp32, h bf16, dh bf16);  dgamma partial
 //   over the block's rows.
 // Each thread owns 8 consecutive columns and walks the rows, so every row
-// access is a coalesced vector sweep.
+// access is a coalesced vector sweep; four rows at a time, their loads issued
+// before any of them is used, so that enough bytes are in flight per SM to
+// keep HBM busy.
 constexpr int kBwdRows = 32;
 constexpr int kBwdThreads = 256;
+constexpr int kBwdUnroll = 4;
 
 __global__ void __launch_bounds__(kBwdThreads) rms_reduce_bwd_kernel(
     const float* __restrict__ pdr, const float* __restrict__ r, const float* __restrict__ d_hg,
@@ -57,24 +60,40 @@ __global__ void __launch_bounds__(kBwdThreads) rms_reduce_bwd_kernel(
     float dg[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) dg[e] = 0.f;
-    for (int rr = 0; rr < nrows; ++rr) {
-      const size_t o = static_cast<size_t>(r0 + rr) * N + c0;
-      const float4 a4lo = *reinterpret_cast<const float4*>(d_hg + o);
-      const float4 a4hi = *reinterpret_cast<const float4*>(d_hg + o + 4);
-      const uint4 h4 = *reinterpret_cast<const uint4*>(h + o);
-      const float av[8] = {a4lo.x, a4lo.y, a4lo.z, a4lo.w, a4hi.x, a4hi.y, a4hi.z, a4hi.w};
-      const uint32_t hw[4] = {h4.x, h4.y, h4.z, h4.w};
-      const float cf = coef[rr];
-      uint32_t out[4];
+    for (int rb = 0; rb < nrows; rb += kBwdUnroll) {
+      float4 alo[kBwdUnroll], ahi[kBwdUnroll];
+      uint4 hv[kBwdUnroll];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float a0 = av[2 * e], a1 = av[2 * e + 1];
-        const float h0 = bf16lo(hw[e]), h1 = bf16hi(hw[e]);
-        dg[2 * e] = fmaf(a0, h0, dg[2 * e]);
-        dg[2 * e + 1] = fmaf(a1, h1, dg[2 * e + 1]);
-        out[e] = pack_bf16x2(fmaf(bf16lo(gw[e]), a0, cf * h0), fmaf(bf16hi(gw[e]), a1, cf * h1));
+      for (int u = 0; u < kBwdUnroll; ++u) {
+        if (rb + u < nrows) {
+          const size_t o = static_cast<size_t>(r0 + rb + u) * N + c0;
+          alo[u] = __ldcs(reinterpret_cast<const float4*>(d_hg + o));
+          ahi[u] = __ldcs(reinterpret_cast<const float4*>(d_hg + o + 4));
+          hv[u] = __ldcs(reinterpret_cast<const uint4*>(h + o));
+        } else {
+          alo[u] = ahi[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          hv[u] = make_uint4(0, 0, 0, 0);
+        }
       }
-      *reinterpret_cast<uint4*>(dh + o) = make_uint4(out[0], out[1], out[2], out[3]);
+#pragma unroll
+      for (int u = 0; u < kBwdUnroll; ++u) {
+        if (rb + u >= nrows) break;
+        const size_t o = static_cast<size_t>(r0 + rb + u) * N + c0;
+        const float av[8] = {alo[u].x, alo[u].y, alo[u].z, alo[u].w, ahi[u].x, ahi[u].y, ahi[u].z, ahi[u].w};
+        const uint32_t hw[4] = {hv[u].x, hv[u].y, hv[u].z, hv[u].w};
+        const float cf = coef[rb + u];
+        uint32_t out[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a0 = av[2 * e], a1 = av[2 * e + 1];
+          const float h0 = bf16lo(hw[e]), h1 = bf16hi(hw[e]);
+          dg[2 * e] = fmaf(a0, h0, dg[2 * e]);
+          dg[2 * e + 1] = fmaf(a1, h1, dg[2 * e + 1]);
+          out[e] = pack_bf16x2(fmaf(bf16lo(gw[e]), a0, cf * h0), fmaf(bf16hi(gw[e]), a1, cf * h1));
+        }
+        // dh is read next by the dx and dW1 GEMMs: a plain store leaves it in L2
+        *reinterpret_cast<uint4*>(dh + o) = make_uint4(out[0], out[1], out[2], out[3]);
+      }
     }
     float* dst = dgamma_part + static_cast<size_t>(blockIdx.x) * N + c0;
     *reinterpret_cast<float4*>(dst) = make_float4(dg[0], dg[1], dg[2], dg[3]);
@@ -82,13 +101,29 @@ __global__ void __launch_bounds__(kBwdThreads) rms_reduce_bwd_kernel(
   }
 }
 
-// dgamma_j = sum over row blocks (fixed order) of the block partials.
-__global__ void dgamma_final_kernel(const float* __restrict__ part, int nblk, int N, float* __restrict__ dgamma) {
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= N) return;
+// dgamma_j = sum over row blocks of the block partials, in a fixed order:
+// a block of 256 threads takes 32 columns; thread (g, j) sums the partials of
+// row blocks g, g + 8, g + 16, ... of column j, and the 8 group sums of a
+// column are added in group order.
+constexpr int kDgCols = 32;
+constexpr int kDgGroups = 8;
+
+__global__ void __launch_bounds__(kDgCols * kDgGroups) dgamma_final_kernel(const float* __restrict__ part, int nblk,
+                                                                         int N, float* __restrict__ dgamma) {
+  __shared__ float red[kDgGroups][kDgCols];
+  const int jl = threadIdx.x % kDgCols, grp = threadIdx.x / kDgCols;
+  const int j = blockIdx.x * kDgCols + jl;
   float s = 0.f;
-  for (int b = 0; b < nblk; ++b) s += part[static_cast<size_t>(b) * N + j];
-  dgamma[j] = s;
+  if (j < N)
+    for (int b = grp; b < nblk; b += kDgGroups) s += part[static_cast<size_t>(b) * N + j];
+  red[grp][jl] = s;
+  __syncthreads();
+  if (grp == 0 && j < N) {
+    float t = 0.f;
+#pragma unroll
+    for (int g = 0; g < kDgGroups; ++g) t += red[g][jl];
+    dgamma[j] = t;
+  }
 }
 
 // Cross-entropy combine: per row, merge the (max, sum-exp) pairs of all
@@ -151,6 +186,38 @@ __global__ void __launch_bounds__(1024) mean_kernel(const float* __restrict__ lo
     __syncthreads();
   }
   if (threadIdx.x == 0) *mean = red[0] / static_cast<float>(M);
+}
+
+// Data-parallel cross-entropy ("What CODA can do": the article is single-GPU;
+// splitting the tokens over ranks is this library's).  A rank reports
+// (sum of its tokens' losses, its token count); the caller sums the pairs over
+// ranks (an all-reduce of 8 bytes); the global mean is sum / count and each
+// token's loss weight in the backward is 1 / count.
+__global__ void __launch_bounds__(1024) loss_stats_kernel(const float* __restrict__ loss, int M,
+                                                          float* __restrict__ stats) {
+  __shared__ float red[1024];
+  float s = 0.f;
+  for (int i = threadIdx.x; i < M; i += 1024) s += loss[i];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 512; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    stats[0] = red[0];
+    stats[1] = static_cast<float>(M);
+  }
+}
+
+__global__ void ce_global_finish_kernel(const float* __restrict__ stats, int M, float* __restrict__ mean,
+                                        float* __restrict__ d_loss) {
+  const float sum = stats[0], count = stats[1];
+  if (mean != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *mean = sum / count;
+  if (d_loss != nullptr) {
+    const float w = 1.0f / count;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < M; i += gridDim.x * blockDim.x) d_loss[i] = w;
+  }
 }
 
 // Cross-entropy backward: exact label entries.  The chunked backward stores the

@@ -80,11 +80,13 @@ const char* coda_status_string(coda_status_t s);
 /* Library ABI version (increments on any signature change). */
 int coda_version(void);
 
-/* Column-tile width used by the partial-sum layouts (partial, pdr): 256. */
+/* Columns summed into one entry of the partial-sum layouts (partial, pdr):
+ * 128, one half of a 256-column GEMM tile (the halves of a tile may be
+ * computed by different CTA pairs when a GEMM's last wave is split). */
 int64_t coda_partial_tile_width(void);
 
-/* Number of column tiles T = ceil(N / coda_partial_tile_width()) for a hidden
- * size N; partial and pdr arrays are [T, M] fp32 (tile-major: entry (t, i) at
+/* Number of column slots T = ceil(N / coda_partial_tile_width()) for a hidden
+ * size N; partial and pdr arrays are [T, M] fp32 (slot-major: entry (t, i) at
  * index t * M + i).  Returns -1 if N <= 0. */
 int64_t coda_partial_cols(int64_t N);
 
@@ -105,7 +107,8 @@ coda_status_t coda_poll_status(void* stream);
  *   acc = x W (fp32);  h = acc + res (res may be NULL: h = acc);
  *   h_out  = bf16(h)                     [M, N]  (NULL: not stored)
  *   hg_out = bf16(gamma * h)             [M, N]  (NULL: not stored; needs gamma)
- *   partial[t, i] = sum_{j in tile t} h_ij^2 (fp32, from the unrounded h) [T, M] (NULL: not stored)
+ *   partial[t, i] = sum_{j in slot t} h_ij^2 (fp32, from the unrounded h) [T, M] (NULL: not stored;
+ *                   slot t = columns [128 t, 128 t + 128))
  * x [M, K] bf16, W [K, N] bf16, res [M, N] bf16, gamma [N] bf16.
  * At least one output must be non-NULL.  Also used as the down projection of
  * the SwiGLU chain (x = act, res = h, partials for the next layer's norm). */
@@ -246,14 +249,29 @@ coda_status_t coda_lmhead_ce_bwd(const uint16_t* H, const uint16_t* W, const int
                                  const float* d_loss, const float* r, float* dH_out, float* dW_out, void* ws,
                                  size_t ws_bytes, int64_t M, int64_t V, int64_t K, void* stream);
 
-/* ---------------------------------------------------------------- backward */
+/* Data-parallel cross-entropy (tokens split over ranks; the article is
+ * single-GPU, section "What CODA can do").  stats_out[0] = sum of loss[0..M),
+ * stats_out[1] = M (fp32; one block, fixed order: deterministic; a NaN loss
+ * makes the sum NaN).  The caller sums stats over ranks (an all-reduce of 8
+ * bytes).  loss [M] fp32, stats_out [2] fp32, device.  0 < M < 2^24. */
+coda_status_t coda_loss_stats(const float* loss, int64_t M, float* stats_out, void* stream);
+
+/* From the rank-summed stats: mean_out[0] = stats[0] / stats[1] (the mean
+ * over every rank's tokens) and d_loss_out[i] = 1 / stats[1] for i < M, the
+ * per-token weight that coda_lmhead_ce_bwd takes as d_loss so that dW is the
+ * gradient of the global mean (to be summed over ranks).  Either output may
+ * be NULL, not both.  stats [2], mean_out [1], d_loss_out [M]: device fp32. */
+coda_status_t coda_ce_global_finish(const float* stats, int64_t M, float* mean_out, float* d_loss_out,
+                                    void* stream);
+
+/* ---------------------------------------------------------------- backward *//* ---------------------------------------------------------------- backward */
 
 /* Bytes of workspace coda_gemm_rowscale_bwd needs (holds y = r * hg, bf16 [M, N]). */
 size_t coda_gemm_rowscale_bwd_workspace_size(int64_t M, int64_t N);
 
 /* Backward of out = r * (hg W2) in block-local form.
  *   P = dOut W2^T (fp32, on chip);  d_hg_out = r * P (fp32)           [M, N]
- *   y = bf16(r * hg) (workspace);  pdr[t, i] = sum_{j in tile t} hg_ij P_ij   [T, M] fp32
+ *   y = bf16(r * hg) (workspace);  pdr[t, i] = sum_{j in slot t} hg_ij P_ij   [T, M] fp32
  *   dW2_out = y^T dOut (fp32)                                          [N, N2]
  * dOut [M, N2] bf16, hg [M, N] bf16, W2 [N, N2] bf16, r [M] fp32.
  * d_hg and pdr feed coda_rms_reduce_bwd. */
@@ -360,8 +378,8 @@ coda_status_t coda_fp8_quantize(const uint16_t* src, int64_t rows, int64_t cols,
 coda_status_t coda_fp8_scale_from_amax(const float* amax, float* scale_out, void* stream);
 
 /* First GEMM of the FP8 block: acc = x8 Wt8^T (e4m3 x e4m3 -> fp32), then in
- * the epilogue h = acc * sx * sw + res, partial[t, i] = sum over 256-column
- * tile t of h^2 (from the fp32 h), h_out = bf16(h),
+ * the epilogue h = acc * sx * sw + res, partial[t, i] = sum over 128-column
+ * slot t of h^2 (from the fp32 h), h_out = bf16(h),
  * hg8_out = e4m3(gamma * h / s_hg), and amax_out = max |gamma * h| over the
  * whole output (zeroed by this call, then raised by atomic max).
  * x8 [M, K], Wt8 [N, K] (the weight transposed), hg8_out [M, N] e4m3;

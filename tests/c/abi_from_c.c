@@ -27,7 +27,7 @@ int main(void) {
     printf("FAIL version\n");
     ++failures;
   }
-  if (coda_partial_tile_width() != 256 || coda_partial_cols(2048) != 8) {
+  if (coda_partial_tile_width() != 128 || coda_partial_cols(2048) != 16) {
     printf("FAIL partial layout\n");
     ++failures;
   }

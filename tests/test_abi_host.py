@@ -48,10 +48,10 @@ def test_status_strings_and_constants(lib):
         assert s.startswith(binding.STATUS_NAMES[code])
     assert lib.coda_status_string(99).decode() == "CODA_ERR_UNKNOWN"
     assert lib.coda_version() >= 1
-    assert lib.coda_partial_tile_width() == 256
-    assert lib.coda_partial_cols(2048) == 8
-    assert lib.coda_partial_cols(512) == 2
-    assert lib.coda_partial_cols(520) == 3
+    assert lib.coda_partial_tile_width() == 128
+    assert lib.coda_partial_cols(2048) == 16
+    assert lib.coda_partial_cols(512) == 4
+    assert lib.coda_partial_cols(520) == 5
     assert lib.coda_partial_cols(0) == -1
     assert lib.coda_lmhead_ce_workspace_size(8192, 128256) >= 2 * 501 * 8192 * 4 + 8192 * 4
     assert lib.coda_gemm_rowscale_bwd_workspace_size(8192, 2048) >= 8192 * 2048 * 2
@@ -152,6 +152,17 @@ def test_argument_errors_of_the_remaining_calls(lib):
     assert rope(A, B, None, D, 16, 384, 64, 64, 192, 5e5, None) == NULL   # positions
     assert rope(A, B, C, MIS, 16, 384, 64, 64, 192, 5e5, None) == ALIGN
     assert rope(A, B, C, D, 0, 384, 64, 64, 192, 5e5, None) == OK
+
+    ls = lib.coda_loss_stats  # (loss, M, stats_out, stream)
+    assert ls(A, 0, B, None) == SHAPE
+    assert ls(A, 1 << 24, B, None) == SHAPE      # the count must stay exact in fp32
+    assert ls(None, 16, B, None) == NULL
+    assert ls(A, 16, MIS, None) == ALIGN
+    gf = lib.coda_ce_global_finish  # (stats, M, mean_out, d_loss_out, stream)
+    assert gf(A, -1, B, C, None) == SHAPE
+    assert gf(A, 16, None, None, None) == NULL
+    assert gf(None, 16, B, C, None) == NULL
+    assert gf(A, 16, B, MIS, None) == ALIGN
 
     sb = lib.coda_gemm_swiglu_bwd  # (d_out, W_down, gateup, d_gateup, M, F, N, stream)
     assert sb(A, B, C, D, 16, 60, 64, None) == SHAPE                     # F not a multiple of 8

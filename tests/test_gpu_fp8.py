@@ -80,7 +80,7 @@ def _oracle_block(ora, res, gamma, s_hg, eps, rows=None):
     x8 = ora["x8"] if rows is None else ora["x8"][rows]
     res = res if rows is None else res[rows]
     return F8.rmsnorm_block_fp8(x8, ora["sx"], ora["W1t8"], ora["sw1"], res, gamma, s_hg, ora["W2t8"], ora["sw2"],
-                                eps)
+                                eps, tile_cols=C.partial_tile_width())
 
 
 def _check_codes(name, got, want, max_frac):

@@ -18,7 +18,6 @@ from tests._util import CE_REL_TOL, b, check, check_rel, dev, host
 
 pytestmark = pytest.mark.gpu
 
-TILE = 256
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -71,14 +70,14 @@ def test_gemm_res_partialrms(M, K, N):
     res = synth.normal_bf16(g, (M, N))
     gamma = synth.gamma_bf16(g, N)
     h, hg, part = C.gemm_res_partialrms(dev(x), dev(W), dev(res), dev(gamma))
-    ref = O.gemm_res_partialrms(b(x), b(W), b(res), b(gamma), TILE)
+    ref = O.gemm_res_partialrms(b(x), b(W), b(res), b(gamma), C.partial_tile_width())
     check("h", h, ref["h"])
     check("hg", hg, ref["hg"])
     assert part.shape == (C.partial_cols(N), M)
     check_rel("partial", part, ref["partial"], 1e-4)
     # without residual, only partials requested
     _, _, p2 = C.gemm_res_partialrms(dev(x), dev(W), None, None, h=False, hg=False)
-    check_rel("partial(no res)", p2, O.gemm_res_partialrms(b(x), b(W), None, None, TILE)["partial"], 1e-4)
+    check_rel("partial(no res)", p2, O.gemm_res_partialrms(b(x), b(W), None, None, C.partial_tile_width())["partial"], 1e-4)
     C.poll_status()
 
 
@@ -181,7 +180,7 @@ def test_swiglu_down_chain():
     # outputs (h2 and its partials) keep the bar.
     check("act", s["act"], d["a"], rel=5e-2, storage_rounding=2.0 ** -7)
     check("h2", s["h2"], d["h2"])
-    p2 = O.gemm_res_partialrms(d["a"], b(inp.W_down), u["h"], None, TILE)["partial"]
+    p2 = O.gemm_res_partialrms(d["a"], b(inp.W_down), u["h"], None, C.partial_tile_width())["partial"]
     check("partial2", s["partial2"], p2)
 
 
@@ -225,7 +224,7 @@ def test_gemm_rowscale_bwd():
     W2 = synth.normal_bf16(g, (N, N2), std=1 / math.sqrt(N))
     r = torch.rand(M, generator=g) + 0.5
     d_hg, dW2, pdr = C.gemm_rowscale_bwd(dev(dOut), dev(hg), dev(W2), dev(r))
-    ref = O.gemm_rowscale_bwd(b(dOut), b(hg), b(W2), r.double().numpy(), TILE)
+    ref = O.gemm_rowscale_bwd(b(dOut), b(hg), b(W2), r.double().numpy(), C.partial_tile_width())
     check("d_hg", d_hg, ref["d_hg"])
     check("dW2", dW2, ref["dW2"])
     check("pdr", pdr, ref["pdr"])
