@@ -58,6 +58,8 @@ _SIGS = {
     "coda_lmhead_ce": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _P]),
     "coda_lmhead_ce_bwd_workspace_size": (_SZ, [_I64, _I64]),
     "coda_lmhead_ce_bwd": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _P]),
+    "coda_loss_stats": (_ST, [_P, _I64, _P, _P]),
+    "coda_ce_global_finish": (_ST, [_P, _I64, _P, _P, _P]),
     "coda_gemm_rowscale_bwd_workspace_size": (_SZ, [_I64, _I64]),
     "coda_gemm_rowscale_bwd": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _SZ, _I64, _I64, _I64, _P]),
     "coda_rms_reduce_bwd_workspace_size": (_SZ, [_I64, _I64]),
@@ -104,9 +106,22 @@ def _check(fn: str, status: int):
         raise CodaError(fn, status, lib.coda_status_string(status).decode())
 
 
+# NVTX ranges around every library call (names as in the C ABI), so that a
+# timeline profiler shows which call launched which kernels; CODA_NVTX=0
+# turns them off.
+_NVTX = os.environ.get("CODA_NVTX", "1") != "0"
+
+
 def _call(name: str, *args):
     lib = load_library()
-    st = getattr(lib, name)(*args)
+    if _NVTX:
+        torch.cuda.nvtx.range_push(name)
+        try:
+            st = getattr(lib, name)(*args)
+        finally:
+            torch.cuda.nvtx.range_pop()
+    else:
+        st = getattr(lib, name)(*args)
     _check(name, st)
 
 
@@ -335,6 +350,23 @@ def lmhead_ce_bwd(H, W, labels, lse, d_loss=None, r=None, ws=None):
     _call("coda_lmhead_ce_bwd", _ptr(H), _ptr(W), _ptr(labels), _ptr(lse), _ptr(d_loss), _ptr(r), _ptr(dH), _ptr(dW),
           _ptr(ws), ws.numel(), M, V, K, _stream())
     return dH, dW
+
+
+def loss_stats(loss, stats_out=None):
+    """(sum of loss, count) as a [2] fp32 device tensor, for an all-reduce over ranks."""
+    _need(loss, F32, "loss")
+    stats_out = _empty((2,), F32, loss) if stats_out is None else stats_out
+    _call("coda_loss_stats", _ptr(loss), loss.numel(), _ptr(stats_out), _stream())
+    return stats_out
+
+
+def ce_global_finish(stats, M: int, mean=True, d_loss=True):
+    """From rank-summed stats: (mean [1] or None, d_loss [M] = 1/count or None)."""
+    _need(stats, F32, "stats", (2,))
+    mean_out = _empty((1,), F32, stats) if mean else None
+    d_out = _empty((M,), F32, stats) if d_loss else None
+    _call("coda_ce_global_finish", _ptr(stats), int(M), _ptr(mean_out), _ptr(d_out), _stream())
+    return mean_out, d_out
 
 
 # ---------------------------------------------------------------- backward
