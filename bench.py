@@ -77,6 +77,8 @@ def parse():
                     help="before each timed step of the headline loop: flush L2 with a 256 MB write, or leave it "
                          "warm (the working set, about 460 MB against a 126 MB L2, evicts most of the inputs "
                          "anyway); the line reports a warm-L2 loop of the block beside the headline either way")
+    ap.add_argument("--warm-steps", type=int, default=50,
+                    help="steps of the warm-L2 loop of the block (0: skip it)")
     ap.add_argument("--kernel-iters", type=int, default=50,
                     help="launches of each fused kernel timed alone for its roofline row")
     ap.add_argument("--no-kernels", action="store_true", help="skip the per-kernel roofline loops")
@@ -499,12 +501,14 @@ def run_ours(args):
     value = DD.weak_scaling_value(FLOPS_BLOCK, args.steps, total_s, ws) / 1e12
 
     # ---- the same block with L2 left warm between steps (no flush)
-    warm_steps = max(args.steps, 50)
-    t0 = time.time()
-    tot_w, _ = timed(block, warm_steps, 3, l2="warm")
-    t1 = time.time()
-    ms_warm = sum(tot_w) / len(tot_w)
-    clocks_warm = clock.window(t0, t1) if clock else None
+    warm_steps = args.warm_steps
+    ms_warm = clocks_warm = None
+    if warm_steps > 0:
+        t0 = time.time()
+        tot_w, _ = timed(block, warm_steps, 3, l2="warm")
+        t1 = time.time()
+        ms_warm = sum(tot_w) / len(tot_w)
+        clocks_warm = clock.window(t0, t1) if clock else None
 
     # ---- every fused kernel in a loop of its own (L2 flushed before each
     # launch), against its roofline; GEMM2's row is the headline roofline
@@ -645,11 +649,12 @@ def run_ours(args):
                 "hbm_bytes_fused_alg": BYTES_FUSED, "hbm_bytes_unfused_alg": BYTES_UNFUSED,
                 "hbm_bytes_removed_alg": BYTES_UNFUSED - BYTES_FUSED,
                 "launches_fused": 2, "launches_unfused": 4,
-                "warm_l2": {"steps": warm_steps, "ms": round(ms_warm, 4),
-                            "tflops": round(FLOPS_BLOCK / (ms_warm / 1e3) / 1e12, 1),
-                            "frac_of_nominal_2250": round(FLOPS_BLOCK / (ms_warm / 1e3) / 2.25e15, 4),
-                            "l2": "no flush between steps (the step's working set is 3.6x the L2)",
-                            "clocks": clocks_warm},
+                "warm_l2": None if ms_warm is None else {
+                    "steps": warm_steps, "ms": round(ms_warm, 4),
+                    "tflops": round(FLOPS_BLOCK / (ms_warm / 1e3) / 1e12, 1),
+                    "frac_of_nominal_2250": round(FLOPS_BLOCK / (ms_warm / 1e3) / 2.25e15, 4),
+                    "l2": "no flush between steps (the step's working set is 3.6x the L2)",
+                    "clocks": clocks_warm},
             },
             "e2e": None if e2e_val is None else {
                 "value": round(e2e_val, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
