@@ -116,6 +116,7 @@ struct GemmParams {
   CUtensorMap tmB2;  // second half of a paired B operand (SwiGLU up columns)
   CUtensorMap tmBh;  // K-major B with a 64-row box: this CTA's columns of a half tile
   int has_bh;        // tmBh is encoded (a K-major B may then be split into half tiles)
+  int no_split;      // the caller rules out half tiles for this launch
   typename Epi::Params ep;
   int M, N, K;       // GEMM sizes; N counts accumulator columns of the output space
   TileSched sched;
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
   constexpr int kKb = kF8 ? 2 * kBK : kBK;       // K elements per k-block (128 bytes per row)
   static_assert(!kF8 || (!A_MN && !B_MN && PAIR), "e4m3 operands: K-major A and B, CTA pairs");
   constexpr bool kSplit = epi_split<Epi>::value;
-  static_assert(!kSplit || (PAIR && kEW == 4 && !kF8 && !Epi::kPairedB), "half tiles: bf16 CTA pairs, 4 epilogue warps");
+  static_assert(!kSplit || (PAIR && !kF8 && !Epi::kPairedB), "half tiles: bf16 CTA pairs, unpaired B");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -459,9 +460,10 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
       c.cbeg = kEW == 8 ? half * (BN / 2) : 0;
       c.cend = kEW == 8 ? (half + 1) * (BN / 2) : BN;
       if (kSplit && half_t >= 0) {
-        // a half tile: its 128 columns, in the accumulator columns of the same range
-        c.cbeg = half_t * (BN / 2);
-        c.cend = c.cbeg + BN / 2;
+        // a half tile: its 128 columns, in the accumulator columns of the same
+        // range (with eight warps, 64 of them per warp)
+        c.cbeg = half_t * (BN / 2) + (kEW == 8 ? half * (BN / 4) : 0);
+        c.cend = c.cbeg + (kEW == 8 ? BN / 4 : BN / 2);
       }
       const bool ok = Epi::template tile<BN>(p.ep, c, st, w);
       tc_fence_before();
@@ -1301,11 +1303,14 @@ struct EpiRope {
   // Eight warps, two per lane quarter, each taking half of the tile's columns
   // (whole heads: 128 columns are two heads of 64 or one of 128).  With
   // 128-wide heads this is 6 % faster than four warps; with 64-wide heads the
-  // two take the same time.
+  // two take the same time.  Half tiles (the split last wave) give each warp
+  // 64 columns: one whole head when heads are 64 wide; the host splits only
+  // then.
   static constexpr int kWarps = 8;
   static constexpr int kSmemPerWarp = 8192;  // two 64-column x 32-row bf16 boxes
   static constexpr int kBarsPerWarp = 0;
   static constexpr bool kPairedB = false;
+  static constexpr bool kSplitN = true;
 
   struct Params {
     CUtensorMap tmOut;      // [M, N] bf16, box 64 x 32
