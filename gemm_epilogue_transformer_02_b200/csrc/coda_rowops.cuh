@@ -102,11 +102,12 @@ __global__ void __launch_bounds__(kBwdThreads) rms_reduce_bwd_kernel(
 }
 
 // dgamma_j = sum over row blocks of the block partials, in a fixed order:
-// a block of 256 threads takes 32 columns; thread (g, j) sums the partials of
-// row blocks g, g + 8, g + 16, ... of column j, and the 8 group sums of a
-// column are added in group order.
-constexpr int kDgCols = 32;
-constexpr int kDgGroups = 8;
+// a block of 256 threads takes 8 columns; thread (g, j) sums the partials of
+// row blocks g, g + 32, g + 64, ... of column j, and the 32 group sums of a
+// column are added in group order.  (N / 8 blocks: 256 for N = 2048, enough
+// loads in flight for a latency-bound 2 MB read.)
+constexpr int kDgCols = 8;
+constexpr int kDgGroups = 32;
 
 __global__ void __launch_bounds__(kDgCols * kDgGroups) dgamma_final_kernel(const float* __restrict__ part, int nblk,
                                                                          int N, float* __restrict__ dgamma) {
