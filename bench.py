@@ -82,6 +82,9 @@ def parse():
     ap.add_argument("--kernel-iters", type=int, default=50,
                     help="launches of each fused kernel timed alone for its roofline row")
     ap.add_argument("--no-kernels", action="store_true", help="skip the per-kernel roofline loops")
+    ap.add_argument("--kernel-cooldown", type=float, default=1.0,
+                    help="seconds the GPU idles before each per-kernel loop, so that one loop's power and heat do "
+                         "not carry into the next")
     ap.add_argument("--sweep", action="store_true",
                     help="also time the block at hidden 4096 (gate/up 28672) and 8192 (gate/up 57344)")
     return ap.parse_args()
@@ -516,6 +519,8 @@ def run_ours(args):
     kern = []
 
     def kloop(name, call, fn, flops, nbytes, bound="tensor", launches=1, dtype="bf16", note=None):
+        torch.cuda.synchronize()
+        time.sleep(args.kernel_cooldown)
         for _ in range(3):
             fn()
         torch.cuda.synchronize()
