@@ -859,6 +859,18 @@ coda_status_t coda_lmhead_ce_bwd(const uint16_t* H, const uint16_t* W, const int
       p.ep.scale = 1.0f / static_cast<float>(M);
       p.ep.col_offset = c0;
       p.ep.resid = resid;
+      if (c0 > 0) {
+        // the previous chunk's label entries of dH, added before this chunk's first tile
+        const int64_t p0 = c0 - kCEBwdChunk;
+        p.ep.fix_entries = entries;
+        p.ep.fix_start = start;
+        p.ep.fix_b0 = static_cast<int>(p0 / kLabelTile);
+        p.ep.fix_b1 = static_cast<int>((c0 + kLabelTile - 1) / kLabelTile);
+        p.ep.fix_W = reinterpret_cast<const __nv_bfloat16*>(W);
+        p.ep.fix_V = V;
+        p.ep.fix_K = static_cast<int>(K);
+        p.ep.fix_dH = dH_out;
+      }
       const coda_status_t st = run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(
           dev, info, p, static_cast<int>(M), static_cast<int>(vc), static_cast<int>(K),
           static_cast<int>((vc + 255) / 256), raster_group(M, vc, K), kKindCEGrad, s);
@@ -890,11 +902,15 @@ coda_status_t coda_lmhead_ce_bwd(const uint16_t* H, const uint16_t* W, const int
       const coda_status_t st = run_grouped(dev, info, p, pb, kKindGroupedCE, s);
       if (st != CODA_OK) return st;
     }
-    // dH's label entries of this chunk, while the chunk of W is still in L2
-    ce_label_dh_fix_kernel<<<info->sms * 4, 256, 0, s>>>(
-        entries, start, static_cast<int>(c0 / kLabelTile), static_cast<int>((c0 + vc + kLabelTile - 1) / kLabelTile),
-        resid, reinterpret_cast<const __nv_bfloat16*>(W), V, static_cast<int>(K), dH_out);
-    if (cudaGetLastError() != cudaSuccess) return CODA_ERR_LAUNCH;
+    if (c0 + vc >= V) {
+      // the last chunk's label entries of dH (every earlier chunk's are added
+      // by the next chunk's gradient GEMM before its first tile)
+      ce_label_dh_fix_kernel<<<info->sms * 4, 256, 0, s>>>(
+          entries, start, static_cast<int>(c0 / kLabelTile),
+          static_cast<int>((c0 + vc + kLabelTile - 1) / kLabelTile), resid, reinterpret_cast<const __nv_bfloat16*>(W),
+          V, static_cast<int>(K), dH_out);
+      if (cudaGetLastError() != cudaSuccess) return CODA_ERR_LAUNCH;
+    }
   }
   return CODA_OK;
 }

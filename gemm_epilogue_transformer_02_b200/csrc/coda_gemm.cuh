@@ -29,6 +29,7 @@
 #pragma once
 
 #include "coda_device.cuh"
+#include "coda_rowops.cuh"
 
 namespace coda {
 
@@ -107,6 +108,17 @@ struct epi_split {
 template <class E>
 struct epi_split<E, decltype(void(E::kSplitN))> {
   static constexpr bool value = E::kSplitN;
+};
+
+// Epilogues that declare kHasPre = true give their warps work to do before
+// the first tile (Epi::pre), while that tile's mainloop runs.
+template <class E, class = void>
+struct epi_pre {
+  static constexpr bool value = false;
+};
+template <class E>
+struct epi_pre<E, decltype(void(E::kHasPre))> {
+  static constexpr bool value = E::kHasPre;
 };
 
 template <class Epi>
@@ -427,6 +439,8 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
     const uint32_t tempty0 = PAIR ? mapa_shared(smem_u32(tempty), 0) : 0u;
     typename Epi::State st;
     Epi::init_state(st);
+    if constexpr (epi_pre<Epi>::value)
+      Epi::pre(p.ep, static_cast<long long>(blockIdx.x) * kEW + ew, static_cast<long long>(gridDim.x) * kEW, lane);
     int it = 0;
     for (int t = tile_first; t < ntiles; t += tile_step, ++it) {
       int mb, nb, half_t;
@@ -1421,6 +1435,7 @@ struct EpiCEGrad {
   static constexpr int kSmemPerWarp = 2 * 4096;
   static constexpr int kBarsPerWarp = 0;
   static constexpr bool kPairedB = false;
+  static constexpr bool kHasPre = true;
 
   struct Params {
     CUtensorMap tmG;        // [M, Vc] bf16, box 64 x 32
@@ -1431,11 +1446,29 @@ struct EpiCEGrad {
     float scale;            // weight of every token when d_loss is null (1/M: the mean)
     float* resid;           // [M]: G - bf16(G) at each row's label entry (or null)
     long long col_offset;   // vocabulary index of this chunk's column 0
+    // The previous chunk's exact label entries of dH (dH[i, :] += resid_i
+    // W[:, label_i] over its label buckets [fix_b0, fix_b1)), added by the
+    // epilogue warps of every CTA before their first tile, while its mainloop
+    // runs; fix_start null: nothing to add.  Launched after the previous
+    // chunk's dH GEMM, so that one has completed (griddepcontrol.wait).
+    const int2* fix_entries;
+    const int* fix_start;
+    int fix_b0, fix_b1;
+    const __nv_bfloat16* fix_W;
+    long long fix_V;
+    int fix_K;
+    float* fix_dH;
   };
   struct State {
     uint32_t cnt;
   };
   __device__ static void init_state(State& s) { s.cnt = 0; }
+
+  __device__ static void pre(const Params& ep, long long warp, long long nwarps, int lane) {
+    if (ep.fix_start != nullptr)
+      ce_label_dh_fix_range(ep.fix_entries, ep.fix_start, ep.fix_b0, ep.fix_b1, ep.resid, ep.fix_W, ep.fix_V,
+                            ep.fix_K, ep.fix_dH, warp, nwarps, lane);
+  }
 
   template <int BN>
   __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {

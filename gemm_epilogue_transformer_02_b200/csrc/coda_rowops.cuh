@@ -323,16 +323,19 @@ __global__ void ce_label_sort_kernel(const int2* __restrict__ unsorted, const in
 // coalesced 128-byte segments of the dH row; every element is written by one
 // thread once.
 constexpr int kDhFixSpan = 8;  // 32-column slices per warp item
-__global__ void ce_label_dh_fix_kernel(const int2* __restrict__ entries, const int* __restrict__ start, int b0,
-                                       int b1, const float* __restrict__ resid, const __nv_bfloat16* __restrict__ W,
-                                       long long V, int K, float* __restrict__ dH) {
+
+// dH[i, :] += resid_i W[:, label_i] for the rows whose labels lie in
+// vocabulary buckets [b0, b1), as warp items (row, 256-column slice) dealt to
+// warps `warp`, `warp + nwarps`, ...; every element receives one addend.
+__device__ __forceinline__ void ce_label_dh_fix_range(const int2* __restrict__ entries, const int* __restrict__ start,
+                                                      int b0, int b1, const float* __restrict__ resid,
+                                                      const __nv_bfloat16* __restrict__ W, long long V, int K,
+                                                      float* __restrict__ dH, long long warp, long long nwarps,
+                                                      int lane) {
   const int first = start[b0];
   const long long n = start[b1] - first;
   const int groups = (K + 32 * kDhFixSpan - 1) / (32 * kDhFixSpan);
-  const int lane = threadIdx.x & 31;
-  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  for (long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; w < n * groups;
-       w += nwarps) {
+  for (long long w = warp; w < n * groups; w += nwarps) {
     const int2 en = entries[first + static_cast<int>(w / groups)];
     const int kbase = static_cast<int>(w % groups) * 32 * kDhFixSpan + lane;
     const float ri = resid[en.y];
@@ -349,6 +352,14 @@ __global__ void ce_label_dh_fix_kernel(const int2* __restrict__ entries, const i
       if (k < K) d[k] += ri * wv[u];
     }
   }
+}
+
+__global__ void ce_label_dh_fix_kernel(const int2* __restrict__ entries, const int* __restrict__ start, int b0,
+                                       int b1, const float* __restrict__ resid, const __nv_bfloat16* __restrict__ W,
+                                       long long V, int K, float* __restrict__ dH) {
+  ce_label_dh_fix_range(entries, start, b0, b1, resid, W, V, K, dH,
+                        (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5,
+                        (static_cast<long long>(gridDim.x) * blockDim.x) >> 5, threadIdx.x & 31);
 }
 
 // ------------------------------------------------------------- FP8 (e4m3)
