@@ -910,14 +910,14 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
     ms = sum(tot) / len(tot)
     res["lmhead_ce_backward"] = {"ms": round(ms, 4), "tflops": round(3 * f_ce / ms / 1e9, 1)}
     if kloop:
-        n_ch = (V_CE + 4095) // 4096
-        # per 4096-column chunk: G = (H, W_c) -> G_c bf16; dH += G_c W_c^T (fp32 read + write);
-        # dW_c = H^T G_c (fp32 write)
-        b_ch = [2 * (M * D + D * 4096 + M * 4096), 2 * (M * 4096 + D * 4096) + 8 * M * D, 2 * (M * D + M * 4096)
-                + 4 * D * 4096]
-        kloop("lmhead_ce_bwd (per chunk: CE-gradient GEMM, grouped dH + dW GEMMs, label fix)", "coda_lmhead_ce_bwd",
-              ceb, 3 * f_ce, n_ch * sum(b_ch), launches=3 * n_ch + 5, note="whole call; per-kernel shares in the "
-              "ncu launch list")
+        CH = 8192  # vocabulary columns per chunk of the backward
+        n_ch = (V_CE + CH - 1) // CH
+        # per chunk: G = (H, W_c) -> G_c bf16; dH += G_c W_c^T (fp32 read + write); dW_c = H^T G_c (fp32 write)
+        b_ch = [2 * (M * D + D * CH + M * CH), 2 * (M * CH + D * CH) + 8 * M * D, 2 * (M * D + M * CH) + 4 * D * CH]
+        kloop("lmhead_ce_bwd (per chunk: CE-gradient GEMM, grouped dH + dW GEMMs)", "coda_lmhead_ce_bwd",
+              ceb, 3 * f_ce, n_ch * sum(b_ch), launches=2 * n_ch + 6, note="whole call: label bucketing (5 "
+              "launches), two GEMM launches per chunk, one label correction after the last; per-kernel shares in "
+              "the ncu launch list")
     del H, Wv, labels, ws_ce, ws_ceb, lse
 
     # backward of the block (dOut std 0.01)

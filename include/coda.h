@@ -225,7 +225,7 @@ coda_status_t coda_lmhead_ce(const uint16_t* H, const uint16_t* W, const int64_t
                              int64_t M, int64_t V, int64_t K, void* stream);
 
 /* Bytes of workspace coda_lmhead_ce_bwd needs: one bf16 gradient chunk of
- * M x min(V, 4096), M fp32 residuals, and the rows bucketed by label (three
+ * M x min(V, 8192), M fp32 residuals, and the rows bucketed by label (three
  * int arrays of ceil(V / 256) entries and two of M (label, row) pairs). */
 size_t coda_lmhead_ce_bwd_workspace_size(int64_t M, int64_t V);
 
@@ -235,14 +235,15 @@ size_t coda_lmhead_ce_bwd_workspace_size(int64_t M, int64_t V);
  * NULL: the mean), with the forward's saved lse:
  *   G_ij = d_i (exp(z_ij - lse_i) - [j == label_i]),  z = r_i (H W)_ij
  *   dH_out = G W^T  [M, K] fp32;   dW_out = H^T G  [K, V] fp32.
- * The vocabulary is processed in chunks of 4096 columns: a GEMM recomputes the
+ * The vocabulary is processed in chunks of 8192 columns: a GEMM recomputes the
  * chunk's logits and its epilogue writes G_chunk (bf16, in the workspace;
  * the logits are never stored), then dH += G_chunk W_chunk^T and
  * dW_chunk = H^T G_chunk run as one grouped launch.  The label entry d_i (p - 1) dominates its dW
- * column, so the part of it that bf16 drops is kept in fp32 and added back in
- * the epilogues of the dH and dW GEMMs (rows bucketed by label beforehand;
- * each dW column sums its rows in increasing row order, so the result is
- * deterministic).  A label outside [0, V) contributes no onehot term.  H [M, K] bf16,
+ * column, so the part of it that bf16 drops is kept in fp32 and added back:
+ * into dW in the dW GEMM's epilogue (rows bucketed by label beforehand; each
+ * dW column sums its rows in increasing row order, so the result is
+ * deterministic), into dH by the next chunk's gradient GEMM before its first
+ * tile (by a small kernel after the last chunk).  A label outside [0, V) contributes no onehot term.  H [M, K] bf16,
  * W [K, V] bf16, labels [M] int64, lse [M] fp32, d_loss and r [M] fp32 or NULL,
  * ws >= coda_lmhead_ce_bwd_workspace_size(M, V). */
 coda_status_t coda_lmhead_ce_bwd(const uint16_t* H, const uint16_t* W, const int64_t* labels, const float* lse,

@@ -28,7 +28,11 @@ def _gpu():
     C.load_library()
 
 
-@pytest.mark.parametrize("M,K,V,weighted", [(300, 136, 5000, False), (129, 64, 4104, True), (64, 256, 1000, False)])
+# V = 17000: two 8192-column chunks and a ragged third (the first two chunks'
+# dH label corrections run inside the next chunk's gradient GEMM, the last
+# one's in its own kernel)
+@pytest.mark.parametrize("M,K,V,weighted", [(300, 136, 5000, False), (129, 64, 4104, True), (64, 256, 1000, False),
+                                            (260, 64, 17000, True)])
 def test_lmhead_ce_bwd_small(M, K, V, weighted):
     g = synth.make_gen(600 + V)
     H = synth.normal_bf16(g, (M, K))
