@@ -124,6 +124,21 @@ bool tmap2d_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, u
   return r == CUDA_SUCCESS;
 }
 
+// e4m3 output rows of 64 bytes without swizzle (staged as plain rows).
+bool tmap2d_u8_plain(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t stride,
+                     uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {stride};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Operand maps of the mainloop.  A: [M, K] K-major (box 64 x 128) or stored
 // transposed as [K, M] (MN-major, box 64 x 64).  B: [K, N] MN-major (box 64 x 64)
 // or stored transposed as [N, K] (K-major, box 64 x BN).
@@ -177,7 +192,8 @@ constexpr int64_t kCEBwdChunk = 8192;
 // of A and B) as fit next to the epilogue's shared memory, at most 8.
 template <class Epi>
 constexpr int pair_stages() {
-  constexpr int budget = 232448 - 1024 - 256 - GemmSmem<256, 1, true, Epi>::kEpiBytes;
+  constexpr int budget = 232448 - 1024 - 256 - GemmSmem<256, 1, true, Epi>::kEpiBytes -
+                         GemmSmem<256, 1, true, Epi>::kXchgBytes;
   constexpr int st = budget / (2 * kBM * kBK * 2);
   return st > 8 ? 8 : st;
 }
@@ -1216,7 +1232,9 @@ coda_status_t coda_gemm_res_partialrms_fp8(const uint8_t* x8, const float* sx, c
   using Epi = EpiLoadStore2<2>;
   GemmParams<Epi> p{};
   bool ok = tmap2d_u8(&p.tmA, x8, K, M, K, 128, kBM) && tmap2d_u8(&p.tmB, Wt8, K, N, K, 128, 128) &&
-            tmap2d_u8(&p.ep.tmOut2, hg8_out, N, M, N, 128, 32);
+            tmap2d_u8(&p.tmBh, Wt8, K, N, K, 128, 64) && tmap2d_u8(&p.ep.tmOut2, hg8_out, N, M, N, 128, 32) &&
+            tmap2d_u8_plain(&p.ep.tmOut2h, hg8_out, N, M, N, 64, 32);
+  p.has_bh = 1;
   if (h_out) ok = ok && map_out_bf16(&p.ep.tmOut1, h_out, M, N, N);
   if (!ok) return CODA_ERR_INTERNAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

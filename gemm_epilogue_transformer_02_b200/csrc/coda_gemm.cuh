@@ -159,6 +159,12 @@ struct TileCtx {
   int cbeg = 0, cend = 256;
   bool split = false;
   int half = 0;
+  // With eight warps, a half-tile unit gives each warp 64 of a partial slot's
+  // 128 columns: the second warp of a lane quarter hands its row sums to the
+  // first through `xchg` (32 floats) behind the single-use mbarrier `xbar`
+  // (a CTA pair runs at most one half-tile unit).  Null otherwise.
+  float* xchg = nullptr;
+  uint64_t* xbar = nullptr;
 };
 
 template <int BN, int STAGES, bool PAIR, class Epi>
@@ -168,9 +174,11 @@ struct GemmSmem {
   static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * kBK * 2;    // this CTA's columns of B
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kEpiBytes = kEW * Epi::kSmemPerWarp;
-  static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1 + kEW * Epi::kBarsPerWarp;
+  static constexpr bool kHalfXchg = kEW == 8 && epi_split<Epi>::value;  // see TileCtx::xchg
+  static constexpr int kXchgBytes = kHalfXchg ? 4 * 32 * 4 : 0;
+  static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1 + kEW * Epi::kBarsPerWarp + (kHalfXchg ? 4 : 0);
   static constexpr int kBytes =
-      1024 /*align slack*/ + STAGES * kStageBytes + kEpiBytes + kNumBars * 8 + 16;
+      1024 /*align slack*/ + STAGES * kStageBytes + kEpiBytes + kXchgBytes + kNumBars * 8 + 16;
   static_assert(kEW == 4 || kEW == 8, "four or eight epilogue warps");
   static_assert(Epi::kSmemPerWarp % 1024 == 0, "per-warp epilogue buffers keep the 128-byte swizzle alignment");
 };
@@ -203,20 +211,22 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
   constexpr int kKb = kF8 ? 2 * kBK : kBK;       // K elements per k-block (128 bytes per row)
   static_assert(!kF8 || (!A_MN && !B_MN && PAIR), "e4m3 operands: K-major A and B, CTA pairs");
   constexpr bool kSplit = epi_split<Epi>::value;
-  static_assert(!kSplit || (PAIR && !kF8 && !Epi::kPairedB), "half tiles: bf16 CTA pairs, unpaired B");
+  static_assert(!kSplit || (PAIR && !Epi::kPairedB), "half tiles: CTA pairs, unpaired B");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * S::kABytes;
   uint8_t* sEpi = smem + STAGES * S::kStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + S::kEpiBytes);
+  float* sXchg = reinterpret_cast<float*>(sEpi + S::kEpiBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + S::kEpiBytes + S::kXchgBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* ebars = drain + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ebars + kEW * Epi::kBarsPerWarp);
+  uint64_t* xbars = ebars + kEW * Epi::kBarsPerWarp;  // kHalfXchg: one per lane quarter
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(xbars + (S::kHalfXchg ? 4 : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -236,6 +246,8 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
     }
     mbar_init(drain, 1);
     for (int i = 0; i < kEW * Epi::kBarsPerWarp; ++i) mbar_init(&ebars[i], 1);
+    if (S::kHalfXchg)
+      for (int i = 0; i < 4; ++i) mbar_init(&xbars[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -367,7 +379,8 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0 && rank == 0) {
       constexpr uint32_t kIdesc = kF8 ? idesc_e4m3_f32(kTileM, BN) : idesc_bf16_f32(kTileM, BN, A_MN, B_MN);
-      constexpr uint32_t kIdescH = idesc_bf16_f32(kTileM, BN / 2, A_MN, B_MN);  // a half tile: N = BN / 2
+      // a half tile: N = BN / 2
+      constexpr uint32_t kIdescH = kF8 ? idesc_e4m3_f32(kTileM, BN / 2) : idesc_bf16_f32(kTileM, BN / 2, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -400,7 +413,7 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
             const uint64_t bd = B_MN ? sdesc_sw128(b0 + kk * 16 * 128, 64 * kBK * 2, 1024)
                                      : sdesc_sw128(b0 + kk * 32, 16, 1024);
             if (kF8)
-              tc_mma_f8_pair(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+              tc_mma_f8_pair(d, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
             else if (PAIR)
               tc_mma_bf16_pair(d, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
             else
@@ -478,6 +491,10 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
         // range (with eight warps, 64 of them per warp)
         c.cbeg = half_t * (BN / 2) + (kEW == 8 ? half * (BN / 4) : 0);
         c.cend = c.cbeg + (kEW == 8 ? BN / 4 : BN / 2);
+        if (S::kHalfXchg) {
+          c.xchg = sXchg + q * 32;
+          c.xbar = &xbars[q];
+        }
       }
       const bool ok = Epi::template tile<BN>(p.ep, c, st, w);
       tc_fence_before();
@@ -556,13 +573,15 @@ struct EpiLoadStore2 {
   static constexpr int kWarps = MODE == 2 ? 8 : 4;
   static constexpr int kBarsPerWarp = 0;
   static constexpr bool kPairedB = false;
-  // bf16 modes take half tiles (the split last wave); the e4m3 mode keeps
-  // whole tiles (its eight warps already halve each tile's columns)
-  static constexpr bool kSplitN = MODE != 2;
+  // Every mode takes half tiles (the split last wave).  In the e4m3 mode a
+  // half tile gives each of its eight warps 64 columns, whose codes are
+  // staged as plain 64-byte rows and stored through tmOut2h.
+  static constexpr bool kSplitN = true;
 
   struct Params {
     CUtensorMap tmOut1;          // [M, N] bf16, box 64 x 32
     CUtensorMap tmOut2;          // [M, N] bf16 box 64 x 32 (MODE 0) or fp32 box 32 x 32 (MODE 1)
+    CUtensorMap tmOut2h;         // MODE 2: [M, N] e4m3, box 64 x 32, no swizzle (a warp's 64 columns of a half tile)
     const __nv_bfloat16* in;     // [M, N]: res (MODE 0, may be null) or hg (MODE 1)
     const __nv_bfloat16* gamma;  // MODE 0 (may be null when out2 is not stored)
     const float* r;              // MODE 1
@@ -597,7 +616,7 @@ struct EpiLoadStore2 {
   }
 
   template <int BN>
-  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx&) {
+  __device__ static bool tile(const Params& ep, const TileCtx& c, State& st, const WaitCtx& w) {
     static_assert(BN == 256, "partials are kept per 128-column half of a 256-column tile");
     const int col0 = c.nb * BN + c.cbeg;  // first column of this warp's share of the tile
     const int row = c.row0 + c.lane;
@@ -681,9 +700,13 @@ struct EpiLoadStore2 {
             q[e] = pack_e4m3x2(g0 * inv_s, g1 * inv_s);
           }
           // 8 codes per j; two j make one 16-byte unit of the 128-column e4m3 row
+          // (of a plain 64-column row when the warp covers 64 columns)
           const uint32_t lo = q[0] | (q[1] << 16), hi = q[2] | (q[3] << 16);
           if (j & 1) {
-            st_shared_v4(G + sw128_off(c.lane, (ch & 1) * 4 + (j >> 1)), make_uint4(q8lo, q8hi, lo, hi));
+            if (c.cend - c.cbeg == 64)
+              st_shared_v4(G + c.lane * 64 + (j >> 1) * 16, make_uint4(q8lo, q8hi, lo, hi));
+            else
+              st_shared_v4(G + sw128_off(c.lane, (ch & 1) * 4 + (j >> 1)), make_uint4(q8lo, q8hi, lo, hi));
           } else {
             q8lo = lo;
             q8hi = hi;
@@ -736,8 +759,12 @@ struct EpiLoadStore2 {
         if (ep.has_out1) tma_store_2d(&ep.tmOut1, R, cc, c.row0);
         if (ep.has_out2) {
           if (MODE == 2) {
-            // the e4m3 row holds two chunks: store after the odd one (or a lone last one)
-            if ((ch & 1) || ch + 1 == nch) tma_store_2d(&ep.tmOut2, G, col0 + (ch & ~1) * 64, c.row0);
+            // the e4m3 row holds two chunks: store after the odd one (or a lone last one);
+            // a warp's 64 columns of a half tile go out as their own 64-byte rows
+            if (c.cend - c.cbeg == 64)
+              tma_store_2d(&ep.tmOut2h, G, col0, c.row0);
+            else if ((ch & 1) || ch + 1 == nch)
+              tma_store_2d(&ep.tmOut2, G, col0 + (ch & ~1) * 64, c.row0);
           } else {
             tma_store_2d(&ep.tmOut2, G, cc, c.row0);
             if (MODE == 1 && cc + 32 < c.N) tma_store_2d(&ep.tmOut2, G + 4096, cc + 32, c.row0);
@@ -755,7 +782,21 @@ struct EpiLoadStore2 {
     // slot 2 nb + 1 its second half (when it starts inside N).  Whichever warp,
     // or half-tile unit, covers a half writes its slot, so halves computed by
     // different warps or CTA pairs need no hand-over.
-    if (ep.partial != nullptr && row < c.M) {
+    if (c.xchg != nullptr) {
+      // a half tile over eight warps: this warp holds 64 of its slot's 128
+      // columns; the second warp of the lane quarter hands its sums to the first
+      const float mine = ss_lo + ss_hi;  // one of the two is zero
+      const int slot = 2 * c.nb + (c.cbeg >= BN / 2 ? 1 : 0);
+      if (c.half == 1) {
+        c.xchg[c.lane] = mine;
+        __syncwarp();
+        if (c.lane == 0) mbar_arrive(c.xbar);
+      } else {
+        if (!__all_sync(0xffffffffu, mbar_wait(c.xbar, 0u, w))) return false;
+        if (ep.partial != nullptr && row < c.M && slot * (BN / 2) < c.N)
+          ep.partial[static_cast<size_t>(slot) * c.M + row] = mine + c.xchg[c.lane];
+      }
+    } else if (ep.partial != nullptr && row < c.M) {
       const int s0 = 2 * c.nb;
       if (c.cbeg < BN / 2) ep.partial[static_cast<size_t>(s0) * c.M + row] = ss_lo;
       if (c.cend > BN / 2 && (s0 + 1) * (BN / 2) < c.N) ep.partial[static_cast<size_t>(s0 + 1) * c.M + row] = ss_hi;
@@ -814,8 +855,20 @@ struct EpiRowScale {
       if (row < c.M) {
         float sum = 0.f;
         // coherent (L2) loads: in the one-launch block the partials are written
-        // by other CTAs of the same kernel
-        for (int t = 0; t < ep.T; ++t) sum += __ldcg(ep.partial + static_cast<size_t>(t) * c.M + row);
+        // by other CTAs of the same kernel.  Up to 16 slots are requested
+        // together and then added in slot order (the order of the standalone
+        // reduction kernel, so both give the same r).
+        const float* pp = ep.partial + row;
+        if (ep.T <= 16) {
+          float pv[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) pv[t] = t < ep.T ? __ldcg(pp + static_cast<size_t>(t) * c.M) : 0.f;
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            if (t < ep.T) sum += pv[t];
+        } else {
+          for (int t = 0; t < ep.T; ++t) sum += __ldcg(pp + static_cast<size_t>(t) * c.M);
+        }
         rs = rsqrtf(sum * ep.inv_n + ep.eps);
         if (ep.r_out != nullptr && c.nb == 0 && c.cbeg == 0) ep.r_out[row] = rs;
       }

@@ -13,7 +13,7 @@
 namespace coda {
 
 // r_i = 1 / sqrt(sum_t partial[t, i] / N + eps).  One thread per row; the
-// partials of a column tile are contiguous over rows, so loads coalesce.
+// partials of a column slot are contiguous over rows, so loads coalesce.
 __global__ void rms_reduce_kernel(const float* __restrict__ partial, int M, int T, float inv_n, float eps,
                                   float* __restrict__ r) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;

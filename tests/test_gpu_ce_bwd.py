@@ -73,14 +73,14 @@ def test_lmhead_ce_bwd_fullsize_sampled():
 
 def test_lmhead_ce_bwd_repeated_labels_and_determinism():
     """Many tokens share a few labels, placed on both sides of 256-column
-    bucket and 4096-column chunk boundaries; two tokens carry labels outside
+    bucket and 8192-column chunk boundaries; two tokens carry labels outside
     [0, V) (no onehot term).  Every dW label column sums its tokens' exact
     label entries in a fixed order, so two calls agree bit for bit."""
-    M, K, V = 300, 136, 5000
+    M, K, V = 300, 136, 9000
     g = synth.make_gen(650)
     H = synth.normal_bf16(g, (M, K))
     W = synth.normal_bf16(g, (K, V), std=1.5 / math.sqrt(K))
-    pool = torch.tensor([0, 1, 255, 256, 4095, 4096, 4999], dtype=torch.int64)
+    pool = torch.tensor([0, 1, 255, 256, 8191, 8192, 8999], dtype=torch.int64)
     labels = pool[torch.randint(0, len(pool), (M,), generator=g)]
     Hd, Wd, Ld = dev(H), dev(W), dev(labels)
     _, lse, _ = C.lmhead_ce(Hd, Wd, Ld)  # lse of every token (labels do not enter it)
