@@ -797,9 +797,11 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
         kloop("gemm_swiglu_bwd (d_act GEMM + SwiGLU backward)", "coda_gemm_swiglu_bwd",
               lambda: C.gemm_swiglu_bwd(d_h2, W_down, gu, out=d_gu), f_swb,
               2 * (M * D + F * D + 2 * M * 2 * F))
-        kloop("gemm_res_partialrms_bwd (SwiGLU MLP d_y + dW_gu, grouped)", "coda_gemm_res_partialrms_bwd",
+        # d_y and dW_gu: two launches here (the grouped launch is taken only when
+        # the weight gradient is the longer product)
+        kloop("gemm_res_partialrms_bwd (SwiGLU MLP d_y + dW_gu)", "coda_gemm_res_partialrms_bwd",
               lambda: C.gemm_res_partialrms_bwd(d_gu, hg, W2), 2 * 2.0 * M * D * N2,
-              2 * (2 * M * N2 + M * D + D * N2 + M * D) + 4 * D * N2)
+              2 * (2 * M * N2 + M * D + D * N2 + M * D) + 4 * D * N2, launches=2)
         kloop("gemm_res_partialrms_bwd (SwiGLU MLP dW_down)", "coda_gemm_res_partialrms_bwd",
               lambda: C.gemm_res_partialrms_bwd(d_h2, act, W_down, dx=False), 2.0 * M * F * D,
               2 * (M * F + M * D) + 4 * F * D)
