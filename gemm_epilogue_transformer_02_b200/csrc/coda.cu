@@ -905,16 +905,14 @@ coda_status_t coda_lmhead_ce_bwd(const uint16_t* H, const uint16_t* W, const int
             map_out_f32_ld(&p.ep0.tmOut, dW_out + c0, K, vc, V) && map_a(&p.tmA[1], G, false, M, vc) &&
             map_b(&p.tmB[1], W + c0, false, K, vc, V, 128) && map_out_f32(&p.ep1.tmOut, dH_out, M, K)))
         return CODA_ERR_INTERNAL;
-      p.ep0.accum = nullptr;
-      p.ep0.ld = V;
+      p.ep0.add_to_out = 0;
       p.ep0.fix_resid = resid;
       p.ep0.fix_col0 = c0;
       p.ep0.fix_start = start;
       p.ep0.fix_entries = entries;
       p.ep0.fix_H = reinterpret_cast<const __nv_bfloat16*>(H);
       p.ep0.fix_tile0 = static_cast<int>(c0 / kLabelTile);
-      p.ep1.accum = c0 == 0 ? nullptr : dH_out;
-      p.ep1.ld = K;
+      p.ep1.add_to_out = c0 == 0 ? 0 : 1;  // dH: the first chunk stores, the others add in L2
       const GroupedProblem pb[2] = {
           {static_cast<int>(K), static_cast<int>(vc), static_cast<int>(M), raster_group(K, vc, M), true, true},
           {static_cast<int>(M), static_cast<int>(K), static_cast<int>(vc), raster_group(M, K, vc), false, false}};

@@ -933,8 +933,7 @@ struct EpiStoreF32 {
 
   struct Params {
     CUtensorMap tmOut;   // [M, N] fp32, box 32 x 32
-    const float* accum;  // null, or the output itself: out = acc + out (accumulation over calls)
-    long long ld;        // row stride (elements) of `accum`
+    int add_to_out;      // 1: out += acc (accumulation over calls, a TMA reduce-add); 0: out = acc
     const float* fix_resid;            // [tokens] label-entry residuals
     long long fix_col0;                // vocabulary index of this chunk's column 0
     const int* fix_start;              // [tiles + 1] bucket offsets, or null (no correction)
@@ -985,30 +984,12 @@ struct EpiStoreF32 {
     if (e0 < e1) fetch_batch(e0);
     for (int ch = 0; ch < nch; ++ch) {
       const int cc = col0 + ch * 32;
-      uint4 old[8];
-      if (ep.accum != nullptr) {
-        const float* src = ep.accum + static_cast<size_t>(row < c.M ? row : 0) * ep.ld + cc;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          old[j] = make_uint4(0, 0, 0, 0);
-          if (row < c.M && cc + 4 * j < c.N) old[j] = *reinterpret_cast<const uint4*>(src + 4 * j);
-        }
-      }
       uint8_t* O = c.wsmem + (st.cnt & 1) * 4096;
       if (c.lane == 0) bulk_wait_read<1>();
       __syncwarp();
       uint32_t v[32];
       tmem_ld32(c.taddr + c.cbeg + ch * 32, v);
       tmem_ld_wait(v);
-      if (ep.accum != nullptr) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + __uint_as_float(old[j].x));
-          v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + __uint_as_float(old[j].y));
-          v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + __uint_as_float(old[j].z));
-          v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + __uint_as_float(old[j].w));
-        }
-      }
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         st_shared_v4(O + sw128_off(c.lane, j), make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
@@ -1036,7 +1017,12 @@ struct EpiStoreF32 {
       fence_async_smem();
       __syncwarp();
       if (c.lane == 0) {
-        if (c.row0 < c.M) tma_store_2d(&ep.tmOut, O, cc, c.row0);
+        if (c.row0 < c.M) {
+          if (ep.add_to_out)
+            tma_reduce_add_2d(&ep.tmOut, O, cc, c.row0);
+          else
+            tma_store_2d(&ep.tmOut, O, cc, c.row0);
+        }
         bulk_commit();
       }
       ++st.cnt;

@@ -237,8 +237,9 @@ size_t coda_lmhead_ce_bwd_workspace_size(int64_t M, int64_t V);
  *   dH_out = G W^T  [M, K] fp32;   dW_out = H^T G  [K, V] fp32.
  * The vocabulary is processed in chunks of 8192 columns: a GEMM recomputes the
  * chunk's logits and its epilogue writes G_chunk (bf16, in the workspace;
- * the logits are never stored), then dH += G_chunk W_chunk^T and
- * dW_chunk = H^T G_chunk run as one grouped launch.  The label entry d_i (p - 1) dominates its dW
+ * the logits are never stored), then dH += G_chunk W_chunk^T (the first
+ * chunk stores, later chunks add in fp32 through TMA reduce-adds, in chunk
+ * order) and dW_chunk = H^T G_chunk run as one grouped launch.  The label entry d_i (p - 1) dominates its dW
  * column, so the part of it that bf16 drops is kept in fp32 and added back:
  * into dW in the dW GEMM's epilogue (rows bucketed by label beforehand; each
  * dW column sums its rows in increasing row order, so the result is
