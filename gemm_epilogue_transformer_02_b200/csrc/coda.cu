@@ -185,7 +185,7 @@ enum KernelKind : uint32_t {
 // bf16 gradient (M x 8192) is written once and read by two GEMMs right after.
 // (Interleaved on one B200 at 8192 x 2048 x 128256: 2048 columns 12.4 ms,
 // 4096 10.9, 8192 10.5, 16384 10.8: wider chunks halve the launches and the
-// fp32 dH read-modify-writes; 16384-column gradients no longer fit in L2.)
+// fp32 dH accumulations; 16384-column gradients no longer fit in L2.)
 constexpr int64_t kCEBwdChunk = 8192;
 
 // Pipeline depth of the pair kernels: as many 32 KB stages (this CTA's halves
