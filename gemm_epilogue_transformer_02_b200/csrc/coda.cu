@@ -202,13 +202,22 @@ constexpr int pair_stages() {
 // that stays resident in L2, so that the other operand streams from DRAM once:
 //   A (M x K) no larger than B (K x N): every M tile of a column block runs
 //     before the next column block (group = all rows): A stays resident and
-//     each column block of B is read once;
+//     each column block of B is read once.  An A of more than 40 MiB (bf16)
+//     does not stay in L2 (126 MB) beside B's column blocks and the output
+//     streaming through it; then the M tiles go in groups whose rows of A
+//     take 32 MiB, each group sweeping all column blocks (B is read once per
+//     group).  At hidden 4096 (A 64 MiB) the second GEMM took 1210 against
+//     1292 us that way, at hidden 8192 (128 MiB) the first 731 against 777
+//     and the second 6925 against 7053 us;
 //   otherwise row-major order (group = 1): B stays resident and each row
 //     block of A is read once.
 constexpr int kAllRows = 1 << 30;
 
 inline int raster_group(int64_t M, int64_t N, int64_t K) {
-  return (M * K <= N * K) ? kAllRows : 1;
+  if (M * K > N * K) return 1;
+  if (M * K * 2 <= (int64_t(40) << 20)) return kAllRows;
+  const int64_t g = (int64_t(32) << 20) / (2 * kBM * K * 2);  // rows of A per pair tile: 2 kBM
+  return g < 1 ? 1 : static_cast<int>(g);
 }
 
 struct KernelCache {
