@@ -281,7 +281,7 @@ coda_status_t run_gemm(int dev, DevInfo* info, GemmParams<Epi>& p, int M, int N,
   // tile-times; the 68 halves take about half of one.  (A grid of fewer
   // tiles than pairs is one such wave: all of its tiles are halved.)
   p.sched.nsplit = 0;
-  if (epi_split<Epi>::value && (B_MN || p.has_bh) && !p.no_split) {
+  if (epi_split<Epi>::value && (B_MN || p.has_bh)) {
     const int last = p.sched.ntiles % kc.max_clusters;
     if (last > 0 && 2 * last <= kc.max_clusters) p.sched.nsplit = last;
   }
@@ -732,7 +732,6 @@ coda_status_t coda_gemm_qkv_rope(const uint16_t* x, const uint16_t* W_qkv, const
     return CODA_ERR_INTERNAL;
   p.ep.positions = positions;
   p.ep.head_dim = static_cast<int>(head_dim);
-  p.no_split = head_dim != 64;  // a warp's share of a half tile (64 columns) must hold whole heads
   p.ep.rope_cols = static_cast<int>(rope_cols);
   // The angle of frequency i in turns, theta^(-2i/head_dim) / (2 pi) < 1, as a
   // 64-bit fraction (ldexp by 64 stays below 2^64; the conversion drops less

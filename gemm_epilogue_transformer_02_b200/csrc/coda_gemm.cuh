@@ -128,7 +128,6 @@ struct GemmParams {
   CUtensorMap tmB2;  // second half of a paired B operand (SwiGLU up columns)
   CUtensorMap tmBh;  // K-major B with a 64-row box: this CTA's columns of a half tile
   int has_bh;        // tmBh is encoded (a K-major B may then be split into half tiles)
-  int no_split;      // the caller rules out half tiles for this launch
   typename Epi::Params ep;
   int M, N, K;       // GEMM sizes; N counts accumulator columns of the output space
   TileSched sched;
@@ -1353,13 +1352,12 @@ struct EpiCE {
 // so the staging takes 8 KB per warp and the mainloop keeps six stages.
 // ---------------------------------------------------------------------------
 struct EpiRope {
-  // Eight warps, two per lane quarter, each taking half of the tile's columns
-  // (whole heads: 128 columns are two heads of 64 or one of 128).  With
-  // 128-wide heads this is 6 % faster than four warps; with 64-wide heads the
-  // two take the same time.  Half tiles (the split last wave) give each warp
-  // 64 columns: one whole head when heads are 64 wide; the host splits only
-  // then.
-  static constexpr int kWarps = 8;
+  // Four warps, each taking all the tile's columns (four heads of 64 or two
+  // of 128), which leaves the mainloop a sixth stage: on the 1B QKV
+  // projection 80.5 against 84.7 us with eight warps (64-wide heads), 88.4
+  // against 92.1 us with 128-wide heads.  A half tile (the split last wave)
+  // gives each warp 128 columns, whole heads either way.
+  static constexpr int kWarps = 4;
   static constexpr int kSmemPerWarp = 8192;  // two 64-column x 32-row bf16 boxes
   static constexpr int kBarsPerWarp = 0;
   static constexpr bool kPairedB = false;
