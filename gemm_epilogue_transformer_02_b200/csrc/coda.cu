@@ -166,6 +166,7 @@ enum KernelKind : uint32_t {
   kKindRowScale,
   kKindRowScaleKK,
   kKindSwiGLU,
+  kKindSwiGLUAct,     // the SwiGLU GEMM without the gate/up save
   kKindCE,
   kKindBwdP,
   kKindF32MN,
@@ -417,6 +418,25 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 size_t ce_ws_bytes(int64_t M, int64_t V) {
   const int64_t n_nt = (V + 255) / 256;
   return 2 * align256(static_cast<size_t>(n_nt) * M * 4) + align256(static_cast<size_t>(M) * 4);
+}
+
+// The SwiGLU GEMM with (EpiSwiGLU) or without (EpiSwiGLUAct) the gate/up save.
+template <class Epi>
+coda_status_t run_swiglu(int dev, DevInfo* info, const uint16_t* A, const uint16_t* W_gu, const float* r,
+                         uint16_t* act_out, uint16_t* gateup_save, int64_t M, int64_t F, int64_t K,
+                         KernelKind kind, cudaStream_t stream) {
+  GemmParams<Epi> p{};
+  bool ok = map_a(&p.tmA, A, false, M, K) && map_b(&p.tmB, W_gu, true, F, K, 2 * F, 128) &&
+            map_b(&p.tmB2, W_gu + F, true, F, K, 2 * F, 128) && map_out_bf16(&p.ep.tmAct, act_out, M, F, F);
+  if (gateup_save)
+    ok = ok && map_out_bf16(&p.ep.tmSaveG, gateup_save, M, F, 2 * F) &&
+         map_out_bf16(&p.ep.tmSaveU, gateup_save + F, M, F, 2 * F);
+  if (!ok) return CODA_ERR_INTERNAL;
+  p.ep.r = r;
+  const int n_nt = static_cast<int>((F + 127) / 128);
+  return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(F),
+                                                                    static_cast<int>(K), n_nt, raster_group(M, 2 * F, K),
+                                                                    kind, stream);
 }
 
 }  // namespace
@@ -694,19 +714,10 @@ coda_status_t coda_gemm_swiglu(const uint16_t* A, const uint16_t* W_gu, const fl
     const coda_status_t ds = current_device(&dev, &info);
     if (ds != CODA_OK) return ds;
   }
-  using Epi = EpiSwiGLU;
-  GemmParams<Epi> p{};
-  bool ok = map_a(&p.tmA, A, false, M, K) && map_b(&p.tmB, W_gu, true, F, K, 2 * F, 128) &&
-            map_b(&p.tmB2, W_gu + F, true, F, K, 2 * F, 128) && map_out_bf16(&p.ep.tmAct, act_out, M, F, F);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (gateup_save)
-    ok = ok && map_out_bf16(&p.ep.tmSaveG, gateup_save, M, F, 2 * F) &&
-         map_out_bf16(&p.ep.tmSaveU, gateup_save + F, M, F, 2 * F);
-  if (!ok) return CODA_ERR_INTERNAL;
-  p.ep.r = r;
-  p.ep.has_save = gateup_save != nullptr;
-  const int n_nt = static_cast<int>((F + 127) / 128);
-  return run_gemm<256, pair_stages<Epi>(), false, true, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(F), static_cast<int>(K), n_nt,
-      raster_group(M, 2 * F, K), kKindSwiGLU, static_cast<cudaStream_t>(stream));
+    return run_swiglu<EpiSwiGLU>(dev, info, A, W_gu, r, act_out, gateup_save, M, F, K, kKindSwiGLU, s);
+  return run_swiglu<EpiSwiGLUAct>(dev, info, A, W_gu, r, act_out, nullptr, M, F, K, kKindSwiGLUAct, s);
 }
 
 coda_status_t coda_gemm_qkv_rope(const uint16_t* x, const uint16_t* W_qkv, const int32_t* positions, uint16_t* out,

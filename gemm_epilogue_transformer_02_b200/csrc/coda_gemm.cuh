@@ -1042,8 +1042,12 @@ struct EpiStoreF32 {
 //   g = r * acc_gate, u = r * acc_up, act = silu(g) * u;
 //   optionally g and u (bf16) are saved for the backward.
 // ---------------------------------------------------------------------------
-struct EpiSwiGLU {
-  static constexpr int kSmemPerWarp = 2 * 4096 + 8192;  // act double buffer + gate/up save buffer
+// kSave: gate and up are also kept (for the backward).  Without them the
+// epilogue needs only the act double buffer, which leaves the mainloop a
+// sixth stage.
+template <bool kSave>
+struct EpiSwiGLUT {
+  static constexpr int kSmemPerWarp = kSave ? 2 * 4096 + 8192 : 2 * 4096;  // act double buffer (+ save buffer)
   static constexpr int kBarsPerWarp = 0;
   static constexpr bool kPairedB = true;
 
@@ -1052,7 +1056,6 @@ struct EpiSwiGLU {
     CUtensorMap tmSaveG;  // gate view of the [M, 2F] save tensor, box 64 x 32
     CUtensorMap tmSaveU;  // up view of the [M, 2F] save tensor, box 64 x 32
     const float* r;       // [M] or null
-    int has_save;
   };
   struct State {
     uint32_t cnt;
@@ -1070,7 +1073,7 @@ struct EpiSwiGLU {
     if (nch > kHalf / 64) nch = kHalf / 64;
     float rs = 1.f;
     if (ep.r != nullptr) rs = (row < c.M) ? __ldg(ep.r + row) : 0.f;
-    const bool save = ep.has_save != 0;
+    constexpr bool save = kSave;
     uint8_t* SG = c.wsmem + 2 * 4096;
     uint8_t* SU = SG + 4096;
     for (int ch = 0; ch < nch; ++ch) {
@@ -1131,6 +1134,8 @@ struct EpiSwiGLU {
     __syncwarp();
   }
 };
+using EpiSwiGLU = EpiSwiGLUT<true>;     // act, gate and up
+using EpiSwiGLUAct = EpiSwiGLUT<false>;  // act only
 
 // ---------------------------------------------------------------------------
 // SwiGLU backward in the down projection's dA GEMM: acc = d_act = d_out W_down^T
