@@ -135,6 +135,11 @@ def test_swiglu_and_its_backward():
     act, gu = Guarded((M, F), BF), Guarded((M, 2 * F), BF)
     _ok(lib.coda_gemm_swiglu(_p(A), _p(Wgu), _p(r), act.ptr(), gu.ptr(), M, F, K, _s()))
     _all_intact(act=act, gateup=gu)
+    act_only = Guarded((M, F), BF)  # the act-only kernel (no gate/up save)
+    _ok(lib.coda_gemm_swiglu(_p(A), _p(Wgu), _p(r), act_only.ptr(), None, M, F, K, _s()))
+    _all_intact(act_only=act_only)
+    torch.cuda.synchronize()
+    assert torch.equal(act_only.t, act.t)
     d_out = synth.normal_bf16(g, (M, N)).cuda()
     W_down = synth.normal_bf16(g, (F, N), std=1 / math.sqrt(N)).cuda()
     dgu = Guarded((M, 2 * F), BF)

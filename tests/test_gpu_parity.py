@@ -166,6 +166,10 @@ def test_gemm_swiglu(M, K, F):
     check("up", gu[:, F:], ref["up"])
     act2, _ = C.gemm_swiglu(dev(A), dev(Wgu), None)
     check("act(no r)", act2, O.gemm_swiglu(b(A), b(Wgu), None)["act"])
+    # without the save the call runs its own kernel (no save buffers, one more
+    # pipeline stage): the same arithmetic, so the same bits
+    act3, gu3 = C.gemm_swiglu(dev(A), dev(Wgu), dev(r))
+    assert gu3 is None and torch.equal(act3, act)
 
 
 def test_swiglu_down_chain():
