@@ -307,6 +307,13 @@ __global__ void __launch_bounds__(kThreads, 1) coda_gemm_grouped_kernel(const __
       const uint32_t aph = (i >> 1) & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], aph, w))) break;
       tc_fence_after();
+      if (prob == 1 && i == mine.nl && i > 0) {
+        // the staging buffers change owners: each epilogue alternates its two
+        // buffers by its own count, so the second one's first buffer may be
+        // the one the first one's last store is still reading
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+      }
       TileCtx c;
       c.M = p.M[prob];
       c.N = p.N[prob];
