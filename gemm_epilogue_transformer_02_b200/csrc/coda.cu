@@ -2,6 +2,7 @@
 // include/coda.h).  Host side: argument validation (before any CUDA call),
 // tensor-map encoding, and launches on the caller's stream.  The library keeps
 // no device allocations of its own.
+#include <algorithm>
 #include <mutex>
 
 #include <cmath>
@@ -228,9 +229,27 @@ struct KernelCache {
 KernelCache g_kcache[64][32];
 static_assert(kKindCount <= 32, "kernel kinds fit the cache");
 
+// An output that K-half units add into (TileSched::kmode): the host zeroes
+// the part of it that the split tiles cover before the launch.  Element
+// (i, j) of the layout is at base + i * pitch + j * elem; a GEMM tile (mb, nb)
+// covers layout rows [mb * tile_rows, ...) and columns [nb * tile_cols, ...),
+// or with `transposed` rows [nb * tile_rows, ...) and columns [mb * tile_cols, ...)
+// (the per-slot row sums, [slot, row]).
+struct ZeroPlan {
+  void* base;
+  size_t pitch, elem;
+  int64_t rows, cols;
+  int tile_rows, tile_cols;
+  bool transposed;
+};
+
+// A K-split needs this many k-blocks (K >= 4096 bf16): then a half takes half
+// of a tile's mainloop, where a 128-column half tile still takes 93-96 % of it.
+constexpr int kKSplitMinKb = 64;
+
 template <int BN, int STAGES, bool A_MN, bool B_MN, bool PAIR, class Epi>
 coda_status_t run_gemm(int dev, DevInfo* info, GemmParams<Epi>& p, int M, int N, int K, int n_nt, int group_m,
-                       KernelKind kind, cudaStream_t stream) {
+                       KernelKind kind, cudaStream_t stream, const ZeroPlan* zp = nullptr, int nzp = 0) {
   auto kern = coda_gemm_kernel<BN, STAGES, A_MN, B_MN, PAIR, Epi>;
   constexpr int smem = GemmSmem<BN, STAGES, PAIR, Epi>::kBytes;
   constexpr int kTileM = PAIR ? 2 * kBM : kBM;
@@ -277,14 +296,51 @@ coda_status_t run_gemm(int dev, DevInfo* info, GemmParams<Epi>& p, int M, int N,
     return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
   }
   // A last partial wave of whole tiles that fills at most half of the CTA
-  // pairs runs as a wave of half tiles (128 columns) on twice as many pairs:
-  // e.g. 256 tiles on 74 pairs end in 34 tiles, 3.46 waves taking four
-  // tile-times; the 68 halves take about half of one.  (A grid of fewer
-  // tiles than pairs is one such wave: all of its tiles are halved.)
+  // pairs runs as a wave of half units on twice as many pairs: e.g. 256
+  // tiles on 74 pairs end in 34 tiles, 3.46 waves taking four tile-times.
+  // (A grid of fewer tiles than pairs is one such wave: all of its tiles are
+  // halved.)  Halves of the k-blocks, for epilogues whose fp32 outputs are
+  // linear in the accumulator and long K: each runs half of the tile's
+  // mainloop at full width and adds into the output zeroed here; otherwise
+  // 128-column halves, whose MMAs still take 93-96 % of a whole tile's time
+  // (they are bound by operand delivery, not by the tensor pipe).
   p.sched.nsplit = 0;
-  if (epi_split<Epi>::value && (B_MN || p.has_bh)) {
+  p.sched.kmode = 0;
+  {
     const int last = p.sched.ntiles % kc.max_clusters;
-    if (last > 0 && 2 * last <= kc.max_clusters) p.sched.nsplit = last;
+    constexpr int kKbElems = epi_fp8<Epi>::value ? 2 * kBK : kBK;
+    const int nkb = (K + kKbElems - 1) / kKbElems;
+    if (last > 0 && 2 * last <= kc.max_clusters) {
+      if (epi_ksplit<Epi>::value && nzp > 0 && nkb >= kKSplitMinKb) {
+        int mb0 = p.sched.n_mt, mb1 = -1, nb0 = n_nt, nb1 = -1;
+        for (int t = p.sched.ntiles - last; t < p.sched.ntiles; ++t) {
+          int mb, nb;
+          p.sched.map(t, mb, nb);
+          mb0 = mb < mb0 ? mb : mb0;
+          mb1 = mb > mb1 ? mb : mb1;
+          nb0 = nb < nb0 ? nb : nb0;
+          nb1 = nb > nb1 ? nb : nb1;
+        }
+        for (int i = 0; i < nzp; ++i) {
+          const ZeroPlan& z = zp[i];
+          const int a0 = z.transposed ? nb0 : mb0, a1 = z.transposed ? nb1 : mb1;
+          const int b0 = z.transposed ? mb0 : nb0, b1 = z.transposed ? mb1 : nb1;
+          const int64_t r0 = static_cast<int64_t>(a0) * z.tile_rows;
+          const int64_t r1 = std::min<int64_t>(static_cast<int64_t>(a1 + 1) * z.tile_rows, z.rows);
+          const int64_t c0 = static_cast<int64_t>(b0) * z.tile_cols;
+          const int64_t c1 = std::min<int64_t>(static_cast<int64_t>(b1 + 1) * z.tile_cols, z.cols);
+          if (r1 <= r0 || c1 <= c0) continue;
+          if (cudaMemset2DAsync(static_cast<uint8_t*>(z.base) + r0 * z.pitch + c0 * z.elem, z.pitch, 0,
+                                static_cast<size_t>(c1 - c0) * z.elem, static_cast<size_t>(r1 - r0),
+                                stream) != cudaSuccess)
+            return CODA_ERR_LAUNCH;
+        }
+        p.sched.kmode = 1;
+        p.sched.nsplit = last;
+      } else if (epi_split<Epi>::value && (B_MN || p.has_bh)) {
+        p.sched.nsplit = last;
+      }
+    }
   }
   const int units = p.sched.ntiles + p.sched.nsplit;
   const int clusters = units < kc.max_clusters ? units : kc.max_clusters;
@@ -1022,9 +1078,13 @@ coda_status_t coda_gemm_rowscale_bwd(const uint16_t* dOut, const uint16_t* hg, c
     p.ep.partial = pdr_out;
     p.ep.has_out1 = 1;
     p.ep.has_out2 = 1;
+    // a split by k-blocks adds into d_hg [M, N] and pdr [T, M]
+    const ZeroPlan zp[2] = {
+        {d_hg_out, static_cast<size_t>(N) * 4, 4, M, N, 256, 256, false},
+        {pdr_out, static_cast<size_t>(M) * 4, 4, coda_partial_cols(N), M, 2, 256, true}};
     coda_status_t st = run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M), static_cast<int>(N),
                                                            static_cast<int>(N2), static_cast<int>((N + 255) / 256),
-                                                           raster_group(M, N, N2), kKindBwdP, s);
+                                                           raster_group(M, N, N2), kKindBwdP, s, zp, 2);
     if (st != CODA_OK) return st;
   }
   {
@@ -1034,8 +1094,9 @@ coda_status_t coda_gemm_rowscale_bwd(const uint16_t* dOut, const uint16_t* hg, c
     if (!(map_a(&p.tmA, y, true, N, M) && map_b(&p.tmB, dOut, true, N2, M, N2, 128) &&
           map_out_f32(&p.ep.tmOut, dW2_out, N, N2)))
       return CODA_ERR_INTERNAL;
+    const ZeroPlan zp = {dW2_out, static_cast<size_t>(N2) * 4, 4, N, N2, 256, 256, false};
     return run_gemm<256, pair_stages<Epi>(), true, true, true, Epi>(dev, info, p, static_cast<int>(N), static_cast<int>(N2), static_cast<int>(M), static_cast<int>((N2 + 255) / 256),
-      raster_group(N, N2, M), kKindF32MN, s);
+      raster_group(N, N2, M), kKindF32MN, s, &zp, 1);
   }
 }
 
@@ -1122,8 +1183,9 @@ coda_status_t coda_gemm_res_partialrms_bwd(const uint16_t* dh, const uint16_t* x
     if (!(map_a(&p.tmA, x, true, K, M) && map_b(&p.tmB, dh, true, N, M, N, 128) &&
           map_out_f32(&p.ep.tmOut, dW1_out, K, N)))
       return CODA_ERR_INTERNAL;
+    const ZeroPlan zp = {dW1_out, static_cast<size_t>(N) * 4, 4, K, N, 256, 256, false};
     return run_gemm<256, pair_stages<Epi>(), true, true, true, Epi>(dev, info, p, static_cast<int>(K), static_cast<int>(N), static_cast<int>(M), static_cast<int>((N + 255) / 256),
-      raster_group(K, N, M), kKindF32MN, s);
+      raster_group(K, N, M), kKindF32MN, s, &zp, 1);
   }
   return CODA_OK;
 }

@@ -44,15 +44,18 @@ struct TileSched {
   int group_m;  // M tiles per raster group
   int ntiles;
   // The last `nsplit` tiles in raster order are handed out as two units each,
-  // their two 128-column halves, so that a last partial wave of whole tiles
-  // on under half of the CTA pairs becomes a wave of half tiles on all of
-  // them (0: every unit is a whole tile).
+  // so that a last partial wave of whole tiles on under half of the CTA pairs
+  // becomes a wave of half units on all of them (0: every unit is a whole
+  // tile).  kmode 0: the halves are the tile's two 128-column halves; kmode
+  // 1: they are full-width tiles over the first and the second half of the
+  // k-blocks, whose epilogues add their results into a zeroed output.
   int nsplit;
+  int kmode;
 
   __device__ __forceinline__ int nunits() const { return ntiles + nsplit; }
 
   // Unit u -> tile (mb, nb) and half (-1 for a whole tile, else 0 or 1).
-  __device__ __forceinline__ void map_unit(int u, int& mb, int& nb, int& half) const {
+  __host__ __device__ __forceinline__ void map_unit(int u, int& mb, int& nb, int& half) const {
     const int s0 = ntiles - nsplit;
     int t = u;
     half = -1;
@@ -63,11 +66,11 @@ struct TileSched {
     map(t, mb, nb);
   }
 
-  __device__ __forceinline__ void map(int t, int& mb, int& nb) const {
+  __host__ __device__ __forceinline__ void map(int t, int& mb, int& nb) const {
     const int per_group = group_m * n_nt;
     const int g = t / per_group;
     const int first = g * group_m;
-    const int gs = min(n_mt - first, group_m);
+    const int gs = n_mt - first < group_m ? n_mt - first : group_m;
     const int r = t - g * per_group;
     mb = first + r % gs;
     nb = r / gs;
@@ -108,6 +111,19 @@ struct epi_split {
 template <class E>
 struct epi_split<E, decltype(void(E::kSplitN))> {
   static constexpr bool value = E::kSplitN;
+};
+
+// Epilogues that declare kSplitK = true produce outputs linear in the
+// accumulator, in fp32 (c.khalf >= 0: they add into the output, which the
+// host has zeroed), so the split last wave may divide a tile's k-blocks
+// instead of its columns (TileSched::kmode).
+template <class E, class = void>
+struct epi_ksplit {
+  static constexpr bool value = false;
+};
+template <class E>
+struct epi_ksplit<E, decltype(void(E::kSplitK))> {
+  static constexpr bool value = E::kSplitK;
 };
 
 // Epilogues that declare kHasPre = true give their warps work to do before
@@ -156,6 +172,7 @@ struct TileCtx {
   // of it; with eight epilogue warps one half (`split`, `half`); or, for a
   // half-tile unit of the split last wave, the 128 columns it computed.
   int cbeg = 0, cend = 256;
+  int khalf = -1;  // a K-half unit (0 or 1, TileSched::kmode): add the result into the output
   bool split = false;
   int half = 0;
   // With eight warps, a half-tile unit gives each warp 64 of a partial slot's
@@ -286,11 +303,15 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
       for (int t = tile_first; ok && t < ntiles; t += tile_step) {
         int mb, nb, half;
         p.sched.map_unit(t, mb, nb, half);
+        // a K-half unit loads the whole tile's columns over its half of the k-blocks
+        const int kb_lo = (p.sched.kmode && half > 0) ? nkb / 2 : 0;
+        const int kb_hi = (p.sched.kmode && half == 0) ? nkb / 2 : nkb;
+        if (p.sched.kmode) half = -1;
         const int arow = mb * kTileM + static_cast<int>(rank) * kBM;  // first A row of this CTA
         // first B column of this CTA: a half tile covers BN/2 columns, kBCols/2 per CTA
         const int bcol = half < 0 ? nb * BN + static_cast<int>(rank) * kBCols
                                   : nb * BN + half * (BN / 2) + static_cast<int>(rank) * (kBCols / 2);
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = kb_lo; kb < kb_hi; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, w)) {
             ok = false;
             break;
@@ -388,16 +409,20 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         int half = -1;
-        if (kSplit) {
+        if (kSplit || epi_ksplit<Epi>::value) {
           int mb_, nb_;
           p.sched.map_unit(t, mb_, nb_, half);
         }
+        // a K-half unit: the whole width over its half of the k-blocks
+        const int kb_lo = (p.sched.kmode && half > 0) ? nkb / 2 : 0;
+        const int kb_hi = (p.sched.kmode && half == 0) ? nkb / 2 : nkb;
+        if (p.sched.kmode) half = -1;
         const uint32_t idesc = (kSplit && half >= 0) ? kIdescH : kIdesc;
         if (!mbar_wait(&tempty[acc], aph ^ 1u, w)) break;
         tc_fence_after();
         // a half tile accumulates into the accumulator columns it covers
         const uint32_t d = tmem_base + acc * BN + (half > 0 ? BN / 2 : 0);
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = kb_lo; kb < kb_hi; ++kb) {
           if (!mbar_wait(&full[stage], phase, w)) {
             ok = false;
             break;
@@ -411,12 +436,13 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
                                      : sdesc_sw128(a0 + kk * 32, 16, 1024);
             const uint64_t bd = B_MN ? sdesc_sw128(b0 + kk * 16 * 128, 64 * kBK * 2, 1024)
                                      : sdesc_sw128(b0 + kk * 32, 16, 1024);
+            const uint32_t accum = (kb != kb_lo || kk != 0) ? 1u : 0u;
             if (kF8)
-              tc_mma_f8_pair(d, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+              tc_mma_f8_pair(d, ad, bd, idesc, accum);
             else if (PAIR)
-              tc_mma_bf16_pair(d, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+              tc_mma_bf16_pair(d, ad, bd, idesc, accum);
             else
-              tc_mma_bf16(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+              tc_mma_bf16(d, ad, bd, kIdesc, accum);
           }
           if (PAIR)
             tc_commit_pair_mc(&empty[stage], 0x3);
@@ -479,7 +505,12 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
         int nmb, nnb, nhalf;
         p.sched.map_unit(t + tile_step, nmb, nnb, nhalf);
         c.nrow0 = nmb * kTileM + static_cast<int>(rank) * kBM + q * 32;
-        c.ncol0 = nnb * BN + (nhalf > 0 ? BN / 2 : 0);
+        c.ncol0 = nnb * BN + (nhalf > 0 && !p.sched.kmode ? BN / 2 : 0);
+      }
+      if (p.sched.kmode) {
+        // a K-half unit covers the whole tile and adds its result into the output
+        c.khalf = half_t;
+        half_t = -1;
       }
       c.split = kEW == 8;
       c.half = half;
@@ -576,6 +607,11 @@ struct EpiLoadStore2 {
   // half tile gives each of its eight warps 64 columns, whose codes are
   // staged as plain 64-byte rows and stored through tmOut2h.
   static constexpr bool kSplitN = true;
+  // MODE 1 (the P GEMM, K = the long output width) may split its last wave
+  // by k-blocks: d_hg = r P and pdr = sum hg P are linear in P, so each half
+  // adds into them (zeroed by the host); y = r hg does not depend on P and
+  // is stored by the first half.
+  static constexpr bool kSplitK = MODE == 1;
 
   struct Params {
     CUtensorMap tmOut1;          // [M, N] bf16, box 64 x 32
@@ -755,7 +791,7 @@ struct EpiLoadStore2 {
       fence_async_smem();
       __syncwarp();
       if (c.lane == 0 && rows_live) {
-        if (ep.has_out1) tma_store_2d(&ep.tmOut1, R, cc, c.row0);
+        if (ep.has_out1 && c.khalf <= 0) tma_store_2d(&ep.tmOut1, R, cc, c.row0);
         if (ep.has_out2) {
           if (MODE == 2) {
             // the e4m3 row holds two chunks: store after the odd one (or a lone last one);
@@ -764,6 +800,9 @@ struct EpiLoadStore2 {
               tma_store_2d(&ep.tmOut2h, G, col0, c.row0);
             else if ((ch & 1) || ch + 1 == nch)
               tma_store_2d(&ep.tmOut2, G, col0 + (ch & ~1) * 64, c.row0);
+          } else if (MODE == 1 && c.khalf >= 0) {
+            tma_reduce_add_2d(&ep.tmOut2, G, cc, c.row0);
+            if (cc + 32 < c.N) tma_reduce_add_2d(&ep.tmOut2, G + 4096, cc + 32, c.row0);
           } else {
             tma_store_2d(&ep.tmOut2, G, cc, c.row0);
             if (MODE == 1 && cc + 32 < c.N) tma_store_2d(&ep.tmOut2, G + 4096, cc + 32, c.row0);
@@ -797,8 +836,17 @@ struct EpiLoadStore2 {
       }
     } else if (ep.partial != nullptr && row < c.M) {
       const int s0 = 2 * c.nb;
-      if (c.cbeg < BN / 2) ep.partial[static_cast<size_t>(s0) * c.M + row] = ss_lo;
-      if (c.cend > BN / 2 && (s0 + 1) * (BN / 2) < c.N) ep.partial[static_cast<size_t>(s0 + 1) * c.M + row] = ss_hi;
+      float* p0 = ep.partial + static_cast<size_t>(s0) * c.M + row;
+      float* p1 = p0 + c.M;
+      const bool hi = c.cend > BN / 2 && (s0 + 1) * (BN / 2) < c.N;
+      if (c.khalf >= 0) {
+        // two K-halves add into a zeroed slot: 0 + a + b in either order
+        if (c.cbeg < BN / 2) atomicAdd(p0, ss_lo);
+        if (hi) atomicAdd(p1, ss_hi);
+      } else {
+        if (c.cbeg < BN / 2) *p0 = ss_lo;
+        if (hi) *p1 = ss_hi;
+      }
     }
     if (MODE == 2) {
       const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(amx));  // |hg| >= 0: bits order as values
@@ -929,6 +977,7 @@ struct EpiStoreF32 {
   static constexpr int kBarsPerWarp = 0;
   static constexpr bool kPairedB = false;
   static constexpr bool kSplitN = true;
+  static constexpr bool kSplitK = true;  // out = acc is linear: K-halves add into a zeroed output
 
   struct Params {
     CUtensorMap tmOut;   // [M, N] fp32, box 32 x 32
@@ -1017,7 +1066,7 @@ struct EpiStoreF32 {
       __syncwarp();
       if (c.lane == 0) {
         if (c.row0 < c.M) {
-          if (ep.add_to_out)
+          if (ep.add_to_out || c.khalf >= 0)
             tma_reduce_add_2d(&ep.tmOut, O, cc, c.row0);
           else
             tma_store_2d(&ep.tmOut, O, cc, c.row0);

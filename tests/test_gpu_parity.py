@@ -234,6 +234,41 @@ def test_gemm_rowscale_bwd():
     check("pdr", pdr, ref["pdr"])
 
 
+def test_gemm_rowscale_bwd_last_wave_split_by_k():
+    """P GEMM with K = 4104 (65 k-blocks): its tiles form a last partial wave,
+    which runs as two halves of the k-blocks adding d_hg and pdr into zeroed
+    outputs; the result is the oracle's and the same bits call after call."""
+    g = gen(26)
+    M, N, N2 = 300, 136, 4104
+    dOut = synth.normal_bf16(g, (M, N2), std=0.5)
+    hg = synth.normal_bf16(g, (M, N))
+    W2 = synth.normal_bf16(g, (N, N2), std=1 / math.sqrt(N))
+    r = torch.rand(M, generator=g) + 0.5
+    d_hg, dW2, pdr = C.gemm_rowscale_bwd(dev(dOut), dev(hg), dev(W2), dev(r))
+    d_hg2, dW22, pdr2 = C.gemm_rowscale_bwd(dev(dOut), dev(hg), dev(W2), dev(r))
+    assert torch.equal(d_hg, d_hg2) and torch.equal(pdr, pdr2) and torch.equal(dW2, dW22)
+    ref = O.gemm_rowscale_bwd(b(dOut), b(hg), b(W2), r.double().numpy(), C.partial_tile_width())
+    check("d_hg", d_hg, ref["d_hg"])
+    check("dW2", dW2, ref["dW2"])
+    check("pdr", pdr, ref["pdr"])
+
+
+@pytest.mark.parametrize("M,K,N", [(4171, 64, 136), (4136, 2048, 2560)])
+def test_weight_gradient_last_wave_split_by_k(M, K, N):
+    """dW1 = x^T dh over 4136-4171 tokens (65-66 k-blocks): the last partial
+    wave (every tile of the 1-tile case; 6 of 80 tiles in the other, beside
+    whole tiles) runs as halves of the k-blocks adding into zeroed rows of
+    dW1.  Oracle parity and the same bits call after call."""
+    g = gen(27 + K)
+    dh = synth.normal_bf16(g, (M, N))
+    x = synth.normal_bf16(g, (M, K))
+    W1 = synth.normal_bf16(g, (K, N), std=1 / math.sqrt(K))
+    _, dW1 = C.gemm_res_partialrms_bwd(dev(dh), dev(x), dev(W1), dx=False)
+    _, dW1b = C.gemm_res_partialrms_bwd(dev(dh), dev(x), dev(W1), dx=False)
+    assert torch.equal(dW1, dW1b)
+    check("dW1", dW1, O.matmul(b(x).T, b(dh)))
+
+
 def test_rms_reduce_bwd():
     g = gen(22)
     M, N = 300, 520
