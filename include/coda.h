@@ -276,7 +276,11 @@ size_t coda_gemm_rowscale_bwd_workspace_size(int64_t M, int64_t N);
  *   y = bf16(r * hg) (workspace);  pdr[t, i] = sum_{j in slot t} hg_ij P_ij   [T, M] fp32
  *   dW2_out = y^T dOut (fp32)                                          [N, N2]
  * dOut [M, N2] bf16, hg [M, N] bf16, W2 [N, N2] bf16, r [M] fp32.
- * d_hg and pdr feed coda_rms_reduce_bwd. */
+ * d_hg and pdr feed coda_rms_reduce_bwd.  When the tiles of a GEMM end in a
+ * partial wave on at most half of the CTA pairs and its K is 4096 or more,
+ * that wave is split by k-blocks: the call first zeroes the part of d_hg and
+ * pdr (or dW2) those tiles cover, and two units add their halves into it
+ * (in fp32; the same bits from call to call). */
 coda_status_t coda_gemm_rowscale_bwd(const uint16_t* dOut, const uint16_t* hg, const uint16_t* W2, const float* r,
                                      float* d_hg_out, float* dW2_out, float* pdr_out, void* ws, size_t ws_bytes,
                                      int64_t M, int64_t N, int64_t N2, void* stream);
@@ -317,7 +321,9 @@ coda_status_t coda_rms_reduce_bwd_noalloc(const float* pdr, const float* r, cons
  * (fp32) [K, N]; dres equals dh.  dh [M, N] bf16, x [M, K] bf16, W1 [K, N] bf16.
  * Either output may be NULL (not computed).  With both requested and M >= N
  * the two GEMMs share one persistent launch (the dW1 tiles first, the dx
- * tiles filling each CTA pair up to a common makespan); otherwise two. */
+ * tiles filling each CTA pair up to a common makespan); otherwise two, and
+ * the dW1 GEMM may split its last partial wave by k-blocks as
+ * coda_gemm_rowscale_bwd does (zeroing, then adding into, part of dW1_out). */
 coda_status_t coda_gemm_res_partialrms_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* W1,
                                            uint16_t* dx_out, float* dW1_out, int64_t M, int64_t N, int64_t K,
                                            void* stream);
