@@ -13,7 +13,7 @@ inputs resident in HBM; L2 is flushed (256 MB write) before every timed step.
 The other hot-path rows (SwiGLU + down projection and its backward, the FP8
 block beside the bf16 one, QKV + RoPE, the fused LM-head cross-entropy and its
 backward, the block backward) are timed in the same run and reported under
-"path"; ``--sweep`` adds the block at larger hidden sizes.
+"path" (with the block at hidden 4096 and 8192 under "hidden_sweep"; ``--no-sweep`` skips it).
 
 Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no
 collective on the data path); time = max over ranks of the device time.
@@ -85,8 +85,8 @@ def parse():
     ap.add_argument("--kernel-cooldown", type=float, default=1.0,
                     help="seconds the GPU idles before each per-kernel loop, so that one loop's power and heat do "
                          "not carry into the next")
-    ap.add_argument("--sweep", action="store_true",
-                    help="also time the block at hidden 4096 (gate/up 28672) and 8192 (gate/up 57344)")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the block at hidden 4096 (gate/up 28672) and 8192 (gate/up 57344)")
     return ap.parse_args()
 
 
@@ -621,7 +621,7 @@ def run_ours(args):
     if not args.no_path:
         path = time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma, h, hg, r, rank,
                          args.path_steps, timed, None if args.no_kernels else kloop)
-    if args.sweep:
+    if not args.no_sweep and not args.no_path:
         path["hidden_sweep"] = time_sweep(C, synth, torch, dev, stream, flush, rank, args.path_steps)
 
     DD.barrier()
