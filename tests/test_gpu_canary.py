@@ -223,6 +223,41 @@ def test_block_backward_calls():
     C.poll_status()
 
 
+def test_backward_gemms_split_by_k():
+    """The long-K backward GEMMs whose last wave splits by k-blocks zero part
+    of their outputs with 2-D memsets before adding into them: the guard
+    bytes around d_hg, pdr and dW1 stay intact, and the guarded call equals
+    the plain one bit for bit."""
+    lib = C.load_library()
+    M, N, N2 = 300, 136, 4104
+    g = synth.make_gen(907)
+    dOut = synth.normal_bf16(g, (M, N2), std=0.5).cuda()
+    hg = synth.normal_bf16(g, (M, N)).cuda()
+    W2 = synth.normal_bf16(g, (N, N2), std=1 / math.sqrt(N)).cuda()
+    r = (torch.rand(M, generator=g) + 0.5).cuda()
+    T = C.partial_cols(N)
+    d_hg, dW2, pdr = Guarded((M, N), F32), Guarded((N, N2), F32), Guarded((T, M), F32)
+    nb = int(lib.coda_gemm_rowscale_bwd_workspace_size(M, N))
+    ws = Guarded((nb,), U8)
+    _ok(lib.coda_gemm_rowscale_bwd(_p(dOut), _p(hg), _p(W2), _p(r), d_hg.ptr(), dW2.ptr(), pdr.ptr(), ws.ptr(), nb,
+                                   M, N, N2, _s()))
+    _all_intact(d_hg=d_hg, dW2=dW2, pdr=pdr, ws=ws)
+    d_hg0, dW20, pdr0 = C.gemm_rowscale_bwd(dOut, hg, W2, r)
+    torch.cuda.synchronize()
+    assert torch.equal(d_hg.t, d_hg0) and torch.equal(pdr.t, pdr0) and torch.equal(dW2.t, dW20)
+    Mt, K, Nw = 4171, 64, 136
+    dh = synth.normal_bf16(g, (Mt, Nw)).cuda()
+    x = synth.normal_bf16(g, (Mt, K)).cuda()
+    W1 = synth.normal_bf16(g, (K, Nw), std=1 / math.sqrt(K)).cuda()
+    dW1 = Guarded((K, Nw), F32)
+    _ok(lib.coda_gemm_res_partialrms_bwd(_p(dh), _p(x), _p(W1), None, dW1.ptr(), Mt, Nw, K, _s()))
+    _all_intact(dW1=dW1)
+    _, dW10 = C.gemm_res_partialrms_bwd(dh, x, W1, dx=False)
+    torch.cuda.synchronize()
+    assert torch.equal(dW1.t, dW10)
+    C.poll_status()
+
+
 def test_fp8_block_and_unfused_pieces():
     lib = C.load_library()
     M, K, N, N2 = 333, 272, 784, 400
