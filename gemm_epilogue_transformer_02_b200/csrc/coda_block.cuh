@@ -11,7 +11,10 @@
 //   tiles [0, n1)       first GEMM  (x W1 + res -> h, hg, partials), row-major
 //                       order so that row blocks complete early;
 //   tiles [n1, n1 + n2) second GEMM (r * (hg W2), r formed in its epilogue from
-//                       the partials), all row blocks of a column block in turn.
+//                       the partials), in groups of `group2` row blocks, each
+//                       group's row blocks for one column block after another,
+//                       so that the first second-GEMM tiles need only the first
+//                       row blocks of the first GEMM.
 //
 // Tiles are dealt round-robin to the resident clusters, so every cluster runs
 // its first-GEMM tiles before any second-GEMM tile.  A first-GEMM tile's
@@ -41,6 +44,7 @@ struct BlockParams {
   // the last nsplit second-GEMM tiles run as two 128-column halves each (a
   // last partial wave on at most half of the pairs becomes a wave of halves)
   int nsplit;
+  int group2;        // row blocks per raster group of the second GEMM
   int ready_target;  // counter value of a finished row block: n_nt1 tiles x 2 CTAs x 4 warps
   uint64_t wait_ns;
 };
@@ -65,8 +69,13 @@ __device__ __forceinline__ BlockTile block_tile(const BlockParams& p, int t) {
       u = s0 + ((u - s0) >> 1);
     }
     b.phase = 1;
-    b.nb = u / p.n_mt;
-    b.mb = u - b.nb * p.n_mt;
+    const int per_group = p.group2 * p.n_nt2;
+    const int g = u / per_group;
+    const int first = g * p.group2;
+    const int gs = p.n_mt - first < p.group2 ? p.n_mt - first : p.group2;
+    const int r = u - g * per_group;
+    b.mb = first + r % gs;
+    b.nb = r / gs;
   }
   return b;
 }
