@@ -1,0 +1,168 @@
+"""fp64 CPU oracle for the block-scaled (MXFP8) variant of the block.
+
+TEST INFRASTRUCTURE ONLY, like ``coda_oracle``: only ``tests/``,
+``__graft_entry__.smoke()`` and ``bench.py`` (its CPU legs) may use it.  It
+shares no code with the CUDA library.
+
+Source: KuCoin news flash "CODA: new research optimizes transformer training
+with GEMM epilogue programming", section "The lazy cost of training large
+models" (low precision speeds up the products while the data movement around
+them stays, so the epilogue's share grows).  The article gives no low-precision
+recipe; this module states the readings the MXFP8 variant takes (each listed in
+the design notes):
+
+* The microscaling format (the OCP "Microscaling Formats (MX)" specification,
+  v1.0): a block of 32 consecutive elements along the reduction dimension K
+  shares one power-of-two scale 2^e, stored as an E8M0 byte e + 127 (biased
+  exponent, no sign or mantissa); the elements are e4m3 codes (the codec of
+  ``coda_oracle_fp8``).  A block holds v ~ 2^e decode(q).
+* The scale exponent is the smallest e with amax(|v|) <= 448 2^e, so that no
+  element saturates; e is clamped to [-127, 127] and an all-zero block takes
+  e = 0.  (The specification's own choice, floor(log2 amax) - 8, saturates
+  elements between 448 and 512 times the scale; the smallest non-saturating
+  exponent is the reading taken here.)
+* Codes are encode(v 2^-e): round to nearest, ties to the even code.  v 2^-e
+  is exact, so the only rounding is the e4m3 one.
+* Both GEMM operands are K-major and block-scaled along K: A [M, K] with
+  scales [M, K/32], B stored as Bt [N, K] with scales [N, K/32].
+* The scales travel in a tiled byte layout (the library's header states it):
+  for 32-block j of row i, with R rows padded to whole 128-row blocks
+  (nrb = ceil(R / 128) row blocks), the byte sits at
+  ((j // 4) nrb + i // 128) 512 + (i % 32) 16 + ((i // 32) % 4) 4 + j % 4,
+  i.e. one 512-byte atom per (128-row block, 128-column block), k-blocks
+  outermost; bytes of padding rows hold 127 (scale 1).
+* The block: the first GEMM keeps the per-tensor e4m3 operands of the FP8
+  block; its epilogue forms hg = gamma h in full precision and quantises it
+  into MXFP8 itself, block by block, so hg's scales are those of the data
+  being written (no scale carried over from an earlier call).  The second
+  GEMM multiplies the block-scaled hg by a block-scaled W2 and applies the
+  row scale r of the folded light reduction.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from . import coda_oracle_fp8 as F8
+
+MX_BLOCK = 32
+E4M3_MAX = 448.0
+E_MIN, E_MAX = -127, 127
+
+
+def mx_exponent(amax) -> np.ndarray:
+    """Scale exponent of each block: the smallest integer e with
+    amax <= 448 * 2^e, clamped to [-127, 127]; 0 for amax == 0."""
+    a = np.asarray(amax, dtype=np.float64)
+    out = np.zeros(a.shape, dtype=np.int32)
+    for idx in np.ndindex(a.shape):
+        v = float(a[idx])
+        if v == 0.0:
+            continue
+        # a first guess from frexp, then step until the definition holds
+        _, ex = math.frexp(v / E4M3_MAX)
+        e = ex
+        while math.ldexp(E4M3_MAX, e) < v:
+            e += 1
+        while math.ldexp(E4M3_MAX, e - 1) >= v:
+            e -= 1
+        out[idx] = min(max(e, E_MIN), E_MAX)
+    return out
+
+
+def mx_quantize(v):
+    """MXFP8 codes and scale exponents of v [R, K] (K a multiple of 32):
+    returns (codes uint8 [R, K], exponents int32 [R, K / 32])."""
+    v = np.asarray(v, dtype=np.float64)
+    R, K = v.shape
+    assert K % MX_BLOCK == 0
+    blocks = v.reshape(R, K // MX_BLOCK, MX_BLOCK)
+    e = mx_exponent(np.abs(blocks).max(axis=2) if K else np.zeros((R, 0)))
+    scaled = blocks * np.ldexp(1.0, -e)[:, :, None]
+    codes = F8.e4m3_encode(scaled).reshape(R, K)
+    return codes, e
+
+
+def mx_dequantize(codes, exps) -> np.ndarray:
+    """fp64 values 2^e decode(q) of MXFP8 data."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    exps = np.asarray(exps, dtype=np.int64)
+    R, K = codes.shape
+    vals = F8.e4m3_decode(codes).reshape(R, K // MX_BLOCK, MX_BLOCK)
+    return (vals * np.ldexp(1.0, exps)[:, :, None]).reshape(R, K)
+
+
+def sf_rows_padded(R: int) -> int:
+    return -(-R // 128) * 128
+
+
+def sf_bytes(R: int, K: int) -> int:
+    """Size of the tiled scale buffer of an [R, K] operand."""
+    return (K // 128) * (sf_rows_padded(R) // 128) * 512
+
+
+def sf_offset(i: int, j: int, R: int) -> int:
+    """Byte offset of the scale of row i, 32-block j, in the tiled layout."""
+    nrb = sf_rows_padded(R) // 128
+    return ((j // 4) * nrb + i // 128) * 512 + (i % 32) * 16 + ((i // 32) % 4) * 4 + j % 4
+
+
+def sf_tile(exps, R: int) -> np.ndarray:
+    """Tiled E8M0 bytes of exponents [R, K/32] (padding rows: 127)."""
+    exps = np.asarray(exps, dtype=np.int64)
+    nblk = exps.shape[1]
+    assert nblk % 4 == 0
+    buf = np.full(sf_bytes(R, nblk * MX_BLOCK), 127, dtype=np.uint8)
+    for i in range(R):
+        for j in range(nblk):
+            buf[sf_offset(i, j, R)] = exps[i, j] + 127
+    return buf
+
+
+def sf_untile(buf, R: int, K: int) -> np.ndarray:
+    """Exponents [R, K/32] read back from the tiled bytes."""
+    buf = np.asarray(buf, dtype=np.uint8).reshape(-1)
+    out = np.empty((R, K // MX_BLOCK), dtype=np.int32)
+    for i in range(R):
+        for j in range(K // MX_BLOCK):
+            out[i, j] = int(buf[sf_offset(i, j, R)]) - 127
+    return out
+
+
+def gemm_res_partialrms_mx(x8, sx, W1t8, sw1, res, gamma, tile_cols: int = 256) -> dict:
+    """First GEMM of the MXFP8 block (per-tensor e4m3 operands):
+    h = (decode(x8) decode(W1t8)^T) sx sw1 + res;  partial[t, i] = sum over
+    column tile t of h^2;  hg = gamma h;  (hq, he) = mx_quantize(hg)."""
+    acc = F8.e4m3_decode(x8) @ F8.e4m3_decode(W1t8).T
+    h = acc * (np.float64(sx) * np.float64(sw1)) + np.asarray(res, dtype=np.float64)
+    M, N = h.shape
+    T = -(-N // tile_cols)
+    partial = np.zeros((T, M))
+    for t in range(T):
+        blk = h[:, t * tile_cols:(t + 1) * tile_cols]
+        partial[t] = (blk * blk).sum(axis=1)
+    hg = np.asarray(gamma, dtype=np.float64)[None, :] * h
+    hq, he = mx_quantize(hg)
+    return {"h": h, "partial": partial, "hg": hg, "hq": hq, "he": he}
+
+
+def gemm_rowscale_partial_mx(aq, ae, bq, be, partial=None, n_norm: int = 0, eps: float = 0.0) -> dict:
+    """Second GEMM of the MXFP8 block: out = r * (A Bt^T) with A, Bt the
+    dequantised block-scaled operands and r = 1 / sqrt(sum_t partial / N + eps)
+    (r = 1 without partials: a plain MXFP8 GEMM)."""
+    A = mx_dequantize(aq, ae)
+    B = mx_dequantize(bq, be)
+    acc = A @ B.T
+    if partial is None:
+        return {"r": None, "out": acc}
+    r = 1.0 / np.sqrt(np.asarray(partial, dtype=np.float64).sum(axis=0) / n_norm + eps)
+    return {"r": r, "out": r[:, None] * acc}
+
+
+def rmsnorm_block_mx(x8, sx, W1t8, sw1, res, gamma, W2q, W2e, eps: float, tile_cols: int = 256) -> dict:
+    """The MXFP8 block: the two steps above composed."""
+    g1 = gemm_res_partialrms_mx(x8, sx, W1t8, sw1, res, gamma, tile_cols)
+    N = g1["h"].shape[1]
+    g2 = gemm_rowscale_partial_mx(g1["hq"], g1["he"], W2q, W2e, g1["partial"], N, eps)
+    return {**g1, "r": g2["r"], "out": g2["out"]}
