@@ -251,19 +251,19 @@ def arm_config(l2, ws):
 
 # ------------------------------------------------------------ per-kernel rows
 
-NOMINAL_TFLOPS = {"bf16": 2250.0, "e4m3": 4500.0}  # dense, per GPU
+NOMINAL_TFLOPS = {"bf16": 2250.0, "e4m3": 4500.0, "mxfp8": 4500.0}  # dense, per GPU
 NOMINAL_GBS = 8000.0
 
 
 def kernel_row(name, call, ts, flops, nbytes, bound, launches, dtype, note, peaks, clk):
     """One kernel's roofline row from its per-launch device times `ts` (ms).
 
-    Tensor-bound rows take the measured bf16 cuBLAS peaks (e4m3: twice them,
-    the nominal ratio); HBM-bound rows the measured copy bandwidth.  The
+    Tensor-bound rows take the measured bf16 cuBLAS peaks (e4m3 and
+    block-scaled MXFP8: twice them, the nominal ratio); HBM-bound rows the measured copy bandwidth.  The
     nominal roofline time is the slower of the FLOPs at the dense nominal rate
     and the bytes at 8 TB/s."""
     burst, sustained, hbm, src = peaks
-    scale = 2.0 if dtype == "e4m3" else 1.0
+    scale = 2.0 if dtype in ("e4m3", "mxfp8") else 1.0
     ms = sum(ts) / len(ts)
     row = {"kernel": name, "call": call, "launches_per_call": launches, "calls": len(ts), "dtype": dtype,
            "bound": bound, "ms": round(ms, 5), "ms_median": round(ts[len(ts) // 2], 5), "ms_min": round(ts[0], 5),
@@ -272,7 +272,7 @@ def kernel_row(name, call, ts, flops, nbytes, bound, launches, dtype, note, peak
         tf = flops / ms / 1e9
         row.update({"tflops": round(tf, 1), "peak": round(burst * scale, 1), "unit": "TFLOP/s",
                     "frac": round(tf / (burst * scale), 4), "frac_of_sustained": round(tf / (sustained * scale), 4),
-                    "peak_kind": f"{dtype} from the bf16 cuBLAS burst ({src})" + (" x 2 (nominal e4m3/bf16 ratio)"
+                    "peak_kind": f"{dtype} from the bf16 cuBLAS burst ({src})" + (f" x 2 (nominal {dtype}/bf16 ratio)"
                                                                                     if scale != 1 else "")})
     if bound == "hbm":
         row.update({"peak": hbm, "unit": "GB/s", "frac": round(nbytes / ms / 1e6 / hbm, 4),
@@ -827,6 +827,15 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
            "partial": torch.empty(C.partial_cols(D), M_TOK, dtype=torch.float32, device=dev),
            "r": torch.empty(M_TOK, dtype=torch.float32, device=dev)}
 
+    # MXFP8 block: W2 quantised once (a weight), hg's scales formed by GEMM1's epilogue
+    W2t_bf = W2.t().contiguous()
+    W2q, W2sf = C.mx_quantize(W2t_bf)
+    bmx = {"h": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
+           "hq": torch.empty(M_TOK, D, dtype=torch.uint8, device=dev),
+           "hsf": torch.empty(C.mx_sf_bytes(M_TOK, D), dtype=torch.uint8, device=dev),
+           "partial": torch.empty(C.partial_cols(D), M_TOK, dtype=torch.float32, device=dev),
+           "r": torch.empty(M_TOK, dtype=torch.float32, device=dev)}
+
     s_y = torch.ones(1, dtype=torch.float32, device=dev)
     bu8 = {"t": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
            "h": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
@@ -852,11 +861,21 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
             evs[4].record(stream)
         C.unfused_block_fp8(x8, sx, W1t8, sw1, res_d, gamma, s_y, W2t8, sw2, EPS, out=out8, bufs=bu8)
         C.fp8_scale_from_amax(bu8["amax"], scale_out=s_y)
+        if evs:
+            evs[5].record(stream)
+            flush.zero_()
+            evs[6].record(stream)
+        C.gemm_res_partialrms_mx(x8, sx, W1t8, sw1, res_d, gamma, h_out=bmx["h"], hq_out=bmx["hq"],
+                                 hsf_out=bmx["hsf"], partial_out=bmx["partial"])
+        if evs:
+            evs[7].record(stream)
+        C.gemm_rowscale_partial_mx(bmx["hq"], bmx["hsf"], W2q, W2sf, bmx["partial"], D, EPS, out=out8,
+                                   r_out=bmx["r"])
 
     for _ in range(3):
         f8(None)
-    _, parts = timed(f8, steps, 0, inner_events=5)
-    k = [sum(p[i] for p in parts) / len(parts) for i in range(6)]
+    _, parts = timed(f8, steps, 0, inner_events=8)
+    k = [sum(p[i] for p in parts) / len(parts) for i in range(9)]
     f_blk = 2.0 * M_TOK * D * (D + N2)
     ms8 = k[2] + k[3]
     res["fp8_block"] = {"ms": round(ms8, 4), "tflops": round(f_blk / ms8 / 1e9, 1),
@@ -867,6 +886,16 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
                         "unfused_fp8_chain_ms": round(k[5], 4), "speedup_vs_unfused_fp8": round(k[5] / ms8, 4),
                         "bf16_block_ms_same_steps": round(k[0], 4), "speedup_vs_bf16_block": round(k[0] / ms8, 4),
                         "scaling": "per-tensor e4m3; hg8 (y8) scale from the previous step's amax"}
+    msx = k[7] + k[8]
+    res["mx_block"] = {"ms": round(msx, 4), "tflops": round(f_blk / msx / 1e9, 1),
+                       "frac_of_nominal_mxfp8_4500": round(f_blk / (msx / 1e3) / 4.5e15, 4),
+                       "gemm_res_partialrms_mx_ms": round(k[7], 4),
+                       "gemm_rowscale_partial_mx_ms": round(k[8], 4),
+                       "gemm_rowscale_partial_mx_tflops": round(2.0 * M_TOK * D * N2 / k[8] / 1e9, 1),
+                       "bf16_block_ms_same_steps": round(k[0], 4), "speedup_vs_bf16_block": round(k[0] / msx, 4),
+                       "fp8_block_ms_same_steps": round(ms8, 4),
+                       "scaling": "MXFP8: an E8M0 scale per 32 elements of K; x and W1 per-tensor e4m3, W2 "
+                                  "quantised once (a weight), hg's scales formed in GEMM1's epilogue"}
     if kloop:
         kloop("gemm_res_partialrms_fp8 (e4m3 GEMM1 + residual + partial RMS + hg8)", "coda_gemm_res_partialrms_fp8",
               lambda: C.gemm_res_partialrms_fp8(x8, sx, W1t8, sw1, res_d, gamma, s_hg, h_out=b8["h"],
@@ -878,7 +907,20 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
               lambda: C.gemm_rowscale_partial_fp8(b8["hg8"], s_hg, W2t8, sw2, b8["partial"], D, EPS, out=out8,
                                                   r_out=b8["r"]),
               2.0 * M * D * N2, M * D + D * N2 + 2 * M * N2 + 4 * M * (D // 128) + 4 * M, dtype="e4m3")
-    del res_d, x8, W1t8, W2t8, b8, out8, out16, b16, bu8
+        sfa, sfb = C.mx_sf_bytes(M, D), C.mx_sf_bytes(N2, D)
+        kloop("gemm_res_partialrms_mx (e4m3 GEMM1 + residual + partial RMS + MXFP8 hg)",
+              "coda_gemm_res_partialrms_mx",
+              lambda: C.gemm_res_partialrms_mx(x8, sx, W1t8, sw1, res_d, gamma, h_out=bmx["h"], hq_out=bmx["hq"],
+                                               hsf_out=bmx["hsf"], partial_out=bmx["partial"]),
+              2.0 * M * D * D, M * D + D * D + 2 * 2 * M * D + M * D + sfa + 4 * M * (D // 128), dtype="e4m3")
+        kloop("gemm_rowscale_partial_mx (block-scaled GEMM2 + folded reduction + row scale)",
+              "coda_gemm_rowscale_partial_mx",
+              lambda: C.gemm_rowscale_partial_mx(bmx["hq"], bmx["hsf"], W2q, W2sf, bmx["partial"], D, EPS, out=out8,
+                                                 r_out=bmx["r"]),
+              2.0 * M * D * N2, M * D + sfa + D * N2 + sfb + 2 * M * N2 + 4 * M * (D // 128) + 4 * M, dtype="mxfp8")
+        kloop("mx_quantize (W2 to MXFP8, once per weight update)", "coda_mx_quantize",
+              lambda: C.mx_quantize(W2t_bf, q_out=W2q, sf_out=W2sf), 0.0, 2 * N2 * D + N2 * D + sfb, bound="hbm")
+    del res_d, x8, W1t8, W2t8, b8, out8, out16, b16, bu8, W2t_bf, W2q, W2sf, bmx
 
     # QKV projection with RoPE in its epilogue (1B attention input: 32 q + 8 k + 8 v heads of 64)
     n_qkv, rope_cols = 48 * 64, 40 * 64

@@ -77,6 +77,10 @@ _SIGS = {
     "coda_rmsnorm_block_host_workspace_size": (_SZ, [_I64, _I64, _I64, _I64]),
     "coda_rmsnorm_block_host": (_ST, [_P, _P, _P, _P, _P, _F, _P, _P, _SZ, _I64, _I64, _I64, _I64, _I64, _P]),
     "coda_unfused_rmsnorm_fp8": (_ST, [_P, _P, _F, _P, _P, _P, _P, _I64, _I64, _P]),
+    "coda_mx_sf_bytes": (_I64, [_I64, _I64]),
+    "coda_mx_quantize": (_ST, [_P, _I64, _I64, _P, _P, _P]),
+    "coda_gemm_res_partialrms_mx": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "coda_gemm_rowscale_partial_mx": (_ST, [_P, _P, _P, _P, _P, _I64, _I64, _F, _P, _P, _I64, _I64, _I64, _P]),
 }
 
 _lib = None
@@ -627,6 +631,87 @@ def unfused_block_fp8(x8, sx, W1t8, sw1, res, gamma, s_y, W2t8, sw2, eps: float,
                                       r_out=b.get("r"))
     out = gemm_fp8(y8, s_y, W2t8, sw2, out=out)
     return {"out": out, "t": t, "h": h, "y8": y8, "amax": amax, "r": r}
+
+
+# ----------------------------------------------- block-scaled e4m3 (MXFP8)
+
+
+def mx_sf_bytes(rows: int, cols: int) -> int:
+    """Bytes of the tiled scale buffer of a [rows, cols] MXFP8 operand."""
+    n = load_library().coda_mx_sf_bytes(int(rows), int(cols))
+    if n < 0:
+        raise ValueError(f"no MXFP8 layout for [{rows}, {cols}] (cols must be a multiple of 128)")
+    return n
+
+
+def mx_quantize(src, q_out=None, sf_out=None):
+    """MXFP8 codes of a bf16 [rows, cols] tensor, blocked along its rows.
+    Returns (codes uint8 [rows, cols], tiled scales uint8)."""
+    rows, cols = src.shape
+    _need(src, BF16, "src")
+    q_out = _empty((rows, cols), U8, src) if q_out is None else q_out
+    sf_out = _empty((mx_sf_bytes(rows, cols),), U8, src) if sf_out is None else sf_out
+    _call("coda_mx_quantize", _ptr(src), rows, cols, _ptr(q_out), _ptr(sf_out), _stream())
+    return q_out, sf_out
+
+
+def gemm_res_partialrms_mx(x8, sx, Wt8, sw, res, gamma, *, h=True, h_out=None, hq_out=None, hsf_out=None,
+                           partial_out=None):
+    """First GEMM of the MXFP8 block.  Returns (h bf16 or None, hg codes,
+    hg's tiled scales, partial [T, M])."""
+    M, K = x8.shape
+    N = Wt8.shape[0]
+    _need(x8, U8, "x8")
+    _need(Wt8, U8, "Wt8", (N, K))
+    _need(sx, F32, "sx", (1,))
+    _need(sw, F32, "sw", (1,))
+    if res is not None:
+        _need(res, BF16, "res", (M, N))
+    _need(gamma, BF16, "gamma", (N,))
+    if h and h_out is None:
+        h_out = _empty((M, N), BF16, x8)
+    hq_out = _empty((M, N), U8, x8) if hq_out is None else hq_out
+    hsf_out = _empty((mx_sf_bytes(M, N),), U8, x8) if hsf_out is None else hsf_out
+    partial_out = _empty((partial_cols(N), M), F32, x8) if partial_out is None else partial_out
+    _call("coda_gemm_res_partialrms_mx", _ptr(x8), _ptr(sx), _ptr(Wt8), _ptr(sw), _ptr(res), _ptr(gamma),
+          _ptr(h_out if h else None), _ptr(hq_out), _ptr(hsf_out), _ptr(partial_out), M, N, K, _stream())
+    return (h_out if h else None), hq_out, hsf_out, partial_out
+
+
+def gemm_rowscale_partial_mx(Aq, Asf, Wq, Wsf, partial=None, N_norm: int = 0, eps: float = 0.0, out=None,
+                             r_out=None):
+    """Second GEMM of the MXFP8 block: out = r * (A Wt^T) with block-scaled
+    operands, r from the partials (partial None: a plain MXFP8 GEMM, r = 1).
+    Returns (out bf16, r or None)."""
+    M, K = Aq.shape
+    N = Wq.shape[0]
+    _need(Aq, U8, "Aq")
+    _need(Wq, U8, "Wq", (N, K))
+    _need(Asf, U8, "Asf", (mx_sf_bytes(M, K),))
+    _need(Wsf, U8, "Wsf", (mx_sf_bytes(N, K),))
+    out = _empty((M, N), BF16, Aq) if out is None else out
+    T = 0
+    if partial is not None:
+        _need(partial, F32, "partial", (partial.shape[0], M))
+        T = partial.shape[0]
+        r_out = _empty((M,), F32, Aq) if r_out is None else r_out
+    else:
+        r_out = None
+    _call("coda_gemm_rowscale_partial_mx", _ptr(Aq), _ptr(Asf), _ptr(Wq), _ptr(Wsf), _ptr(partial), T, N_norm,
+          float(eps), _ptr(r_out), _ptr(out), M, N, K, _stream())
+    return out, r_out
+
+
+def gemm_rmsnorm_gemm_mx(x8, sx, W1t8, sw1, res, gamma, W2q, W2sf, eps: float, out=None, bufs=None):
+    """The MXFP8 block in two launches: returns dict(out, h, hq, hsf,
+    partial, r).  hg's scales are formed in the first GEMM's epilogue."""
+    N = W1t8.shape[0]
+    b = bufs or {}
+    h, hq, hsf, partial = gemm_res_partialrms_mx(x8, sx, W1t8, sw1, res, gamma, h_out=b.get("h"),
+                                                 hq_out=b.get("hq"), hsf_out=b.get("hsf"),
+                                                 partial_out=b.get("partial"))
+    out, r = gemm_rowscale_partial_mx(hq, hsf, W2q, W2sf, partial, N, eps, out=out, r_out=b.get("r"))
+    return {"out": out, "h": h, "hq": hq, "hsf": hsf, "partial": partial, "r": r}
 
 
 def _need_host(t, dtype, name, shape=None):

@@ -140,6 +140,21 @@ bool tmap2d_u8_plain(CUtensorMap* m, const void* base, uint64_t cols, uint64_t r
   return r == CUDA_SUCCESS;
 }
 
+// Scale bytes of a block-scaled operand: the tiled layout seen as rows of 128
+// 32-bit words (one 512-byte atom per row), `box_rows` atoms per copy.
+bool tmap_sf(CUtensorMap* m, const void* base, uint64_t atoms, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {128, atoms};
+  cuuint64_t strides[1] = {512};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Operand maps of the mainloop.  A: [M, K] K-major (box 64 x 128) or stored
 // transposed as [K, M] (MN-major, box 64 x 64).  B: [K, N] MN-major (box 64 x 64)
 // or stored transposed as [N, K] (K-major, box 64 x BN).
@@ -178,6 +193,8 @@ enum KernelKind : uint32_t {
   kKindBlock,
   kKindResPartialF8,
   kKindRowScaleF8,
+  kKindResPartialMX,
+  kKindRowScaleMX,
   kKindGroupedCE,      // CE backward: dW (long) + dH
   kKindGroupedWX,      // first-GEMM backward: dW1 (long) + dx
   kKindCount
@@ -191,12 +208,13 @@ enum KernelKind : uint32_t {
 constexpr int64_t kCEBwdChunk = 8192;
 
 // Pipeline depth of the pair kernels: as many 32 KB stages (this CTA's halves
-// of A and B) as fit next to the epilogue's shared memory, at most 8.
+// of A and B, plus 1.5 KB of scales for block-scaled operands) as fit next to
+// the epilogue's shared memory, at most 8.
 template <class Epi>
 constexpr int pair_stages() {
   constexpr int budget = 232448 - 1024 - 256 - GemmSmem<256, 1, true, Epi>::kEpiBytes -
                          GemmSmem<256, 1, true, Epi>::kXchgBytes;
-  constexpr int st = budget / (2 * kBM * kBK * 2);
+  constexpr int st = budget / (2 * kBM * kBK * 2 + GemmSmem<256, 1, true, Epi>::kSFStage);
   return st > 8 ? 8 : st;
 }
 
@@ -1399,6 +1417,114 @@ coda_status_t coda_gemm_fp8(const uint8_t* A8, const float* sa, const uint8_t* W
   return run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M),
                                                                     static_cast<int>(N), static_cast<int>(K), n_nt,
                                                                     raster_group(M, N, K), kKindRowScaleF8,
+                                                                    static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------ block-scaled e4m3 (MXFP8)
+
+int64_t coda_mx_sf_bytes(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0 || cols % 128 != 0) return -1;
+  return (cols / 128) * ((rows + 127) / 128) * 512;
+}
+
+namespace {
+inline bool mx_dim_ok(int64_t v) { return dim_ok(v) && v % 128 == 0; }
+}  // namespace
+
+coda_status_t coda_mx_quantize(const uint16_t* src, int64_t rows, int64_t cols, uint8_t* q_out, uint8_t* sf_out,
+                               void* stream) {
+  CODA_CHECK(rows >= 0 && rows < (int64_t(1) << 31) && mx_dim_ok(cols) &&
+                 (rows + 127) / 128 * 128 * (cols / 32) < (int64_t(1) << 40),
+             CODA_ERR_SHAPE);
+  if (rows == 0) return CODA_OK;
+  CODA_CHECK(src && q_out && sf_out, CODA_ERR_NULL);
+  CODA_CHECK(al16(src) && al16(q_out) && al16(sf_out), CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  mx_quantize_kernel<<<info->sms * 4, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const __nv_bfloat16*>(src), static_cast<int>(rows), static_cast<int>(cols), q_out, sf_out);
+  return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
+}
+
+coda_status_t coda_gemm_res_partialrms_mx(const uint8_t* x8, const float* sx, const uint8_t* Wt8, const float* sw,
+                                          const uint16_t* res, const uint16_t* gamma, uint16_t* h_out,
+                                          uint8_t* hq_out, uint8_t* hsf_out, float* partial, int64_t M, int64_t N,
+                                          int64_t K, void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && mx_dim_ok(N) && fp8_dim_ok(K), CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(x8 && sx && Wt8 && sw && gamma && hq_out && hsf_out && partial, CODA_ERR_NULL);
+  CODA_CHECK(al16(x8) && al16(Wt8) && al16(res) && al16(gamma) && al16(h_out) && al16(hq_out) && al16(hsf_out) &&
+                 al16(partial),
+             CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  using Epi = EpiLoadStore2<3>;
+  GemmParams<Epi> p{};
+  bool ok = tmap2d_u8(&p.tmA, x8, K, M, K, 128, kBM) && tmap2d_u8(&p.tmB, Wt8, K, N, K, 128, 128) &&
+            tmap2d_u8(&p.tmBh, Wt8, K, N, K, 128, 64) && tmap2d_u8(&p.ep.tmOut2, hq_out, N, M, N, 128, 32) &&
+            tmap2d_u8_plain(&p.ep.tmOut2h, hq_out, N, M, N, 64, 32);
+  p.has_bh = 1;
+  if (h_out) ok = ok && map_out_bf16(&p.ep.tmOut1, h_out, M, N, N);
+  if (!ok) return CODA_ERR_INTERNAL;
+  p.ep.in = reinterpret_cast<const __nv_bfloat16*>(res);
+  p.ep.gamma = reinterpret_cast<const __nv_bfloat16*>(gamma);
+  p.ep.partial = partial;
+  p.ep.has_out1 = h_out != nullptr;
+  p.ep.has_out2 = 1;
+  p.ep.sa = sx;
+  p.ep.sb = sw;
+  p.ep.sf_out = hsf_out;
+  p.ep.sf_rb = static_cast<int>((M + 127) / 128);
+  const int n_nt = static_cast<int>((N + 255) / 256);
+  return run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M),
+                                                                    static_cast<int>(N), static_cast<int>(K), n_nt,
+                                                                    raster_group(M, N, K), kKindResPartialMX,
+                                                                    static_cast<cudaStream_t>(stream));
+}
+
+coda_status_t coda_gemm_rowscale_partial_mx(const uint8_t* Aq, const uint8_t* Asf, const uint8_t* Wq,
+                                            const uint8_t* Wsf, const float* partial, int64_t T, int64_t N_norm,
+                                            float eps, float* r_out, uint16_t* out, int64_t M, int64_t N, int64_t K,
+                                            void* stream) {
+  CODA_CHECK(M >= 0 && M < (int64_t(1) << 31) && mx_dim_ok(N) && mx_dim_ok(K) &&
+                 (partial == nullptr || (T > 0 && T <= 1 << 20 && N_norm > 0 && eps >= 0.f)),
+             CODA_ERR_SHAPE);
+  if (M == 0) return CODA_OK;
+  CODA_CHECK(Aq && Asf && Wq && Wsf && out, CODA_ERR_NULL);
+  CODA_CHECK(al16(Aq) && al16(Asf) && al16(Wq) && al16(Wsf) && al16(partial) && al16(r_out) && al16(out),
+             CODA_ERR_ALIGN);
+  int dev = 0;
+  DevInfo* info = nullptr;
+  {
+    const coda_status_t ds = current_device(&dev, &info);
+    if (ds != CODA_OK) return ds;
+  }
+  using Epi = EpiRowScaleMX;
+  GemmParams<Epi> p{};
+  const int64_t rba = (M + 127) / 128, rbb = N / 128, nkb = K / 128;
+  if (!(tmap2d_u8(&p.tmA, Aq, K, M, K, 128, kBM) && tmap2d_u8(&p.tmB, Wq, K, N, K, 128, 128) &&
+        tmap_sf(&p.tmSFA, Asf, static_cast<uint64_t>(nkb * rba), 1) &&
+        tmap_sf(&p.tmSFB, Wsf, static_cast<uint64_t>(nkb * rbb), 2) && map_out_bf16(&p.ep.tmOut, out, M, N, N)))
+    return CODA_ERR_INTERNAL;
+  p.sf_rba = static_cast<int>(rba);
+  p.sf_rbb = static_cast<int>(rbb);
+  p.ep.partial = partial;
+  p.ep.T = static_cast<int>(T);
+  p.ep.inv_n = partial ? 1.0f / static_cast<float>(N_norm) : 1.0f;
+  p.ep.eps = eps;
+  p.ep.r_out = partial ? r_out : nullptr;
+  const int n_nt = static_cast<int>((N + 255) / 256);
+  return run_gemm<256, pair_stages<Epi>(), false, false, true, Epi>(dev, info, p, static_cast<int>(M),
+                                                                    static_cast<int>(N), static_cast<int>(K), n_nt,
+                                                                    raster_group(M, N, K), kKindRowScaleMX,
                                                                     static_cast<cudaStream_t>(stream));
 }
 

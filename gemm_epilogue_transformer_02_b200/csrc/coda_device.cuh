@@ -396,6 +396,86 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
                : "memory");
 }
 
+// ---------------------------------- block-scaled e4m3 operands (MXFP8)
+//
+// tcgen05.mma kind::mxf8f6f4.block_scale multiplies e4m3 operands whose K
+// runs in blocks of 32 elements, each block with an E8M0 scale (a power of
+// two, byte = exponent + 127).  The scales are read from tensor memory: a
+// 128-row group's scales for one 128-wide k-block are a 512-byte atom whose
+// byte (i % 32) * 16 + ((i / 32) % 4) * 4 + b holds row i's scale of K block
+// b (b = 0..3, one per 32-wide MMA step); tcgen05.cp copies the atom, as 32
+// rows of 16 bytes, into 32 lanes x 4 columns of every lane quarter, and the
+// MMA's instruction descriptor selects the byte b of each 32-bit word.
+
+// Shared-memory descriptor of an unswizzled, K-major matrix of 16-byte rows
+// (the source of tcgen05.cp): rows 16 bytes apart, so its eight-row core
+// matrices sit 128 bytes apart (stride byte offset); layout type 0 (no
+// swizzle) in bits 61-63, descriptor version 1 in bits 46-47.  The leading
+// byte offset is unused by a matrix one core matrix wide.
+__device__ __forceinline__ uint64_t sdesc_plain16(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(16 >> 4) << 16;
+  d |= static_cast<uint64_t>(128 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// Copy a 32-row x 16-byte matrix from shared memory into tensor memory at
+// taddr (32 lanes x 4 columns), replicated into all four lane quarters; in a
+// CTA pair each CTA copies from its own shared memory into its own tensor
+// memory.  Issued by the thread that issues the MMAs, so it is ordered before
+// them and tracked by the same tcgen05.commit.
+__device__ __forceinline__ void tc_cp_32x128_w4_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Instruction descriptor of kind::mxf8f6f4 block-scaled: E4M3 A and B (format
+// code 0 in bits 7-9 and 10-12), both K-major, N >> 3 in bits 17-22, E8M0
+// scales (bit 23), M >> 4 in bits 24-28; bits 4-5 and 29-30 select the byte
+// of B's and A's scale words (sf_id: the 32-wide K step within the k-block).
+// The accumulator is fp32 (no format field).
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, uint32_t sf_id) {
+  return (sf_id << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24) | (sf_id << 29);
+}
+
+// One 256-row block-scaled MMA of a CTA pair; sfa / sfb: tensor-memory
+// addresses of the A and B scales (the scale byte also in bits 30-31).
+__device__ __forceinline__ void tc_mma_mx_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Scale exponent of a block whose largest magnitude is amax (finite, >= 0):
+// the smallest e with amax <= 448 * 2^e.  With amax = (1 + f) 2^E and
+// 448 = 1.75 * 2^8 that is E - 8 when f <= 0.75 and E - 7 otherwise, read
+// exactly from the bits of amax; at least -127 (the smallest E8M0 scale),
+// and 0 for an all-zero block.
+__device__ __forceinline__ int mx_e4m3_exponent(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  if (b == 0u) return 0;
+  const int field = static_cast<int>(b >> 23);
+  if (field == 0) return -127;  // below the normal range
+  const int e = field - 127 - ((b & 0x7FFFFFu) <= 0x600000u ? 8 : 7);
+  return e < -127 ? -127 : e;
+}
+
+// 2^-e as an fp32 value (-127 <= e <= 126; finite fp32 data gives e <= 120).
+__device__ __forceinline__ float exp2_neg(int e) { return __uint_as_float(static_cast<uint32_t>(127 - e) << 23); }
+
+// Byte offset of the scale of row i, 32-element K block j, in the tiled scale
+// layout of an operand with `nrb` 128-row blocks: one 512-byte atom per
+// (128-wide k-block, 128-row block), k-blocks outermost.
+__host__ __device__ __forceinline__ size_t mx_sf_offset(int i, int j, int nrb) {
+  return ((static_cast<size_t>(j >> 2) * nrb + (i >> 7)) << 9) + ((i & 31) << 4) + (((i >> 5) & 3) << 2) + (j & 3);
+}
+
 // ------------------------------------------- cross-CTA completion counters
 
 // Order this thread's completed async-proxy (TMA) global writes before its

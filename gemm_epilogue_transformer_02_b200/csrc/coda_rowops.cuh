@@ -411,6 +411,55 @@ __global__ void __launch_bounds__(256) quantize_e4m3_kernel(const __nv_bfloat16*
   }
 }
 
+// MXFP8 codes of a row-major bf16 matrix [rows, cols] (cols % 128 == 0),
+// blocked along the row: each thread takes one 32-element block, finds its
+// largest magnitude, takes the smallest power-of-two scale 2^e that keeps it
+// within the e4m3 range and writes the 32 codes of v * 2^-e (round to nearest
+// even) and the E8M0 byte e + 127 into the tiled scale layout.  Scale bytes of
+// the padding rows (up to a whole 128-row block) are set to 127 (scale 1).
+__global__ void __launch_bounds__(256) mx_quantize_kernel(const __nv_bfloat16* __restrict__ src, int rows, int cols,
+                                                          uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+  const int nb = cols >> 5;
+  const int nrb = (rows + 127) >> 7;
+  const size_t total = static_cast<size_t>(nrb) * 128 * nb;
+  for (size_t t = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; t < total;
+       t += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int row = static_cast<int>(t / nb);
+    const int j = static_cast<int>(t - static_cast<size_t>(row) * nb);
+    int e = 0;
+    if (row < rows) {
+      const uint4* p = reinterpret_cast<const uint4*>(src + static_cast<size_t>(row) * cols + j * 32);
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = __ldg(p + u);
+      float amax = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w[k])), fabsf(bf16hi(w[k]))));
+      }
+      e = mx_e4m3_exponent(amax);
+      const float inv = exp2_neg(e);
+      uint32_t out[8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        const uint32_t c0 = pack_e4m3x2(bf16lo(w[0]) * inv, bf16hi(w[0]) * inv);
+        const uint32_t c1 = pack_e4m3x2(bf16lo(w[1]) * inv, bf16hi(w[1]) * inv);
+        const uint32_t c2 = pack_e4m3x2(bf16lo(w[2]) * inv, bf16hi(w[2]) * inv);
+        const uint32_t c3 = pack_e4m3x2(bf16lo(w[3]) * inv, bf16hi(w[3]) * inv);
+        out[2 * u] = c0 | (c1 << 16);
+        out[2 * u + 1] = c2 | (c3 << 16);
+      }
+      uint4* d = reinterpret_cast<uint4*>(q + static_cast<size_t>(row) * cols + j * 32);
+      d[0] = make_uint4(out[0], out[1], out[2], out[3]);
+      d[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    }
+    sf[mx_sf_offset(row, j, nrb)] = static_cast<uint8_t>(e + 127);
+  }
+}
+
 // Transposing form: src [rows, cols] -> dst [cols, rows] (a weight stored
 // K-major for the e4m3 mainloop), 64 x 64 tiles through shared memory.
 // Needs cols % 8 == 0 and rows % 4 == 0.

@@ -422,6 +422,58 @@ coda_status_t coda_unfused_rmsnorm_fp8(const uint16_t* h, const uint16_t* gamma,
                                        uint8_t* y8_out, float* amax_out, float* r_out, int64_t M, int64_t N,
                                        void* stream);
 
+/* ---------------------------------------------- block-scaled e4m3 (MXFP8)
+ *
+ * The block with microscaled FP8 operands (the OCP "Microscaling Formats (MX)"
+ * layout; the article gives no low-precision recipe, see the FP8 section):
+ * every 32 consecutive elements along the reduction dimension K share one
+ * power-of-two scale 2^e, stored as the byte e + 127 (E8M0); the elements are
+ * e4m3 codes of v * 2^-e.  e is the smallest exponent that keeps the block's
+ * largest magnitude within 448 (no element saturates), clamped to
+ * [-127, 127]; an all-zero block takes e = 0.  The scales replace the FP8
+ * block's per-tensor scale of hg, which had to come from an earlier call.
+ *
+ * Scale layout ("tiled"): for an operand of R rows and K columns (K a
+ * multiple of 128), with nrb = ceil(R / 128), the scale of row i, 32-element
+ * block j sits at byte ((j / 4) * nrb + i / 128) * 512 + (i % 32) * 16 +
+ * ((i / 32) % 4) * 4 + j % 4: one 512-byte atom per (128-wide k-block,
+ * 128-row block), k-blocks outermost, which the GEMM copies into tensor
+ * memory as it is.  Padding rows (R up to 128 nrb) hold 127.
+ * coda_mx_sf_bytes(R, K) = (K / 128) * nrb * 512 (-1 for a bad shape). */
+int64_t coda_mx_sf_bytes(int64_t rows, int64_t cols);
+
+/* MXFP8 codes of a row-major bf16 matrix src [rows, cols], blocked along
+ * each row: q_out [rows, cols] e4m3, sf_out the tiled scales
+ * (coda_mx_sf_bytes(rows, cols) bytes, every byte written).  cols % 128 == 0.
+ * Used for the weight W2 stored transposed ([N2, N], K-major). */
+coda_status_t coda_mx_quantize(const uint16_t* src, int64_t rows, int64_t cols, uint8_t* q_out, uint8_t* sf_out,
+                               void* stream);
+
+/* First GEMM of the MXFP8 block: as coda_gemm_res_partialrms_fp8 (e4m3 x8
+ * [M, K] and Wt8 [N, K] with per-tensor scales sx, sw; h = acc * sx * sw +
+ * res; partial[t, i] over 128-column slots; h_out bf16 or NULL), except that
+ * hg = gamma * h is written in MXFP8 from the epilogue: hq_out [M, N] e4m3
+ * codes and hsf_out its tiled scales (coda_mx_sf_bytes(M, N) bytes; each
+ * 32-column block of a row quantised from the fp32 values as they are
+ * formed).  N a multiple of 128, K of 16. */
+coda_status_t coda_gemm_res_partialrms_mx(const uint8_t* x8, const float* sx, const uint8_t* Wt8, const float* sw,
+                                          const uint16_t* res, const uint16_t* gamma, uint16_t* h_out,
+                                          uint8_t* hq_out, uint8_t* hsf_out, float* partial, int64_t M, int64_t N,
+                                          int64_t K, void* stream);
+
+/* Second GEMM of the MXFP8 block: acc = A Wt^T with block-scaled operands
+ * (tcgen05 kind::mxf8f6f4: the scales are applied inside the MMA), then as
+ * coda_gemm_rowscale_partial: r_i = 1/sqrt(sum_t partial[t, i] / N_norm +
+ * eps), out = bf16(r_i * acc_ij), r_out [M] or NULL.  partial == NULL gives
+ * a plain MXFP8 GEMM (r = 1; T, N_norm, eps, r_out ignored).  Aq [M, K] with
+ * tiled scales Asf, Wq [N, K] (W2 transposed) with tiled scales Wsf; out
+ * [M, N] bf16.  N and K multiples of 128.  Launched with programmatic stream
+ * serialisation after coda_gemm_res_partialrms_mx, as the FP8 pair. */
+coda_status_t coda_gemm_rowscale_partial_mx(const uint8_t* Aq, const uint8_t* Asf, const uint8_t* Wq,
+                                            const uint8_t* Wsf, const float* partial, int64_t T, int64_t N_norm,
+                                            float eps, float* r_out, uint16_t* out, int64_t M, int64_t N, int64_t K,
+                                            void* stream);
+
 /* ---------------------------------------------------------------- testing */
 
 /* Launches one block that waits on a barrier nothing ever signals, with time

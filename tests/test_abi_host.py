@@ -191,6 +191,31 @@ def test_argument_errors_of_the_remaining_calls(lib):
     assert u8(A, B, 1e-6, None, D, A, None, 16, 64, None) == NULL  # s_y
     assert u8(A, B, 1e-6, C, D, A, MIS, 16, 64, None) == ALIGN     # r_out
 
+    # MXFP8: the scale layout's size, and the calls' argument checks
+    assert lib.coda_mx_sf_bytes(300, 256) == 2 * 3 * 512
+    assert lib.coda_mx_sf_bytes(1, 128) == 512
+    assert lib.coda_mx_sf_bytes(16, 96) == -1            # cols not a multiple of 128
+    assert lib.coda_mx_sf_bytes(-1, 128) == -1
+    mq = lib.coda_mx_quantize  # (src, rows, cols, q, sf, stream)
+    assert mq(A, 16, 192, B, C, None) == SHAPE
+    assert mq(A, 16, 128, None, C, None) == NULL
+    assert mq(A, 16, 128, B, MIS, None) == ALIGN
+    assert mq(A, 0, 128, B, C, None) == OK
+    pm = lib.coda_gemm_res_partialrms_mx  # (x8, sx, Wt8, sw, res, gamma, h, hq, hsf, partial, M, N, K, s)
+    assert pm(A, B, C, D, None, A, None, B, C, D, 16, 192, 64, None) == SHAPE  # N not a multiple of 128
+    assert pm(A, B, C, D, None, A, None, B, C, D, 16, 256, 40, None) == SHAPE  # K not a multiple of 16
+    assert pm(A, B, C, D, None, A, None, B, None, D, 16, 256, 64, None) == NULL  # scales
+    assert pm(A, B, C, D, None, None, None, B, C, D, 16, 256, 64, None) == NULL  # gamma
+    assert pm(A, B, C, D, None, A, None, B, MIS, D, 16, 256, 64, None) == ALIGN
+    assert pm(A, B, C, D, None, A, None, B, C, D, 0, 256, 64, None) == OK
+    rm = lib.coda_gemm_rowscale_partial_mx  # (Aq, Asf, Wq, Wsf, partial, T, N_norm, eps, r, out, M, N, K, s)
+    assert rm(A, B, C, D, None, 0, 0, 0.0, None, A, 16, 256, 192, None) == SHAPE   # K
+    assert rm(A, B, C, D, None, 0, 0, 0.0, None, A, 16, 200, 256, None) == SHAPE   # N
+    assert rm(A, B, C, D, A, 0, 64, 1e-6, None, A, 16, 256, 256, None) == SHAPE    # T with partials
+    assert rm(A, B, C, None, None, 0, 0, 0.0, None, A, 16, 256, 256, None) == NULL
+    assert rm(A, B, C, D, None, 0, 0, 0.0, None, MIS, 16, 256, 256, None) == ALIGN
+    assert rm(A, B, C, D, None, 0, 0, 0.0, None, A, 0, 256, 256, None) == OK
+
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_valid_arguments_without_a_gpu_report_device_error(lib):
@@ -198,6 +223,8 @@ def test_valid_arguments_without_a_gpu_report_device_error(lib):
     assert lib.coda_rms_reduce(A, 16, 1, 64, 1e-6, B, None) == DEVICE
     assert lib.coda_fp8_quantize(A, 16, 16, 1, B, C, D, None) == DEVICE
     assert lib.coda_gemm_rowscale_partial_fp8(A, B, C, D, A, 1, 64, 1e-6, None, B, 16, 64, 64, None) == DEVICE
+    assert lib.coda_mx_quantize(A, 16, 128, B, C, None) == DEVICE
+    assert lib.coda_gemm_rowscale_partial_mx(A, B, C, D, None, 0, 0, 0.0, None, A, 16, 256, 256, None) == DEVICE
 
 
 def test_binding_refuses_cpu_tensors(lib):
