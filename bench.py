@@ -836,6 +836,13 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
            "partial": torch.empty(C.partial_cols(D), M_TOK, dtype=torch.float32, device=dev),
            "r": torch.empty(M_TOK, dtype=torch.float32, device=dev)}
 
+    bumx = {"t": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
+            "h": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
+            "y": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
+            "yq": torch.empty(M_TOK, D, dtype=torch.uint8, device=dev),
+            "ysf": torch.empty(C.mx_sf_bytes(M_TOK, D), dtype=torch.uint8, device=dev),
+            "r": torch.empty(M_TOK, dtype=torch.float32, device=dev)}
+
     s_y = torch.ones(1, dtype=torch.float32, device=dev)
     bu8 = {"t": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
            "h": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
@@ -871,11 +878,16 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
             evs[7].record(stream)
         C.gemm_rowscale_partial_mx(bmx["hq"], bmx["hsf"], W2q, W2sf, bmx["partial"], D, EPS, out=out8,
                                    r_out=bmx["r"])
+        if evs:
+            evs[8].record(stream)
+            flush.zero_()
+            evs[9].record(stream)
+        C.unfused_block_mx(x8, sx, W1t8, sw1, res_d, gamma, W2q, W2sf, EPS, out=out8, bufs=bumx)
 
     for _ in range(3):
         f8(None)
-    _, parts = timed(f8, steps, 0, inner_events=8)
-    k = [sum(p[i] for p in parts) / len(parts) for i in range(9)]
+    _, parts = timed(f8, steps, 0, inner_events=10)
+    k = [sum(p[i] for p in parts) / len(parts) for i in range(11)]
     f_blk = 2.0 * M_TOK * D * (D + N2)
     ms8 = k[2] + k[3]
     res["fp8_block"] = {"ms": round(ms8, 4), "tflops": round(f_blk / ms8 / 1e9, 1),
@@ -894,6 +906,7 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
                        "gemm_rowscale_partial_mx_tflops": round(2.0 * M_TOK * D * N2 / k[8] / 1e9, 1),
                        "bf16_block_ms_same_steps": round(k[0], 4), "speedup_vs_bf16_block": round(k[0] / msx, 4),
                        "fp8_block_ms_same_steps": round(ms8, 4),
+                       "unfused_mx_chain_ms": round(k[10], 4), "speedup_vs_unfused_mx": round(k[10] / msx, 4),
                        "scaling": "MXFP8: an E8M0 scale per 32 elements of K; x and W1 per-tensor e4m3, W2 "
                                   "quantised once (a weight), hg's scales formed in GEMM1's epilogue"}
     if kloop:
@@ -920,7 +933,7 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
               2.0 * M * D * N2, M * D + sfa + D * N2 + sfb + 2 * M * N2 + 4 * M * (D // 128) + 4 * M, dtype="mxfp8")
         kloop("mx_quantize (W2 to MXFP8, once per weight update)", "coda_mx_quantize",
               lambda: C.mx_quantize(W2t_bf, q_out=W2q, sf_out=W2sf), 0.0, 2 * N2 * D + N2 * D + sfb, bound="hbm")
-    del res_d, x8, W1t8, W2t8, b8, out8, out16, b16, bu8, W2t_bf, W2q, W2sf, bmx
+    del res_d, x8, W1t8, W2t8, b8, out8, out16, b16, bu8, W2t_bf, W2q, W2sf, bmx, bumx
 
     # QKV projection with RoPE in its epilogue (1B attention input: 32 q + 8 k + 8 v heads of 64)
     n_qkv, rope_cols = 48 * 64, 40 * 64

@@ -714,6 +714,23 @@ def gemm_rmsnorm_gemm_mx(x8, sx, W1t8, sw1, res, gamma, W2q, W2sf, eps: float, o
     return {"out": out, "h": h, "hq": hq, "hsf": hsf, "partial": partial, "r": r}
 
 
+def unfused_block_mx(x8, sx, W1t8, sw1, res, gamma, W2q, W2sf, eps: float, out=None, bufs=None):
+    """The unfused MXFP8 chain: FP8 GEMM -> residual add -> RMSNorm (bf16 y) ->
+    MXFP8 quantisation of y -> block-scaled GEMM, every intermediate in HBM.
+    Returns dict(out, t, h, y, yq, ysf, r)."""
+    b = bufs or {}
+    M = x8.shape[0]
+    t = gemm_fp8(x8, sx, W1t8, sw1, out=b.get("t"))
+    h = unfused_add(t, res, out=b.get("h"))
+    r = b.get("r")
+    if r is None:
+        r = _empty((M,), F32, x8)
+    y = unfused_rmsnorm(h, gamma, eps, y_out=b.get("y"), r_out=r)
+    yq, ysf = mx_quantize(y, q_out=b.get("yq"), sf_out=b.get("ysf"))
+    out, _ = gemm_rowscale_partial_mx(yq, ysf, W2q, W2sf, out=out)
+    return {"out": out, "t": t, "h": h, "y": y, "yq": yq, "ysf": ysf, "r": r}
+
+
 def _need_host(t, dtype, name, shape=None):
     if not isinstance(t, torch.Tensor) or t.is_cuda:
         raise ValueError(f"{name} must be a host (CPU) tensor")

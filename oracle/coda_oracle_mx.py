@@ -166,3 +166,20 @@ def rmsnorm_block_mx(x8, sx, W1t8, sw1, res, gamma, W2q, W2e, eps: float, tile_c
     N = g1["h"].shape[1]
     g2 = gemm_rowscale_partial_mx(g1["hq"], g1["he"], W2q, W2e, g1["partial"], N, eps)
     return {**g1, "r": g2["r"], "out": g2["out"]}
+
+
+def rmsnorm_block_mx_unfused(x8, sx, W1t8, sw1, res, gamma, W2q, W2e, eps: float) -> dict:
+    """The MXFP8 block as separate operators, the comparison chain for the
+    fused MXFP8 block, each intermediate stored in bf16 as the chain stores
+    it: t = bf16((decode(x8) decode(W1t8)^T) sx sw1); h = bf16(t + res);
+    r = 1 / sqrt(mean(h^2) + eps); y = bf16(gamma h r); (yq, ye) =
+    mx_quantize(y); out = mx_dequantize(yq, ye) mx_dequantize(W2q, W2e)^T.
+    Here the normalised y is quantised, block by block from its own values."""
+    t = F8.round_bf16(F8.e4m3_decode(x8) @ F8.e4m3_decode(W1t8).T * (np.float64(sx) * np.float64(sw1)))
+    h = F8.round_bf16(t + np.asarray(res, dtype=np.float64))
+    N = h.shape[1]
+    r = 1.0 / np.sqrt((h * h).sum(axis=1) / N + eps)
+    y = F8.round_bf16(np.asarray(gamma, dtype=np.float64)[None, :] * h * r[:, None])
+    yq, ye = mx_quantize(y)
+    out = mx_dequantize(yq, ye) @ mx_dequantize(W2q, W2e).T
+    return {"t": t, "h": h, "r": r, "y": y, "yq": yq, "ye": ye, "out": out}

@@ -247,6 +247,35 @@ def test_mx_block_tail_full_size_sampled_rows():
     check("out (chain, sampled rows)", f["out"][ri], chain["out"], strict=True)
 
 
+@pytest.mark.parametrize("shape", [(256, 512, 512, 1536), (333, 272, 768, 384)])
+def test_mx_unfused_chain(shape):
+    """The comparison chain of the MXFP8 block (FP8 GEMM, add, RMSNorm with a
+    bf16 output, MXFP8 quantisation of y, block-scaled GEMM): the quantiser
+    fed the chain's own y is bit-exact, the last GEMM fed the chain's own
+    MXFP8 y is held to the bar (the step), and the whole chain against its
+    oracle (which rounds t, h and y to bf16 as the chain stores them)."""
+    M, K, N, N2 = shape
+    inp = synth.tiny_block() if shape == (256, 512, 512, 1536) else \
+        synth.block_inputs(M, K, N, N2, seed=95 + M, w_std=0.04)
+    gpu, ora = _mx_inputs(inp)
+    res, gamma = O.bf16_to_f64(b(inp.res)), O.bf16_to_f64(b(inp.gamma))
+    u = C.unfused_block_mx(gpu["x8"], gpu["sx"], gpu["W1t8"], gpu["sw1"], dev(inp.res), dev(inp.gamma),
+                           gpu["W2q"], gpu["W2sf"], inp.eps)
+    C.poll_status()
+    ref = MX.rmsnorm_block_mx_unfused(ora["x8"], ora["sx"], ora["W1t8"], ora["sw1"], res, gamma, ora["W2q"],
+                                      ora["W2e"], inp.eps)
+    check("t", u["t"], ref["t"])
+    check("h", u["h"], ref["h"])
+    check_rel("r", u["r"], ref["r"], 1e-3)
+    check("y", u["y"], ref["y"])
+    yq, ye = MX.mx_quantize(u["y"].double().cpu().numpy())
+    np.testing.assert_array_equal(u["yq"].cpu().numpy(), yq)
+    np.testing.assert_array_equal(_exps(u["ysf"], M, N), ye)
+    step = MX.gemm_rowscale_partial_mx(yq, ye, ora["W2q"], ora["W2e"])
+    check("out (step)", u["out"], step["out"], strict=True)
+    check("out (chain)", u["out"], ref["out"])
+
+
 # ---------------------------------------------------------------- guard regions
 
 GUARD = 8192

@@ -182,3 +182,28 @@ def test_mx_block_first_gemm_matches_fp8_block_and_quantises_hg():
     e = int(MX.mx_exponent(np.array([np.abs(blk).max()]))[0])
     assert int(g["he"][4, 5]) == e
     assert np.array_equal(g["hq"][4, 160:192], F8.e4m3_encode(blk * 2.0 ** -e))
+
+
+def test_mx_unfused_chain_steps():
+    """The unfused MXFP8 chain: t, h and r as the FP8 chain's (the same
+    GEMM, add and norm), y rounded to bf16 (8 significant bits) from
+    gamma h r, then quantised block by block from its own values."""
+    rng = np.random.default_rng(13)
+    M, K, N, N2 = 7, 64, 128, 96
+    x8 = F8.e4m3_encode(rng.standard_normal((M, K)))
+    w8 = F8.e4m3_encode(rng.standard_normal((N, K)) * 4)
+    res = rng.standard_normal((M, N))
+    gamma = rng.uniform(0.5, 1.5, N)
+    w2q, w2e = MX.mx_quantize(rng.standard_normal((N2, N)) * 0.1)
+    u = MX.rmsnorm_block_mx_unfused(x8, 0.5, w8, 0.125, res, gamma, w2q, w2e, 1e-5)
+    f = F8.rmsnorm_block_fp8_unfused(x8, 0.5, w8, 0.125, res, gamma, 1.0, np.zeros((1, N), np.uint8), 1.0, 1e-5)
+    assert np.array_equal(u["t"], f["t"]) and np.array_equal(u["h"], f["h"])
+    assert np.allclose(u["r"], f["r"], rtol=1e-15)
+    y = u["y"]
+    m, _ = np.frexp(y)
+    assert np.all(np.abs(m * 256 - np.round(m * 256)) == 0)  # 8 significant bits
+    assert np.all(np.abs(y - f["y"]) <= 2.0 ** -8 * np.abs(f["y"]))
+    q, e = MX.mx_quantize(y)
+    assert np.array_equal(q, u["yq"]) and np.array_equal(e, u["ye"])
+    ref = _brute_gemm(u["yq"], u["ye"], w2q, w2e)
+    assert np.allclose(u["out"], ref, rtol=1e-12, atol=1e-300)
