@@ -829,10 +829,10 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
 
     # MXFP8 block: W2 quantised once (a weight), hg's scales formed by GEMM1's epilogue
     W2t_bf = W2.t().contiguous()
-    W2q, W2sf = C.mx_quantize(W2t_bf)
+    W2q, W2sf = C.mx_quantize(W2t_bf, C.MX_B)
     bmx = {"h": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
            "hq": torch.empty(M_TOK, D, dtype=torch.uint8, device=dev),
-           "hsf": torch.empty(C.mx_sf_bytes(M_TOK, D), dtype=torch.uint8, device=dev),
+           "hsf": torch.empty(C.mx_sf_bytes(M_TOK, D, C.MX_A), dtype=torch.uint8, device=dev),
            "partial": torch.empty(C.partial_cols(D), M_TOK, dtype=torch.float32, device=dev),
            "r": torch.empty(M_TOK, dtype=torch.float32, device=dev)}
 
@@ -840,7 +840,7 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
             "h": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
             "y": torch.empty(M_TOK, D, dtype=torch.bfloat16, device=dev),
             "yq": torch.empty(M_TOK, D, dtype=torch.uint8, device=dev),
-            "ysf": torch.empty(C.mx_sf_bytes(M_TOK, D), dtype=torch.uint8, device=dev),
+            "ysf": torch.empty(C.mx_sf_bytes(M_TOK, D, C.MX_A), dtype=torch.uint8, device=dev),
             "r": torch.empty(M_TOK, dtype=torch.float32, device=dev)}
 
     s_y = torch.ones(1, dtype=torch.float32, device=dev)
@@ -920,19 +920,22 @@ def time_path(C, synth, torch, dev, stream, flush, inp, x, W1, W2, W_down, gamma
               lambda: C.gemm_rowscale_partial_fp8(b8["hg8"], s_hg, W2t8, sw2, b8["partial"], D, EPS, out=out8,
                                                   r_out=b8["r"]),
               2.0 * M * D * N2, M * D + D * N2 + 2 * M * N2 + 4 * M * (D // 128) + 4 * M, dtype="e4m3")
-        sfa, sfb = C.mx_sf_bytes(M, D), C.mx_sf_bytes(N2, D)
+        # scale bytes: hg's written by GEMM1 (one per 32 elements); the images
+        # GEMM2 loads (A's half-used, B's four copies of each scale)
+        sfw, sfa, sfb = M * D // 32, C.mx_sf_bytes(M, D, C.MX_A), C.mx_sf_bytes(N2, D, C.MX_B)
         kloop("gemm_res_partialrms_mx (e4m3 GEMM1 + residual + partial RMS + MXFP8 hg)",
               "coda_gemm_res_partialrms_mx",
               lambda: C.gemm_res_partialrms_mx(x8, sx, W1t8, sw1, res_d, gamma, h_out=bmx["h"], hq_out=bmx["hq"],
                                                hsf_out=bmx["hsf"], partial_out=bmx["partial"]),
-              2.0 * M * D * D, M * D + D * D + 2 * 2 * M * D + M * D + sfa + 4 * M * (D // 128), dtype="e4m3")
+              2.0 * M * D * D, M * D + D * D + 2 * 2 * M * D + M * D + sfw + 4 * M * (D // 128), dtype="e4m3")
         kloop("gemm_rowscale_partial_mx (block-scaled GEMM2 + folded reduction + row scale)",
               "coda_gemm_rowscale_partial_mx",
               lambda: C.gemm_rowscale_partial_mx(bmx["hq"], bmx["hsf"], W2q, W2sf, bmx["partial"], D, EPS, out=out8,
                                                  r_out=bmx["r"]),
               2.0 * M * D * N2, M * D + sfa + D * N2 + sfb + 2 * M * N2 + 4 * M * (D // 128) + 4 * M, dtype="mxfp8")
         kloop("mx_quantize (W2 to MXFP8, once per weight update)", "coda_mx_quantize",
-              lambda: C.mx_quantize(W2t_bf, q_out=W2q, sf_out=W2sf), 0.0, 2 * N2 * D + N2 * D + sfb, bound="hbm")
+              lambda: C.mx_quantize(W2t_bf, C.MX_B, q_out=W2q, sf_out=W2sf), 0.0, 2 * N2 * D + N2 * D + sfb,
+              bound="hbm")
     del res_d, x8, W1t8, W2t8, b8, out8, out16, b16, bu8, W2t_bf, W2q, W2sf, bmx, bumx
 
     # QKV projection with RoPE in its epilogue (1B attention input: 32 q + 8 k + 8 v heads of 64)

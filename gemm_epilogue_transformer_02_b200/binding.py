@@ -77,8 +77,8 @@ _SIGS = {
     "coda_rmsnorm_block_host_workspace_size": (_SZ, [_I64, _I64, _I64, _I64]),
     "coda_rmsnorm_block_host": (_ST, [_P, _P, _P, _P, _P, _F, _P, _P, _SZ, _I64, _I64, _I64, _I64, _I64, _P]),
     "coda_unfused_rmsnorm_fp8": (_ST, [_P, _P, _F, _P, _P, _P, _P, _I64, _I64, _P]),
-    "coda_mx_sf_bytes": (_I64, [_I64, _I64]),
-    "coda_mx_quantize": (_ST, [_P, _I64, _I64, _P, _P, _P]),
+    "coda_mx_sf_bytes": (_I64, [_I64, _I64, ctypes.c_int]),
+    "coda_mx_quantize": (_ST, [_P, _I64, _I64, ctypes.c_int, _P, _P, _P]),
     "coda_gemm_res_partialrms_mx": (_ST, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "coda_gemm_rowscale_partial_mx": (_ST, [_P, _P, _P, _P, _P, _I64, _I64, _F, _P, _P, _I64, _I64, _I64, _P]),
 }
@@ -636,29 +636,34 @@ def unfused_block_fp8(x8, sx, W1t8, sw1, res, gamma, s_y, W2t8, sw2, eps: float,
 # ----------------------------------------------- block-scaled e4m3 (MXFP8)
 
 
-def mx_sf_bytes(rows: int, cols: int) -> int:
-    """Bytes of the tiled scale buffer of a [rows, cols] MXFP8 operand."""
-    n = load_library().coda_mx_sf_bytes(int(rows), int(cols))
+MX_A, MX_B = 0, 1  # scale layouts: the GEMM's left operand, its right operand (stored [N, K])
+
+
+def mx_sf_bytes(rows: int, cols: int, operand: int = MX_A) -> int:
+    """Bytes of the scale buffer of a [rows, cols] MXFP8 operand in the
+    layout of `operand` (MX_A or MX_B)."""
+    n = load_library().coda_mx_sf_bytes(int(rows), int(cols), int(operand))
     if n < 0:
-        raise ValueError(f"no MXFP8 layout for [{rows}, {cols}] (cols must be a multiple of 128)")
+        raise ValueError(f"no MXFP8 layout for [{rows}, {cols}], operand {operand} (cols must be a multiple of 128)")
     return n
 
 
-def mx_quantize(src, q_out=None, sf_out=None):
-    """MXFP8 codes of a bf16 [rows, cols] tensor, blocked along its rows.
-    Returns (codes uint8 [rows, cols], tiled scales uint8)."""
+def mx_quantize(src, operand: int = MX_A, q_out=None, sf_out=None):
+    """MXFP8 codes of a bf16 [rows, cols] tensor, blocked along its rows, with
+    its scales in the layout of `operand`.  Returns (codes uint8 [rows, cols],
+    scales uint8)."""
     rows, cols = src.shape
     _need(src, BF16, "src")
     q_out = _empty((rows, cols), U8, src) if q_out is None else q_out
-    sf_out = _empty((mx_sf_bytes(rows, cols),), U8, src) if sf_out is None else sf_out
-    _call("coda_mx_quantize", _ptr(src), rows, cols, _ptr(q_out), _ptr(sf_out), _stream())
+    sf_out = _empty((mx_sf_bytes(rows, cols, operand),), U8, src) if sf_out is None else sf_out
+    _call("coda_mx_quantize", _ptr(src), rows, cols, int(operand), _ptr(q_out), _ptr(sf_out), _stream())
     return q_out, sf_out
 
 
 def gemm_res_partialrms_mx(x8, sx, Wt8, sw, res, gamma, *, h=True, h_out=None, hq_out=None, hsf_out=None,
                            partial_out=None):
     """First GEMM of the MXFP8 block.  Returns (h bf16 or None, hg codes,
-    hg's tiled scales, partial [T, M])."""
+    hg's scales in the A layout, partial [T, M])."""
     M, K = x8.shape
     N = Wt8.shape[0]
     _need(x8, U8, "x8")
@@ -671,7 +676,7 @@ def gemm_res_partialrms_mx(x8, sx, Wt8, sw, res, gamma, *, h=True, h_out=None, h
     if h and h_out is None:
         h_out = _empty((M, N), BF16, x8)
     hq_out = _empty((M, N), U8, x8) if hq_out is None else hq_out
-    hsf_out = _empty((mx_sf_bytes(M, N),), U8, x8) if hsf_out is None else hsf_out
+    hsf_out = _empty((mx_sf_bytes(M, N, MX_A),), U8, x8) if hsf_out is None else hsf_out
     partial_out = _empty((partial_cols(N), M), F32, x8) if partial_out is None else partial_out
     _call("coda_gemm_res_partialrms_mx", _ptr(x8), _ptr(sx), _ptr(Wt8), _ptr(sw), _ptr(res), _ptr(gamma),
           _ptr(h_out if h else None), _ptr(hq_out), _ptr(hsf_out), _ptr(partial_out), M, N, K, _stream())
@@ -681,14 +686,14 @@ def gemm_res_partialrms_mx(x8, sx, Wt8, sw, res, gamma, *, h=True, h_out=None, h
 def gemm_rowscale_partial_mx(Aq, Asf, Wq, Wsf, partial=None, N_norm: int = 0, eps: float = 0.0, out=None,
                              r_out=None):
     """Second GEMM of the MXFP8 block: out = r * (A Wt^T) with block-scaled
-    operands, r from the partials (partial None: a plain MXFP8 GEMM, r = 1).
-    Returns (out bf16, r or None)."""
+    operands (Asf in the A layout, Wsf in the B layout), r from the partials
+    (partial None: a plain MXFP8 GEMM, r = 1).  Returns (out bf16, r or None)."""
     M, K = Aq.shape
     N = Wq.shape[0]
     _need(Aq, U8, "Aq")
     _need(Wq, U8, "Wq", (N, K))
-    _need(Asf, U8, "Asf", (mx_sf_bytes(M, K),))
-    _need(Wsf, U8, "Wsf", (mx_sf_bytes(N, K),))
+    _need(Asf, U8, "Asf", (mx_sf_bytes(M, K, MX_A),))
+    _need(Wsf, U8, "Wsf", (mx_sf_bytes(N, K, MX_B),))
     out = _empty((M, N), BF16, Aq) if out is None else out
     T = 0
     if partial is not None:
@@ -726,7 +731,7 @@ def unfused_block_mx(x8, sx, W1t8, sw1, res, gamma, W2q, W2sf, eps: float, out=N
     if r is None:
         r = _empty((M,), F32, x8)
     y = unfused_rmsnorm(h, gamma, eps, y_out=b.get("y"), r_out=r)
-    yq, ysf = mx_quantize(y, q_out=b.get("yq"), sf_out=b.get("ysf"))
+    yq, ysf = mx_quantize(y, MX_A, q_out=b.get("yq"), sf_out=b.get("ysf"))
     out, _ = gemm_rowscale_partial_mx(yq, ysf, W2q, W2sf, out=out)
     return {"out": out, "t": t, "h": h, "y": y, "yq": yq, "ysf": ysf, "r": r}
 

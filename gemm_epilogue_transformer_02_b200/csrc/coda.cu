@@ -19,7 +19,7 @@ namespace {
 using namespace coda;
 
 constexpr int64_t kPartialTile = 128;  // columns per partial sum: one half of a 256-column tile
-constexpr int kVersion = 2;  // 2: partial sums per 128-column slot
+constexpr int kVersion = 3;  // 2: partial sums per 128-column slot; 3: the MXFP8 calls
 
 int64_t g_wait_ns = 1000000000LL;
 
@@ -140,8 +140,8 @@ bool tmap2d_u8_plain(CUtensorMap* m, const void* base, uint64_t cols, uint64_t r
   return r == CUDA_SUCCESS;
 }
 
-// Scale bytes of a block-scaled operand: the tiled layout seen as rows of 128
-// 32-bit words (one 512-byte atom per row), `box_rows` atoms per copy.
+// Scale bytes of a block-scaled operand seen as rows of 128 32-bit words
+// (512 bytes), `box_rows` rows per copy.
 bool tmap_sf(CUtensorMap* m, const void* base, uint64_t atoms, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
@@ -1422,19 +1422,21 @@ coda_status_t coda_gemm_fp8(const uint8_t* A8, const float* sa, const uint8_t* W
 
 // ------------------------------------------------ block-scaled e4m3 (MXFP8)
 
-int64_t coda_mx_sf_bytes(int64_t rows, int64_t cols) {
-  if (rows < 0 || cols < 0 || cols % 128 != 0) return -1;
-  return (cols / 128) * ((rows + 127) / 128) * 512;
+int64_t coda_mx_sf_bytes(int64_t rows, int64_t cols, int operand) {
+  if (rows < 0 || cols < 0 || cols % 128 != 0 || (operand != 0 && operand != 1)) return -1;
+  const int64_t nkb = cols / 128;
+  // A: a 512-byte atom per (k-block, 128-row block); B: a 4 KB image per (k-block, 256-row tile)
+  return operand == 0 ? nkb * ((rows + 127) / 128) * 512 : nkb * ((rows + 255) / 256) * 4096;
 }
 
 namespace {
 inline bool mx_dim_ok(int64_t v) { return dim_ok(v) && v % 128 == 0; }
 }  // namespace
 
-coda_status_t coda_mx_quantize(const uint16_t* src, int64_t rows, int64_t cols, uint8_t* q_out, uint8_t* sf_out,
-                               void* stream) {
-  CODA_CHECK(rows >= 0 && rows < (int64_t(1) << 31) && mx_dim_ok(cols) &&
-                 (rows + 127) / 128 * 128 * (cols / 32) < (int64_t(1) << 40),
+coda_status_t coda_mx_quantize(const uint16_t* src, int64_t rows, int64_t cols, int operand, uint8_t* q_out,
+                               uint8_t* sf_out, void* stream) {
+  CODA_CHECK(rows >= 0 && rows < (int64_t(1) << 30) && mx_dim_ok(cols) && (operand == 0 || operand == 1) &&
+                 (rows + 255) / 256 * 256 * (cols / 32) < (int64_t(1) << 40),
              CODA_ERR_SHAPE);
   if (rows == 0) return CODA_OK;
   CODA_CHECK(src && q_out && sf_out, CODA_ERR_NULL);
@@ -1446,7 +1448,8 @@ coda_status_t coda_mx_quantize(const uint16_t* src, int64_t rows, int64_t cols, 
     if (ds != CODA_OK) return ds;
   }
   mx_quantize_kernel<<<info->sms * 4, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const __nv_bfloat16*>(src), static_cast<int>(rows), static_cast<int>(cols), q_out, sf_out);
+      reinterpret_cast<const __nv_bfloat16*>(src), static_cast<int>(rows), static_cast<int>(cols), operand, q_out,
+      sf_out);
   return cudaGetLastError() == cudaSuccess ? CODA_OK : CODA_ERR_LAUNCH;
 }
 
@@ -1509,13 +1512,14 @@ coda_status_t coda_gemm_rowscale_partial_mx(const uint8_t* Aq, const uint8_t* As
   }
   using Epi = EpiRowScaleMX;
   GemmParams<Epi> p{};
-  const int64_t rba = (M + 127) / 128, rbb = N / 128, nkb = K / 128;
+  // scales as rows of 512 bytes: A's atoms (one row each), B's 4 KB images (8 rows)
+  const int64_t rba = (M + 127) / 128, ntl = (N + 255) / 256, nkb = K / 128;
   if (!(tmap2d_u8(&p.tmA, Aq, K, M, K, 128, kBM) && tmap2d_u8(&p.tmB, Wq, K, N, K, 128, 128) &&
         tmap_sf(&p.tmSFA, Asf, static_cast<uint64_t>(nkb * rba), 1) &&
-        tmap_sf(&p.tmSFB, Wsf, static_cast<uint64_t>(nkb * rbb), 2) && map_out_bf16(&p.ep.tmOut, out, M, N, N)))
+        tmap_sf(&p.tmSFB, Wsf, static_cast<uint64_t>(nkb * ntl * 8), 8) && map_out_bf16(&p.ep.tmOut, out, M, N, N)))
     return CODA_ERR_INTERNAL;
   p.sf_rba = static_cast<int>(rba);
-  p.sf_rbb = static_cast<int>(rbb);
+  p.sf_ntl = static_cast<int>(ntl);
   p.ep.partial = partial;
   p.ep.T = static_cast<int>(T);
   p.ep.inv_n = partial ? 1.0f / static_cast<float>(N_norm) : 1.0f;

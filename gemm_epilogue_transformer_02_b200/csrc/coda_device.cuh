@@ -400,16 +400,23 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
 //
 // tcgen05.mma kind::mxf8f6f4.block_scale multiplies e4m3 operands whose K
 // runs in blocks of 32 elements, each block with an E8M0 scale (a power of
-// two, byte = exponent + 127).  The scales are read from tensor memory: a
-// 128-row group's scales for one 128-wide k-block are a 512-byte atom whose
-// byte (i % 32) * 16 + ((i / 32) % 4) * 4 + b holds row i's scale of K block
-// b (b = 0..3, one per 32-wide MMA step); tcgen05.cp copies the atom, as 32
-// rows of 16 bytes, into 32 lanes x 4 columns of every lane quarter, and the
-// MMA's instruction descriptor selects the byte b of each 32-bit word.
+// two, byte = exponent + 127).  The scales are read from tensor memory, four
+// to a 32-bit word (one per 32-wide MMA step of a 128-wide k-block, selected
+// by the instruction descriptor):
+//   A (rows m of the tile's 128 per CTA): lane quarter q = m / 32 reads the
+//     word of row m from its own lane m at column base + q;
+//   B (all N rows of the tile): every lane quarter reads row n's word at
+//     column base + n / 32 of its lane 32 q + n % 32.
+// A's 128 rows come as one 512-byte atom per k-block (32 rows of 16 bytes:
+// row r holds the words of rows r, r + 32, r + 64, r + 96), copied by
+// tcgen05.cp .32x128b.warpx4 into every lane quarter; B's 256 rows as one
+// 4 KB image per k-block (each of its two atoms four times), copied by one
+// .128x256b, so that every lane of every quarter holds the words of rows
+// r + 32 c (c = 0..7) of the tile -- one copy instead of two.
 
 // Shared-memory descriptor of an unswizzled, K-major matrix of 16-byte rows
-// (the source of tcgen05.cp): rows 16 bytes apart, so its eight-row core
-// matrices sit 128 bytes apart (stride byte offset); layout type 0 (no
+// (the source of a .32x128b copy): rows 16 bytes apart, so its eight-row
+// core matrices sit 128 bytes apart (stride byte offset); layout type 0 (no
 // swizzle) in bits 61-63, descriptor version 1 in bits 46-47.  The leading
 // byte offset is unused by a matrix one core matrix wide.
 __device__ __forceinline__ uint64_t sdesc_plain16(uint32_t saddr) {
@@ -428,6 +435,27 @@ __device__ __forceinline__ uint64_t sdesc_plain16(uint32_t saddr) {
 // them and tracked by the same tcgen05.commit.
 __device__ __forceinline__ void tc_cp_32x128_w4_pair(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of the source of a .128x256b copy: an unswizzled
+// K-major image of 128 rows x 32 bytes whose first 16 bytes of every row
+// form a 2 KB block (rows 16 bytes apart, eight-row core matrices 128 bytes
+// apart: stride byte offset) and whose second 16 bytes form the next 2 KB
+// block (leading byte offset 2048); layout type 0 (no swizzle) in bits
+// 61-63, descriptor version 1 in bits 46-47.
+__device__ __forceinline__ uint64_t sdesc_sf_image(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(2048 >> 4) << 16;
+  d |= static_cast<uint64_t>(128 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// Copy a 128-row x 32-byte image from shared memory into tensor memory at
+// taddr (128 lanes x 8 columns); otherwise as tc_cp_32x128_w4_pair.
+__device__ __forceinline__ void tc_cp_128x256_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // Instruction descriptor of kind::mxf8f6f4 block-scaled: E4M3 A and B (format
@@ -469,11 +497,25 @@ __device__ __forceinline__ int mx_e4m3_exponent(float amax) {
 // 2^-e as an fp32 value (-127 <= e <= 126; finite fp32 data gives e <= 120).
 __device__ __forceinline__ float exp2_neg(int e) { return __uint_as_float(static_cast<uint32_t>(127 - e) << 23); }
 
-// Byte offset of the scale of row i, 32-element K block j, in the tiled scale
-// layout of an operand with `nrb` 128-row blocks: one 512-byte atom per
-// (128-wide k-block, 128-row block), k-blocks outermost.
-__host__ __device__ __forceinline__ size_t mx_sf_offset(int i, int j, int nrb) {
+// Scale layouts in global memory.
+//
+// A layout: one 512-byte atom per (128-wide k-block, 128-row block), k-blocks
+// outermost (nrb row blocks); row i's scale of 32-element K block j at
+// (i % 32) * 16 + ((i / 32) % 4) * 4 + j % 4 within atom (j / 4) * nrb + i / 128.
+__host__ __device__ __forceinline__ size_t mx_sf_offset_a(int i, int j, int nrb) {
   return ((static_cast<size_t>(j >> 2) * nrb + (i >> 7)) << 9) + ((i & 31) << 4) + (((i >> 5) & 3) << 2) + (j & 3);
+}
+
+// B layout: one 4 KB image per (k-block kb, 256-row tile t), images ordered
+// kb-major (ntl tiles), the source of one .128x256b copy (bytes 0-2047: the
+// first 16 bytes of its 128 rows, the tile's first atom four times; bytes
+// 2048-4095: the second 16 bytes, its second atom four times); row i's
+// scale of block j sits, four times (rep = 0..3), at ((i / 128) % 2) * 2048 +
+// rep * 512 + (i % 32) * 16 + ((i / 32) % 4) * 4 + j % 4.  This returns the
+// rep = 0 copy.
+__host__ __device__ __forceinline__ size_t mx_sf_offset_b(int i, int j, int ntl) {
+  return ((static_cast<size_t>(j >> 2) * ntl + (i >> 8)) << 12) + (((i >> 7) & 1) << 11) + ((i & 31) << 4) +
+         (((i >> 5) & 3) << 2) + (j & 3);
 }
 
 // ------------------------------------------- cross-CTA completion counters

@@ -128,11 +128,12 @@ struct epi_ksplit<E, decltype(void(E::kSplitK))> {
 
 // Epilogues that declare kMX = true take block-scaled e4m3 operands
 // (MXFP8: kind::mxf8f6f4.block_scale, an E8M0 scale per 32 elements of K,
-// loaded with each k-block and copied into tensor memory beside the
-// accumulator).  The scales take tensor-memory columns, so the tile keeps
-// one 256-column accumulator instead of two; the epilogue frees it as soon
-// as it has read it (arriving on TileCtx::trel itself) and writes the tile
-// out while the next tile's MMAs run.
+// loaded with every k-block -- A's as a 512-byte atom, B's as a 4 KB copy
+// image -- and copied into tensor memory beside the accumulator).  The
+// scales take tensor-memory columns, so the tile keeps one 256-column
+// accumulator instead of two; the epilogue frees it as soon as it has read
+// it (arriving on TileCtx::trel itself) and writes the tile out while the
+// next tile's MMAs run.
 template <class E, class = void>
 struct epi_mx {
   static constexpr bool value = false;
@@ -171,13 +172,12 @@ struct GemmParams {
   // global read, until the previous grid has completed and its writes are
   // visible (a hardware dependency, like stream order).
   int pdl_trigger, pdl_wait;
-  // Block-scaled operands: the tiled scale bytes of A and B seen as rows of
-  // 128 words (one 512-byte atom per row: atom row kb * sf_rb + row block),
-  // boxes of one (A: this CTA's 128 rows) and two atoms (B: the tile's 256
-  // columns).
+  // Block-scaled operands: the scales of A and B seen as rows of 128 words
+  // (512 bytes): A's atom kb * sf_rba + this CTA's row block (one row), B's
+  // image kb * sf_ntl + the tile's column block (4 KB = 8 rows).
   CUtensorMap tmSFA;
   CUtensorMap tmSFB;
-  int sf_rba, sf_rbb;  // 128-row blocks of A and of B
+  int sf_rba, sf_ntl;  // 128-row blocks of A; 256-row tiles of B
 };
 
 // Per-warp context handed to the epilogue for one tile.
@@ -218,8 +218,8 @@ struct GemmSmem {
   static constexpr int kEpiBytes = kEW * Epi::kSmemPerWarp;
   static constexpr bool kHalfXchg = kEW == 8 && epi_split<Epi>::value;  // see TileCtx::xchg
   static constexpr int kXchgBytes = kHalfXchg ? 4 * 32 * 4 : 0;
-  // block-scaled operands: per stage this CTA's A-scale atom and the tile's two B-scale atoms
-  static constexpr int kSFStage = epi_mx<Epi>::value ? 3 * 512 : 0;
+  // block-scaled operands: per stage this CTA's A-scale atom and the tile's B-scale image
+  static constexpr int kSFStage = epi_mx<Epi>::value ? 512 + 4096 : 0;
   static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1 + kEW * Epi::kBarsPerWarp + (kHalfXchg ? 4 : 0);
   static constexpr int kBytes = 1024 /*align slack*/ + STAGES * kStageBytes + kEpiBytes + STAGES * kSFStage +
                                 kXchgBytes + kNumBars * 8 + 16;
@@ -388,10 +388,10 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
                 tma_load_2d_pair(b + j * (64 * kBK * 2), &p.tmB, fb, bcol + j * 64, kb * kBK);
             }
             if (kMX) {
-              // the scales of this k-block: this CTA's 128 rows of A, all 256 columns of B
+              // the scales of this k-block: this CTA's 128 rows of A, the tile's 256 columns of B
               uint8_t* sf = sSF + stage * S::kSFStage;
               tma_load_2d_pair(sf, &p.tmSFA, fb, 0, kb * p.sf_rba + mb * 2 + static_cast<int>(rank));
-              tma_load_2d_pair(sf + 512, &p.tmSFB, fb, 0, kb * p.sf_rbb + nb * 2);
+              tma_load_2d_pair(sf + 512, &p.tmSFB, fb, 0, (kb * p.sf_ntl + nb) * 8);
             }
           } else {
             mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
@@ -475,13 +475,12 @@ __global__ void __launch_bounds__(64 + 32 * epi_warps<Epi>::value, 1)
           const uint32_t a0 = smem_u32(sA + stage * S::kABytes);
           const uint32_t b0 = smem_u32(sB + stage * S::kBBytes);
           // block-scaled: this stage's scales go to 16 tensor-memory columns of
-          // their own (A's atom at +0, B's two atoms at +8 and +12)
+          // their own (A's atom at +0, B's image at +8)
           const uint32_t tsf = tmem_base + kSFCol + static_cast<uint32_t>(stage) * 16u;
           if (kMX) {
             const uint32_t sf = smem_u32(sSF + stage * S::kSFStage);
             tc_cp_32x128_w4_pair(tsf, sdesc_plain16(sf));
-            tc_cp_32x128_w4_pair(tsf + 8, sdesc_plain16(sf + 512));
-            tc_cp_32x128_w4_pair(tsf + 12, sdesc_plain16(sf + 1024));
+            tc_cp_128x256_pair(tsf + 8, sdesc_sf_image(sf + 512));
           }
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
@@ -642,7 +641,7 @@ __device__ __forceinline__ float acc_at(const uint32_t (&v0)[32], const uint32_t
 //     h and partial as MODE 2; out2 = hg in MXFP8: each 32-column block of
 //     gamma * h gets the smallest power-of-two scale 2^e that keeps it within
 //     the e4m3 range, its codes are e4m3(gamma * h * 2^-e) and the byte e + 127
-//     goes to the tiled scale layout (sf_out) -- the scales of the data being
+//     goes to the A scale layout (sf_out) -- the scales of the data being
 //     written, in the epilogue, with no scale carried over between calls
 // The input tile is read straight into registers (each thread its own row)
 // 32 columns ahead, and the first columns of the next tile are requested
@@ -692,7 +691,7 @@ struct EpiLoadStore2 {
     const float* sb;
     const float* s_out;          // MODE 2: scale hg8 is quantised with
     unsigned* amax;              // MODE 2: running max |hg| (fp32 bits; zeroed by the caller)
-    uint8_t* sf_out;             // MODE 3: hg's scale bytes, tiled (N % 128 == 0)
+    uint8_t* sf_out;             // MODE 3: hg's scale bytes, A layout (N % 128 == 0)
     int sf_rb;                   // MODE 3: 128-row blocks of that layout (ceil(M / 128))
   };
 
@@ -819,7 +818,7 @@ struct EpiLoadStore2 {
           st_shared_v4(G + sw128_off(c.lane, (ch & 1) * 4 + 2 * hh + 1), u1);
         }
         if (row < ep.sf_rb * 128)  // rows past M (zero) get e = 0: scale 1, as padding
-          ep.sf_out[mx_sf_offset(row, (cc + hh * 32) >> 5, ep.sf_rb)] = static_cast<uint8_t>(ex + 127);
+          ep.sf_out[mx_sf_offset_a(row, (cc + hh * 32) >> 5, ep.sf_rb)] = static_cast<uint8_t>(ex + 127);
         continue;
       }
 #pragma unroll

@@ -415,13 +415,16 @@ __global__ void __launch_bounds__(256) quantize_e4m3_kernel(const __nv_bfloat16*
 // blocked along the row: each thread takes one 32-element block, finds its
 // largest magnitude, takes the smallest power-of-two scale 2^e that keeps it
 // within the e4m3 range and writes the 32 codes of v * 2^-e (round to nearest
-// even) and the E8M0 byte e + 127 into the tiled scale layout.  Scale bytes of
-// the padding rows (up to a whole 128-row block) are set to 127 (scale 1).
+// even) and the E8M0 byte e + 127 into the A or the B scale layout (b_layout;
+// B's bytes four times).  Scale bytes of the padding rows (up to a whole
+// 128-row block for A, a whole 256-row tile for B) are set to 127 (scale 1).
 __global__ void __launch_bounds__(256) mx_quantize_kernel(const __nv_bfloat16* __restrict__ src, int rows, int cols,
-                                                          uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+                                                          int b_layout, uint8_t* __restrict__ q,
+                                                          uint8_t* __restrict__ sf) {
   const int nb = cols >> 5;
   const int nrb = (rows + 127) >> 7;
-  const size_t total = static_cast<size_t>(nrb) * 128 * nb;
+  const int ntl = (rows + 255) >> 8;
+  const size_t total = static_cast<size_t>(b_layout ? ntl * 2 : nrb) * 128 * nb;
   for (size_t t = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; t < total;
        t += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const int row = static_cast<int>(t / nb);
@@ -456,7 +459,14 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const __nv_bfloat16* _
       d[0] = make_uint4(out[0], out[1], out[2], out[3]);
       d[1] = make_uint4(out[4], out[5], out[6], out[7]);
     }
-    sf[mx_sf_offset(row, j, nrb)] = static_cast<uint8_t>(e + 127);
+    const uint8_t byte = static_cast<uint8_t>(e + 127);
+    if (b_layout) {
+      const size_t o = mx_sf_offset_b(row, j, ntl);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) sf[o + r * 512] = byte;
+    } else {
+      sf[mx_sf_offset_a(row, j, nrb)] = byte;
+    }
   }
 }
 

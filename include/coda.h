@@ -433,29 +433,40 @@ coda_status_t coda_unfused_rmsnorm_fp8(const uint16_t* h, const uint16_t* gamma,
  * [-127, 127]; an all-zero block takes e = 0.  The scales replace the FP8
  * block's per-tensor scale of hg, which had to come from an earlier call.
  *
- * Scale layout ("tiled"): for an operand of R rows and K columns (K a
- * multiple of 128), with nrb = ceil(R / 128), the scale of row i, 32-element
- * block j sits at byte ((j / 4) * nrb + i / 128) * 512 + (i % 32) * 16 +
- * ((i / 32) % 4) * 4 + j % 4: one 512-byte atom per (128-wide k-block,
- * 128-row block), k-blocks outermost, which the GEMM copies into tensor
- * memory as it is.  Padding rows (R up to 128 nrb) hold 127.
- * coda_mx_sf_bytes(R, K) = (K / 128) * nrb * 512 (-1 for a bad shape). */
-int64_t coda_mx_sf_bytes(int64_t rows, int64_t cols);
+ * Scale layouts (nkb = K / 128 k-blocks for an operand of R rows and K
+ * columns, K a multiple of 128; E(i, j) = the byte of row i, 32-element
+ * block j, whose k-block is kb = j / 4 and step s = j % 4).  Which layout an
+ * operand takes depends on its side of the GEMM:
+ *   operand 0, the left operand A: one 512-byte atom per (k-block, 128-row
+ *     block), atoms kb-major (nrb = ceil(R / 128) row blocks); E(i, j) at
+ *     (kb * nrb + i / 128) * 512 + (i % 32) * 16 + ((i / 32) % 4) * 4 + s.
+ *   operand 1, the right operand B (stored [N, K]): one 4 KB image per
+ *     (k-block, 256-row tile), images kb-major (ntl = ceil(R / 256) tiles),
+ *     each tile's two atoms four times over, so that the GEMM copies the
+ *     image into tensor memory at once; E(i, j) at (kb * ntl + i / 256) *
+ *     4096 + ((i / 128) % 2) * 2048 + rep * 512 + (i % 32) * 16 +
+ *     ((i / 32) % 4) * 4 + s for each rep = 0..3.
+ * Padding rows (up to whole row blocks / tiles) hold 127.
+ * coda_mx_sf_bytes(R, K, operand) = nkb * nrb * 512 (A) or nkb * ntl * 4096
+ * (B); -1 for a bad shape or operand. */
+int64_t coda_mx_sf_bytes(int64_t rows, int64_t cols, int operand);
 
 /* MXFP8 codes of a row-major bf16 matrix src [rows, cols], blocked along
- * each row: q_out [rows, cols] e4m3, sf_out the tiled scales
- * (coda_mx_sf_bytes(rows, cols) bytes, every byte written).  cols % 128 == 0.
- * Used for the weight W2 stored transposed ([N2, N], K-major). */
-coda_status_t coda_mx_quantize(const uint16_t* src, int64_t rows, int64_t cols, uint8_t* q_out, uint8_t* sf_out,
-                               void* stream);
+ * each row: q_out [rows, cols] e4m3, sf_out the scales in the layout of
+ * `operand` (0: A, 1: B; coda_mx_sf_bytes(rows, cols, operand) bytes, every
+ * byte written).  cols % 128 == 0.  Used for the weight W2
+ * stored transposed ([N2, N], operand 1) and for the unfused chain's y
+ * (operand 0). */
+coda_status_t coda_mx_quantize(const uint16_t* src, int64_t rows, int64_t cols, int operand, uint8_t* q_out,
+                               uint8_t* sf_out, void* stream);
 
 /* First GEMM of the MXFP8 block: as coda_gemm_res_partialrms_fp8 (e4m3 x8
  * [M, K] and Wt8 [N, K] with per-tensor scales sx, sw; h = acc * sx * sw +
  * res; partial[t, i] over 128-column slots; h_out bf16 or NULL), except that
  * hg = gamma * h is written in MXFP8 from the epilogue: hq_out [M, N] e4m3
- * codes and hsf_out its tiled scales (coda_mx_sf_bytes(M, N) bytes; each
- * 32-column block of a row quantised from the fp32 values as they are
- * formed).  N a multiple of 128, K of 16. */
+ * codes and hsf_out its scales in the A layout (coda_mx_sf_bytes(M, N, 0)
+ * bytes; each 32-column block of a row quantised from the fp32 values as
+ * they are formed).  N a multiple of 128, K of 16. */
 coda_status_t coda_gemm_res_partialrms_mx(const uint8_t* x8, const float* sx, const uint8_t* Wt8, const float* sw,
                                           const uint16_t* res, const uint16_t* gamma, uint16_t* h_out,
                                           uint8_t* hq_out, uint8_t* hsf_out, float* partial, int64_t M, int64_t N,
@@ -466,9 +477,10 @@ coda_status_t coda_gemm_res_partialrms_mx(const uint8_t* x8, const float* sx, co
  * coda_gemm_rowscale_partial: r_i = 1/sqrt(sum_t partial[t, i] / N_norm +
  * eps), out = bf16(r_i * acc_ij), r_out [M] or NULL.  partial == NULL gives
  * a plain MXFP8 GEMM (r = 1; T, N_norm, eps, r_out ignored).  Aq [M, K] with
- * tiled scales Asf, Wq [N, K] (W2 transposed) with tiled scales Wsf; out
- * [M, N] bf16.  N and K multiples of 128.  Launched with programmatic stream
- * serialisation after coda_gemm_res_partialrms_mx, as the FP8 pair. */
+ * scales Asf in the A layout, Wq [N, K] (W2 transposed) with scales Wsf in
+ * the B layout; out [M, N] bf16.  N and K multiples of 128.  Launched with
+ * programmatic stream serialisation after coda_gemm_res_partialrms_mx, as
+ * the FP8 pair. */
 coda_status_t coda_gemm_rowscale_partial_mx(const uint8_t* Aq, const uint8_t* Asf, const uint8_t* Wq,
                                             const uint8_t* Wsf, const float* partial, int64_t T, int64_t N_norm,
                                             float eps, float* r_out, uint16_t* out, int64_t M, int64_t N, int64_t K,

@@ -25,12 +25,14 @@ the design notes):
   is exact, so the only rounding is the e4m3 one.
 * Both GEMM operands are K-major and block-scaled along K: A [M, K] with
   scales [M, K/32], B stored as Bt [N, K] with scales [N, K/32].
-* The scales travel in a tiled byte layout (the library's header states it):
-  for 32-block j of row i, with R rows padded to whole 128-row blocks
-  (nrb = ceil(R / 128) row blocks), the byte sits at
-  ((j // 4) nrb + i // 128) 512 + (i % 32) 16 + ((i // 32) % 4) 4 + j % 4,
-  i.e. one 512-byte atom per (128-row block, 128-column block), k-blocks
-  outermost; bytes of padding rows hold 127 (scale 1).
+* The scales travel in one of two byte layouts (the library's header states
+  them): operand 0, the GEMM's left operand A (rows i, nrb = ceil(R / 128)
+  row blocks): one 512-byte atom per (k-block, row block), E(i, j) at
+  ((j // 4) nrb + i // 128) 512 + (i % 32) 16 + ((i // 32) % 4) 4 + j % 4;
+  operand 1, the right operand B (ntl = ceil(R / 256) tiles): one 4 KB image
+  per (k-block, 256-row tile), E(i, j) four times at ((j // 4) ntl + i // 256)
+  4096 + ((i // 128) % 2) 2048 + rep 512 + (i % 32) 16 + ((i // 32) % 4) 4 +
+  j % 4, rep = 0..3.  Bytes of padding rows hold 127 (scale 1).
 * The block: the first GEMM keeps the per-tensor e4m3 operands of the FP8
   block; its epilogue forms hg = gamma h in full precision and quantises it
   into MXFP8 itself, block by block, so hg's scales are those of the data
@@ -93,40 +95,56 @@ def mx_dequantize(codes, exps) -> np.ndarray:
     return (vals * np.ldexp(1.0, exps)[:, :, None]).reshape(R, K)
 
 
-def sf_rows_padded(R: int) -> int:
-    return -(-R // 128) * 128
+def sf_rows_padded(R: int, operand: int = 0) -> int:
+    """Rows the layout holds: whole 128-row blocks (A) or 256-row tiles (B)."""
+    unit = 128 if operand == 0 else 256
+    return -(-R // unit) * unit
 
 
-def sf_bytes(R: int, K: int) -> int:
-    """Size of the tiled scale buffer of an [R, K] operand."""
-    return (K // 128) * (sf_rows_padded(R) // 128) * 512
+def sf_bytes(R: int, K: int, operand: int = 0) -> int:
+    """Size of the scale buffer of an [R, K] operand."""
+    nkb = K // 128
+    if operand == 0:
+        return nkb * (sf_rows_padded(R, 0) // 128) * 512
+    return nkb * (sf_rows_padded(R, 1) // 256) * 4096
 
 
-def sf_offset(i: int, j: int, R: int) -> int:
-    """Byte offset of the scale of row i, 32-block j, in the tiled layout."""
-    nrb = sf_rows_padded(R) // 128
-    return ((j // 4) * nrb + i // 128) * 512 + (i % 32) * 16 + ((i // 32) % 4) * 4 + j % 4
+def sf_offsets(i: int, j: int, R: int, operand: int = 0) -> list:
+    """Byte offsets of the scale of row i, 32-block j (one for A, four for B)."""
+    kb, s = j // 4, j % 4
+    within = (i % 32) * 16 + ((i // 32) % 4) * 4 + s
+    if operand == 0:
+        nrb = sf_rows_padded(R, 0) // 128
+        return [(kb * nrb + i // 128) * 512 + within]
+    ntl = sf_rows_padded(R, 1) // 256
+    base = (kb * ntl + i // 256) * 4096 + ((i // 128) % 2) * 2048 + within
+    return [base + rep * 512 for rep in range(4)]
 
 
-def sf_tile(exps, R: int) -> np.ndarray:
-    """Tiled E8M0 bytes of exponents [R, K/32] (padding rows: 127)."""
+def sf_tile(exps, R: int, operand: int = 0):
+    """E8M0 bytes of exponents [R, K/32] in the layout, and the mask of the
+    bytes it defines (all of them; padding rows hold 127)."""
     exps = np.asarray(exps, dtype=np.int64)
     nblk = exps.shape[1]
     assert nblk % 4 == 0
-    buf = np.full(sf_bytes(R, nblk * MX_BLOCK), 127, dtype=np.uint8)
-    for i in range(R):
+    size = sf_bytes(R, nblk * MX_BLOCK, operand)
+    buf = np.full(size, 127, dtype=np.uint8)
+    used = np.zeros(size, dtype=bool)
+    for i in range(sf_rows_padded(R, operand)):
         for j in range(nblk):
-            buf[sf_offset(i, j, R)] = exps[i, j] + 127
-    return buf
+            for o in sf_offsets(i, j, R, operand):
+                buf[o] = exps[i, j] + 127 if i < R else 127
+                used[o] = True
+    return buf, used
 
 
-def sf_untile(buf, R: int, K: int) -> np.ndarray:
-    """Exponents [R, K/32] read back from the tiled bytes."""
+def sf_untile(buf, R: int, K: int, operand: int = 0) -> np.ndarray:
+    """Exponents [R, K/32] read back from the layout (the first copy)."""
     buf = np.asarray(buf, dtype=np.uint8).reshape(-1)
     out = np.empty((R, K // MX_BLOCK), dtype=np.int32)
     for i in range(R):
         for j in range(K // MX_BLOCK):
-            out[i, j] = int(buf[sf_offset(i, j, R)]) - 127
+            out[i, j] = int(buf[sf_offsets(i, j, R, operand)[0]]) - 127
     return out
 
 

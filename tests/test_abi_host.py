@@ -191,16 +191,20 @@ def test_argument_errors_of_the_remaining_calls(lib):
     assert u8(A, B, 1e-6, None, D, A, None, 16, 64, None) == NULL  # s_y
     assert u8(A, B, 1e-6, C, D, A, MIS, 16, 64, None) == ALIGN     # r_out
 
-    # MXFP8: the scale layout's size, and the calls' argument checks
-    assert lib.coda_mx_sf_bytes(300, 256) == 2 * 3 * 512
-    assert lib.coda_mx_sf_bytes(1, 128) == 512
-    assert lib.coda_mx_sf_bytes(16, 96) == -1            # cols not a multiple of 128
-    assert lib.coda_mx_sf_bytes(-1, 128) == -1
-    mq = lib.coda_mx_quantize  # (src, rows, cols, q, sf, stream)
-    assert mq(A, 16, 192, B, C, None) == SHAPE
-    assert mq(A, 16, 128, None, C, None) == NULL
-    assert mq(A, 16, 128, B, MIS, None) == ALIGN
-    assert mq(A, 0, 128, B, C, None) == OK
+    # MXFP8: the scale layouts' sizes, and the calls' argument checks
+    assert lib.coda_mx_sf_bytes(300, 1024, 0) == 8 * 3 * 512      # A: k-blocks x row blocks x 512-byte atoms
+    assert lib.coda_mx_sf_bytes(300, 1152, 0) == 9 * 3 * 512
+    assert lib.coda_mx_sf_bytes(300, 256, 1) == 2 * 2 * 4096      # B: k-blocks x 256-row tiles
+    assert lib.coda_mx_sf_bytes(1, 128, 1) == 4096
+    assert lib.coda_mx_sf_bytes(16, 96, 0) == -1            # cols not a multiple of 128
+    assert lib.coda_mx_sf_bytes(-1, 128, 0) == -1
+    assert lib.coda_mx_sf_bytes(16, 128, 2) == -1           # no such operand
+    mq = lib.coda_mx_quantize  # (src, rows, cols, operand, q, sf, stream)
+    assert mq(A, 16, 192, 0, B, C, None) == SHAPE
+    assert mq(A, 16, 128, 2, B, C, None) == SHAPE
+    assert mq(A, 16, 128, 1, None, C, None) == NULL
+    assert mq(A, 16, 128, 0, B, MIS, None) == ALIGN
+    assert mq(A, 0, 128, 0, B, C, None) == OK
     pm = lib.coda_gemm_res_partialrms_mx  # (x8, sx, Wt8, sw, res, gamma, h, hq, hsf, partial, M, N, K, s)
     assert pm(A, B, C, D, None, A, None, B, C, D, 16, 192, 64, None) == SHAPE  # N not a multiple of 128
     assert pm(A, B, C, D, None, A, None, B, C, D, 16, 256, 40, None) == SHAPE  # K not a multiple of 16
@@ -223,7 +227,7 @@ def test_valid_arguments_without_a_gpu_report_device_error(lib):
     assert lib.coda_rms_reduce(A, 16, 1, 64, 1e-6, B, None) == DEVICE
     assert lib.coda_fp8_quantize(A, 16, 16, 1, B, C, D, None) == DEVICE
     assert lib.coda_gemm_rowscale_partial_fp8(A, B, C, D, A, 1, 64, 1e-6, None, B, 16, 64, 64, None) == DEVICE
-    assert lib.coda_mx_quantize(A, 16, 128, B, C, None) == DEVICE
+    assert lib.coda_mx_quantize(A, 16, 128, 1, B, C, None) == DEVICE
     assert lib.coda_gemm_rowscale_partial_mx(A, B, C, D, None, 0, 0, 0.0, None, A, 16, 256, 256, None) == DEVICE
 
 

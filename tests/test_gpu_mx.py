@@ -42,12 +42,28 @@ def _gpu():
     C.load_library()
 
 
-def _exps(sf, R, K):
-    return MX.sf_untile(sf.cpu().numpy(), R, K)
+def _exps(sf, R, K, operand=0):
+    return MX.sf_untile(sf.cpu().numpy(), R, K, operand)
 
 
-@pytest.mark.parametrize("rows,cols", [(300, 384), (1, 128), (128, 256), (257, 1024)])
-def test_mx_quantize_bit_exact(rows, cols):
+def _check_sf_bytes(sf, exps, R, operand):
+    """The scale buffer byte for byte where the layout defines bytes
+    (bytes of an A image that no scale maps to are never read)."""
+    want, used = MX.sf_tile(exps, R, operand)
+    got = sf.cpu().numpy()
+    assert got.shape == want.shape
+    np.testing.assert_array_equal(got[used], want[used])
+
+
+def _same_sf(a, b, R, K, operand=0):
+    """Two scale buffers equal where the layout defines bytes."""
+    used = MX.sf_tile(np.zeros((R, K // 32), dtype=np.int64), R, operand)[1]
+    return bool(np.array_equal(a.cpu().numpy()[used], b.cpu().numpy()[used]))
+
+
+@pytest.mark.parametrize("rows,cols,operand", [(300, 384, 0), (300, 384, 1), (1, 128, 0), (1, 128, 1),
+                                               (128, 256, 1), (257, 1152, 0), (257, 1024, 1)])
+def test_mx_quantize_bit_exact(rows, cols, operand):
     g = synth.make_gen(1200 + rows + cols)
     t = synth.normal_bf16(g, (rows, cols), std=1.0).float()
     mag = torch.exp2(torch.randint(-24, 24, (rows, 1), generator=g).float())
@@ -57,11 +73,11 @@ def test_mx_quantize_bit_exact(rows, cols):
     if rows > 1:
         t[1, :32] = 0.0
         t[1, :2] = torch.tensor([448.0, -3.5])          # exactly at the boundary: scale 1
-    q, sf = C.mx_quantize(dev(t))
+    q, sf = C.mx_quantize(dev(t), operand)
     C.poll_status()
     wq, we = MX.mx_quantize(O.bf16_to_f64(b(t)))
     np.testing.assert_array_equal(q.cpu().numpy(), wq)
-    np.testing.assert_array_equal(sf.cpu().numpy(), MX.sf_tile(we, rows))
+    _check_sf_bytes(sf, we, rows, operand)
     assert int(we[0, 1]) == 1 and (rows == 1 or int(we[1, 0]) == 0)
 
 
@@ -71,9 +87,9 @@ def _small_int_mx(rng, R, K, vals, erange):
     return codes, exps
 
 
-def _to_dev(codes, exps, R):
+def _to_dev(codes, exps, R, operand):
     return (torch.from_numpy(np.ascontiguousarray(codes)).cuda(),
-            torch.from_numpy(MX.sf_tile(exps, R)).cuda())
+            torch.from_numpy(MX.sf_tile(exps, R, operand)[0]).cuda())
 
 
 @pytest.mark.parametrize("M,N,K", [(300, 384, 512), (256, 256, 128), (77, 640, 256)])
@@ -87,8 +103,8 @@ def test_mx_gemm_exact_small_integers(M, N, K):
     vals = [0.0, 0.5, 1.0, -0.5, -1.0]
     aq, ae = _small_int_mx(rng, M, K, vals, (-2, 2))
     bq, be = _small_int_mx(rng, N, K, vals, (-2, 2))
-    A, Asf = _to_dev(aq, ae, M)
-    W, Wsf = _to_dev(bq, be, N)
+    A, Asf = _to_dev(aq, ae, M, 0)
+    W, Wsf = _to_dev(bq, be, N, 1)
     out, r = C.gemm_rowscale_partial_mx(A, Asf, W, Wsf)
     C.poll_status()
     assert r is None
@@ -101,13 +117,13 @@ def test_mx_gemm_with_folded_row_scale(M, N, K):
     g = synth.make_gen(1300 + M)
     a = synth.normal_bf16(g, (M, K), std=2.0)
     w = synth.normal_bf16(g, (N, K), std=0.05)
-    A, Asf = C.mx_quantize(dev(a))
-    W, Wsf = C.mx_quantize(dev(w))
+    A, Asf = C.mx_quantize(dev(a), C.MX_A)
+    W, Wsf = C.mx_quantize(dev(w), C.MX_B)
     T = 6
     partial = torch.rand((T, M), generator=g).mul(50.0).cuda()
     out, r = C.gemm_rowscale_partial_mx(A, Asf, W, Wsf, partial, 700, 1e-5)
     C.poll_status()
-    ref = MX.gemm_rowscale_partial_mx(A.cpu().numpy(), _exps(Asf, M, K), W.cpu().numpy(), _exps(Wsf, N, K),
+    ref = MX.gemm_rowscale_partial_mx(A.cpu().numpy(), _exps(Asf, M, K), W.cpu().numpy(), _exps(Wsf, N, K, 1),
                                       partial.double().cpu().numpy(), 700, 1e-5)
     check_rel("r", r, ref["r"], 1e-6)
     # random partials spread r over a decade, so the largest outputs sit far
@@ -123,7 +139,7 @@ def _mx_inputs(inp):
     W2t = dev(inp.W2.t().contiguous())
     x8, _, sx = C.fp8_quantize(xd)
     W1t8, _, sw1 = C.fp8_quantize(W1d, transpose=True)
-    W2q, W2sf = C.mx_quantize(W2t)
+    W2q, W2sf = C.mx_quantize(W2t, C.MX_B)
     vx = O.bf16_to_f64(b(inp.x))
     vw1 = O.bf16_to_f64(b(inp.W1)).T
     osx, osw1 = F8.quant_scale(np.abs(vx).max()), F8.quant_scale(np.abs(vw1).max())
@@ -134,7 +150,7 @@ def _mx_inputs(inp):
     np.testing.assert_array_equal(W1t8.cpu().numpy(), oW1)
     np.testing.assert_array_equal(W2q.cpu().numpy(), oW2q)
     N2, N = W2q.shape
-    np.testing.assert_array_equal(_exps(W2sf, N2, N), oW2e)
+    np.testing.assert_array_equal(_exps(W2sf, N2, N, 1), oW2e)
     assert np.float32(sx.item()) == osx and np.float32(sw1.item()) == osw1
     gpu = dict(x8=x8, sx=sx, W1t8=W1t8, sw1=sw1, W2q=W2q, W2sf=W2sf)
     ora = dict(x8=ox8, sx=float(osx), W1t8=oW1, sw1=float(osw1), W2q=oW2q, W2e=oW2e)
@@ -183,7 +199,7 @@ def test_mx_first_gemm_exact_small_integers():
     C.poll_status()
     ref = MX.gemm_res_partialrms_mx(x8, 1.0, w8, 1.0, res, gamma, tile_cols=C.partial_tile_width())
     np.testing.assert_array_equal(hq.cpu().numpy(), ref["hq"])
-    np.testing.assert_array_equal(hsf.cpu().numpy(), MX.sf_tile(ref["he"], M))
+    _check_sf_bytes(hsf, ref["he"], M, 0)
     check("h", h, ref["h"], strict=True)
     check("partial", part, ref["partial"], rel=1e-6)
 
@@ -219,8 +235,9 @@ def test_mx_block_small(shape):
     # a repeated call is bitwise identical
     again = C.gemm_rmsnorm_gemm_mx(gpu["x8"], gpu["sx"], gpu["W1t8"], gpu["sw1"], dev(inp.res), dev(inp.gamma),
                                    gpu["W2q"], gpu["W2sf"], inp.eps)
-    for k in ("out", "h", "hq", "hsf", "partial", "r"):
+    for k in ("out", "h", "hq", "partial", "r"):
         assert torch.equal(f[k], again[k]), k
+    assert _same_sf(f["hsf"], again["hsf"], M, N)
 
 
 def test_mx_block_tail_full_size_sampled_rows():
@@ -319,14 +336,14 @@ def test_mx_calls_stay_inside_their_buffers():
     gpu, _ = _mx_inputs(inp)
     W2t = dev(inp.W2.t().contiguous())
     q = _Guarded(N2 * N, torch.uint8, (N2, N))
-    sf = _Guarded(C.mx_sf_bytes(N2, N), torch.uint8)
-    assert lib.coda_mx_quantize(_p(W2t), N2, N, q.ptr(), sf.ptr(), _s()) == 0
+    sf = _Guarded(C.mx_sf_bytes(N2, N, C.MX_B), torch.uint8)
+    assert lib.coda_mx_quantize(_p(W2t), N2, N, C.MX_B, q.ptr(), sf.ptr(), _s()) == 0
     assert q.intact() and sf.intact()
     assert torch.equal(q.t, gpu["W2q"]) and torch.equal(sf.t, gpu["W2sf"])
     T = C.partial_cols(N)
     h = _Guarded(M * N, torch.bfloat16, (M, N))
     hq = _Guarded(M * N, torch.uint8, (M, N))
-    hsf = _Guarded(C.mx_sf_bytes(M, N), torch.uint8)
+    hsf = _Guarded(C.mx_sf_bytes(M, N, C.MX_A), torch.uint8)
     part = _Guarded(T * M, torch.float32, (T, M))
     res, gamma = dev(inp.res), dev(inp.gamma)
     assert lib.coda_gemm_res_partialrms_mx(_p(gpu["x8"]), _p(gpu["sx"]), _p(gpu["W1t8"]), _p(gpu["sw1"]), _p(res),
@@ -340,6 +357,7 @@ def test_mx_calls_stay_inside_their_buffers():
     assert out.intact() and r.intact()
     ref = C.gemm_rmsnorm_gemm_mx(gpu["x8"], gpu["sx"], gpu["W1t8"], gpu["sw1"], res, gamma, gpu["W2q"],
                                  gpu["W2sf"], inp.eps)
-    for k, g in (("h", h), ("hq", hq), ("hsf", hsf), ("partial", part), ("out", out), ("r", r)):
+    for k, g in (("h", h), ("hq", hq), ("partial", part), ("out", out), ("r", r)):
         assert torch.equal(g.t, ref[k]), k
+    assert _same_sf(hsf.t, ref["hsf"], M, N)
     C.poll_status()

@@ -116,24 +116,43 @@ def test_round_trip_of_representable_blocks():
 
 
 def test_sf_layout_offsets_by_hand():
-    # R = 300 rows: 3 row blocks; row 33, block 5: k-block 1, row block 0,
-    # lane 1, column 1 of the atom, byte 1 -> (1 * 3 + 0) * 512 + 16 + 4 + 1
-    assert MX.sf_offset(33, 5, 300) == 1536 + 21
+    # A layout, R = 300 (3 row blocks).  Row 33, block 5: k-block 1 (step 1),
+    # row block 0, lane 1, column 1 -> (1 * 3 + 0) * 512 + 16 + 4 + 1
+    assert MX.sf_offsets(33, 5, 300, 0) == [1536 + 21]
     # row 299 (row block 2, lane 11, column 1), block 0: 2 * 512 + 176 + 4
-    assert MX.sf_offset(299, 0, 300) == 1204
+    assert MX.sf_offsets(299, 0, 300, 0) == [1204]
     # row 127 (lane 31, column 3), block 7: (1 * 3) * 512 + 496 + 12 + 3
-    assert MX.sf_offset(127, 7, 300) == 1536 + 511
-    assert MX.sf_bytes(300, 256) == 2 * 3 * 512
+    assert MX.sf_offsets(127, 7, 300, 0) == [1536 + 511]
+    assert MX.sf_bytes(300, 256, 0) == 2 * 3 * 512
+    # B layout, R = 384 (2 tiles of 256 rows), K = 256 (2 k-blocks).  Row 300,
+    # block 6: k-block 1 (step 2), tile 1, atom 0 of the tile, lane 12, column
+    # (300 // 32) % 4 = 1 -> (1 * 2 + 1) * 4096 + 12 * 16 + 4 + 2, and its three
+    # copies 512 bytes apart
+    assert MX.sf_offsets(300, 6, 384, 1) == [12486, 12998, 13510, 14022]
+    # row 130, block 0: tile 0, atom 1 (rows 128-255), lane 2, column 0
+    assert MX.sf_offsets(130, 0, 384, 1) == [2080, 2592, 3104, 3616]
+    assert MX.sf_bytes(384, 256, 1) == 2 * 2 * 4096
+    assert MX.sf_bytes(300, 256, 1) == 2 * 2 * 4096  # 300 rows: two tiles, the second part padding
     rng = np.random.default_rng(9)
-    e = rng.integers(-30, 30, (300, 8))
-    buf = MX.sf_tile(e, 300)
-    assert np.array_equal(MX.sf_untile(buf, 300, 256), e)
-    used = np.zeros(buf.size, dtype=bool)
-    for i in range(300):
-        for j in range(8):
-            used[MX.sf_offset(i, j, 300)] = True
-    assert used.sum() == 300 * 8  # no two scales share a byte
-    assert np.all(buf[~used] == 127)  # padding rows: scale 1
+    for operand, R, K in ((0, 300, 256), (0, 1, 384), (1, 300, 256), (1, 128, 512)):
+        e = rng.integers(-30, 30, (R, K // 32))
+        buf, used = MX.sf_tile(e, R, operand)
+        assert np.array_equal(MX.sf_untile(buf, R, K, operand), e)
+        seen = np.zeros(buf.size, dtype=int)
+        for i in range(MX.sf_rows_padded(R, operand)):
+            for j in range(K // 32):
+                for o in MX.sf_offsets(i, j, R, operand):
+                    seen[o] += 1
+        assert seen.max() == 1  # no two scales (or copies) share a byte
+        assert np.array_equal(seen == 1, used)
+        pad = [o for i in range(R, MX.sf_rows_padded(R, operand)) for j in range(K // 32)
+               for o in MX.sf_offsets(i, j, R, operand)]
+        assert np.all(buf[pad] == 127)  # padding rows: scale 1
+        assert used.all()  # every byte belongs to a scale or a padding row
+        if operand == 1:  # four copies of each scale
+            for i in range(R):
+                for j in range(K // 32):
+                    assert len({int(buf[o]) for o in MX.sf_offsets(i, j, R, 1)}) == 1
 
 
 def _brute_gemm(aq, ae, bq, be):
