@@ -105,14 +105,40 @@ def load_peaks():
     return 1590.0, 1400.0, 6650.0, "fallback"
 
 
+def strip_comments(src: str) -> str:
+    """C++ source without its // and /* */ comments (string and character
+    literals kept as they are; line breaks kept)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            out.append("\n" * src.count("\n", i, n if j < 0 else j))
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return "".join(out)
+
+
 def source_hash():
-    """Hash of the device code (the .cuh kernel headers); a recorded ncu traffic
-    figure is reported only while the kernels it was measured on are unchanged."""
+    """Hash of the device code (the .cuh kernel headers, comments removed); a
+    recorded ncu traffic figure is reported only while the kernels it was
+    measured on are unchanged."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gemm_epilogue_transformer_02_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
         if f.endswith(".cuh"):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+            h.update(strip_comments(open(os.path.join(csrc, f)).read()).encode())
     return h.hexdigest()[:16]
 
 

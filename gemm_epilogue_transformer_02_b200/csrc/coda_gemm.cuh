@@ -1083,10 +1083,10 @@ struct EpiRowScaleF8 : EpiRowScale {
 // the light reduction folded in as in the bf16 block.  The tile has the only
 // accumulator, so the epilogue first reads all of it into registers (bf16
 // pairs, 128 per thread), releases it to the MMA, and only then stores the
-// tile, chunk by chunk through one staging buffer: with one 4 KB buffer per
-// warp the mainloop keeps a sixth pipeline stage (261.9 against 266.5 us with
-// two buffers, five stages and half of the tile staged before the release,
-// on the 1B block's second GEMM).
+// tile, chunk by chunk through one staging buffer: one 4 KB buffer per warp
+// leaves the mainloop a stage more (261.9 against 266.5 us with two buffers
+// and half of the tile staged before the release, both with three scale
+// copies per k-block, on the 1B block's second GEMM).
 struct EpiRowScaleMX : EpiRowScale {
   static constexpr int kSmemPerWarp = 4096;
   static constexpr bool kFp8 = true;

@@ -41,3 +41,19 @@ def test_hbm_row_and_clock_cycles():
     assert math.isclose(r["kcycles"], 0.025 * 1500.0)          # ms x MHz = thousands of cycles
     assert r["reasons"] == ["sw_power_cap"] and r["note"] == "note"
     assert r["ms_median"] == 0.03 and r["ms_min"] == 0.02
+
+
+def test_device_code_hash_ignores_comments_only():
+    src = '''// a comment with "quotes" and 'ticks'
+    asm volatile("mov.u64 %0, %%globaltimer; // not a comment" : "=l"(t));  /* block
+    comment */ x = '/'; y = "a\\"b//c";
+'''
+    got = bench.strip_comments(src)
+    assert got.count("\n") == src.count("\n")
+    assert '"mov.u64 %0, %%globaltimer; // not a comment"' in got
+    assert "'/'" in got and '"a\\"b//c"' in got
+    assert "comment with" not in got and "block" not in got
+    # the same code with other comments strips to the same text
+    other = src.replace("a comment with", "another remark,").replace("block\n    comment", "x\n    y")
+    assert bench.strip_comments(other) == got
+    assert bench.strip_comments(src.replace("x = '/'", "x = '+'")) != got
